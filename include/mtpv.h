@@ -1,0 +1,234 @@
+/*
+ * mtpv.h -- C ABI of libmtpv, the speculative-decoding verify step on NVIDIA
+ * B200 (sm_100a).
+ *
+ * The verify step is the part of self-speculative (multi-token-prediction)
+ * decoding that runs after the model's own MTP head has drafted K tokens:
+ *   1. a small-M projection of the hidden states through the LM head: K+1
+ *      target rows through the bf16 head and K draft rows through a
+ *      group-64 int4 copy of the same head (hazakura.dev MTPLX notes,
+ *      "4-layer architecture", Layer 0: small-matrix (M=3..6) shader and the
+ *      draft-only 4-bit LM head that keeps the target's own precision);
+ *   2. Leviathan-Chen rejection sampling with residual correction and a bonus
+ *      token (devtrends.cc MTPLX overview, "no second model" section;
+ *      hazakura.dev notes, Layer 2: draft -> parallel verify -> ratio
+ *      acceptance -> residual correction -> bonus token), with temperature
+ *      and top-p applied so that the output distribution equals plain
+ *      sampling at those settings (devtrends.cc overview: temperature=0.6,
+ *      top_p=0.95).
+ *
+ * Conventions shared by every call
+ *   - All tensors are dense, row-major and owned by the caller.  Device
+ *     pointers must be 16-byte aligned unless stated otherwise.
+ *   - The library never allocates device memory and never synchronises the
+ *     stream (except mtpv_verify_step_host, which is synchronous by design).
+ *     Scratch memory is the caller's workspace; its size comes from the
+ *     matching *_workspace_bytes query.  A workspace may be reused by later
+ *     calls on the same stream but not by calls that overlap in time.
+ *   - Every compute call is asynchronous on `stream` (NULL = legacy default
+ *     stream).  Argument errors are returned synchronously and nothing is
+ *     launched.  A launch failure returns MTPV_ERR_CUDA.
+ *   - Errors in the DATA (a draft id outside [0, V), a non-finite logit) are
+ *     reported per sequence in row_status; they never fault the GPU.
+ *   - The caller supplies every uniform random number (fp32 in [0, 1)); the
+ *     library holds no random-number generator.
+ *   - The calling thread's current CUDA context must be the one that owns
+ *     the pointers (the primary context of the device, as PyTorch sets it).
+ */
+#ifndef MTPV_H_
+#define MTPV_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MTPV_API __attribute__((visibility("default")))
+#else
+#define MTPV_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t / CUstream. */
+typedef struct CUstream_st *mtpv_stream;
+
+typedef enum {
+    MTPV_OK = 0,
+    MTPV_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or parameter   */
+    MTPV_ERR_UNSUPPORTED = 2, /* valid request this build does not handle    */
+    MTPV_ERR_WORKSPACE = 3,   /* workspace missing or smaller than required  */
+    MTPV_ERR_CUDA = 4,        /* a CUDA call or kernel launch failed         */
+    MTPV_ERR_TIMEOUT = 5      /* a bounded device-side wait gave up          */
+} mtpv_status;
+
+/* Weight storage formats of mtpv_lm_head_smallm. */
+typedef enum {
+    MTPV_W_BF16 = 0,     /* w: bf16 [N, Kd]; scales unused (NULL)             */
+    MTPV_W_INT4_G64 = 1  /* w: uint8 [N, Kd/2], scales: bf16 [N, Kd/64]       */
+} mtpv_wfmt;
+
+/* Per-sequence data status written to row_status. */
+#define MTPV_ROW_OK 0
+#define MTPV_ROW_BAD_DRAFT 1    /* a draft token id outside [0, V)          */
+#define MTPV_ROW_NONFINITE 2    /* a NaN or +-inf logit in one of its rows  */
+
+/* Library version: major*10000 + minor*100 + patch. */
+MTPV_API int mtpv_version(void);
+
+/* Static, human-readable name of a status code (never NULL). */
+MTPV_API const char *mtpv_status_string(mtpv_status st);
+
+/* ------------------------------------------------------------------------
+ * mtpv_lm_head_smallm -- small-M weight-streaming projection.
+ *
+ * Passage: hazakura.dev MTPLX notes, Layer 0 (a matmul specialised for M=3..6
+ * rows; a 4-bit LM head used for drafting while the target keeps its own
+ * precision); gist.science BaseRT explainer, methodology (decode GEMV per
+ * quantisation format with dequantisation inside the inner loop).
+ *
+ *   y[m][n] = sum_k x[m][k] * Wd[n][k],  0 <= m < M, 0 <= n < N   (fp32 out)
+ *
+ *   x       device, bf16 [M, Kd] row-major (activations / hidden states).
+ *   M       rows, 1 <= M <= 64.  The kernel is built for M <= 8; larger M is
+ *           processed in groups of 8 rows (the weights are re-read per group).
+ *   Kd      reduction length, a positive multiple of 64.
+ *   N       output columns (vocabulary rows of the head), N >= 1.
+ *   w       device weights, layout per fmt:
+ *             MTPV_W_BF16:     bf16 [N, Kd] (nn.Linear out x in layout);
+ *                              Wd = w.
+ *             MTPV_W_INT4_G64: uint8 [N, Kd/2]; weight k of row n is the low
+ *                              nibble of byte k/2 when k is even, the high
+ *                              nibble when k is odd; the nibble stores q+8
+ *                              for q in [-8, 7];
+ *                              Wd[n][k] = scales[n][k/64] * (nibble - 8).
+ *   scales  device bf16 [N, Kd/64] for MTPV_W_INT4_G64 (2-byte aligned);
+ *           ignored for MTPV_W_BF16.
+ *   y       device fp32 [M, N] row-major, fully overwritten (4-byte aligned).
+ *   ws, ws_bytes  workspace (may be NULL when the query returns 0).
+ * Accumulation is fp32.  Errors: MTPV_ERR_INVALID_ARG for NULL pointers,
+ * M/Kd/N out of range or misaligned x/w; MTPV_ERR_WORKSPACE when ws_bytes is
+ * below mtpv_lm_head_workspace_bytes().
+ * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_lm_head_workspace_bytes(int M, int Kd, int N, mtpv_wfmt fmt);
+MTPV_API mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, const void *w,
+                                const void *scales, mtpv_wfmt fmt, float *y, void *ws,
+                                size_t ws_bytes, mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
+ * mtpv_verify -- Leviathan-Chen verification of B independent sequences.
+ *
+ * Passages: devtrends.cc MTPLX overview and devtrends.ru page (exact rejection
+ * sampling of Leviathan and Chen with residual correction; temperature 0.6 /
+ * top_p 0.95 reproduce non-speculative sampling); hazakura.dev notes,
+ * Layer 2 (ratio acceptance, residual correction, bonus token) and results
+ * section (distribution identical, max_diff = 0.0; not greedy-only).
+ *
+ * Every row l (target or draft) is warped the same way:
+ *   T > 0:  p_j = exp((l_j - max l)/T) / sum_i exp((l_i - max l)/T); tokens
+ *           are ranked by (logit desc, index asc); rank r is kept iff the mass
+ *           of the ranks before it is < top_p (top_p >= 1 keeps every token
+ *           with p > 0); p'_j = p_j / (kept mass) for kept tokens, else 0.
+ *   T == 0: p' is one-hot at the argmax (lowest index among equal maxima).
+ * For sequence b with drafts d_0..d_{K-1} (p'_i from target row i, q'_i from
+ * draft row i):
+ *   accept d_i iff u_accept[b][i] < p'_i(d_i) / q'_i(d_i)
+ *   (+inf when q'_i(d_i) == 0 < p'_i(d_i), 0 when both are 0); n = number of
+ *   drafts accepted before the first rejection (K if none);
+ *   n < K:  x ~ normalise(max(0, p'_n - q'_n))  (p'_n if that is all zero);
+ *   n == K: x ~ p'_K (the bonus token);
+ *   the draw is the inverse CDF in vocabulary order with u = u_sample[b][n]:
+ *   x = min{k : sum_{j<=k} w_j > u * sum_j w_j}.
+ *   Outputs: out_tokens[b] = d_0..d_{n-1}, x, then -1 up to K+1 entries;
+ *   out_accepted[b] = n.
+ *
+ *   target_logits  device fp32 [B, K+1, V] (4-byte aligned)
+ *   draft_logits   device fp32 [B, K, V]
+ *   draft_tokens   device int32 [B, K]
+ *   u_accept       device fp32 [B, K], values in [0, 1)
+ *   u_sample       device fp32 [B, K+1], values in [0, 1)
+ *   B >= 1, 1 <= K <= 16, 1 <= V <= 2^24 (B*(2K+1) <= 65535)
+ *   temperature    >= 0 and finite; top_p in (0, 1] (values above 1 mean 1).
+ *   out_tokens     device int32 [B, K+1];  out_accepted device int32 [B]
+ *   row_status     device int32 [B] or NULL; MTPV_ROW_* per sequence.  A
+ *                  sequence with a data error gets out_accepted = -1 and
+ *                  out_tokens all -1.
+ *   ws, ws_bytes   workspace of at least mtpv_verify_workspace_bytes(B, K, V)
+ *                  bytes, 256-byte aligned.  It need not be initialised: the
+ *                  call clears what it needs on `stream` before the kernel.
+ * Arithmetic: exp, sums, ratios and CDFs in fp64 on fp32 logits.
+ * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_verify_workspace_bytes(int B, int K, int V);
+MTPV_API mtpv_status mtpv_verify(const float *target_logits, const float *draft_logits,
+                        const int32_t *draft_tokens, const float *u_accept,
+                        const float *u_sample, int B, int K, int V, float temperature,
+                        float top_p, int32_t *out_tokens, int32_t *out_accepted,
+                        int32_t *row_status, void *ws, size_t ws_bytes, mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
+ * mtpv_sample -- one draw from the warped distribution of each of R rows
+ * (temperature + top-p exactly as in mtpv_verify, inverse CDF with u[r]).
+ * This is the draft phase's own sampling step (hazakura.dev notes, Layer 2
+ * "Draft"), used to draw draft tokens from q'.
+ *
+ *   logits     device fp32 [R, V];  u device fp32 [R] in [0, 1)
+ *   out        device int32 [R] (-1 for a row with a non-finite logit)
+ *   row_status device int32 [R] or NULL (MTPV_ROW_OK / MTPV_ROW_NONFINITE)
+ *   1 <= R <= 65535, 1 <= V <= 2^24; ws as returned by the query.
+ * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_sample_workspace_bytes(int R, int V);
+MTPV_API mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, float top_p,
+                        const float *u, int32_t *out, int32_t *row_status, void *ws,
+                        size_t ws_bytes, mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
+ * mtpv_verify_step -- the whole verify step for B sequences in one call:
+ * target logits of the B*(K+1) target rows through the bf16 head, draft
+ * logits of the B*K draft rows through the int4 group-64 head, then
+ * mtpv_verify.  (Passages: those of mtpv_lm_head_smallm and mtpv_verify; the
+ * devtrends.cc overview's single forward pass that verifies the whole draft.)
+ *
+ *   w_target        device bf16 [V, h]
+ *   w_draft, s_draft device uint8 [V, h/2] and bf16 [V, h/64] (int4 g64)
+ *   h_target        device bf16 [B*(K+1), h]: row b*(K+1)+i is position i of
+ *                   sequence b
+ *   h_draft         device bf16 [B*K, h]: row b*K+i is draft position i
+ *   draft_tokens, u_accept, u_sample, temperature, top_p, out_*: as in
+ *                   mtpv_verify.
+ *   target_logits, draft_logits  device fp32 [B, K+1, V] / [B, K, V] outputs,
+ *                   or NULL to keep them inside the workspace.
+ *   h a positive multiple of 64; B*(K+1) <= 64; other limits as above.
+ *   ws of at least mtpv_verify_step_workspace_bytes(B, K, V, h) bytes.
+ * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_verify_step_workspace_bytes(int B, int K, int V, int h);
+MTPV_API mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const void *s_draft,
+                             const void *h_target, const void *h_draft,
+                             const int32_t *draft_tokens, const float *u_accept,
+                             const float *u_sample, int B, int K, int V, int h,
+                             float temperature, float top_p, int32_t *out_tokens,
+                             int32_t *out_accepted, int32_t *row_status, float *target_logits,
+                             float *draft_logits, void *ws, size_t ws_bytes, mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
+ * mtpv_verify_step_host -- mtpv_verify_step with the per-step inputs and
+ * outputs in HOST memory: h_target, h_draft, draft_tokens, u_accept, u_sample
+ * are copied host->device, out_tokens / out_accepted / row_status (row_status
+ * may be NULL) device->host, all on `stream`, and the call returns after the
+ * stream has drained.  Weights and ws stay on the device.  Page-locked host
+ * buffers give asynchronous copies; pageable ones work but are slower.
+ * ws of at least mtpv_verify_step_host_workspace_bytes(B, K, V, h) bytes.
+ * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_verify_step_host_workspace_bytes(int B, int K, int V, int h);
+MTPV_API mtpv_status mtpv_verify_step_host(const void *w_target, const void *w_draft, const void *s_draft,
+                                  const void *h_target_host, const void *h_draft_host,
+                                  const int32_t *draft_tokens_host, const float *u_accept_host,
+                                  const float *u_sample_host, int B, int K, int V, int h,
+                                  float temperature, float top_p, int32_t *out_tokens_host,
+                                  int32_t *out_accepted_host, int32_t *row_status_host, void *ws,
+                                  size_t ws_bytes, mtpv_stream stream);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MTPV_H_ */

@@ -1,0 +1,286 @@
+// extern "C" entry points of libmtpv: argument checks, workspace layout and
+// kernel launches.  Semantics and citations are in include/mtpv.h.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "lm_head.cuh"
+#include "sampler.cuh"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMaxK = 16;
+constexpr int kMaxV = 1 << 24;
+constexpr int kMaxRows = 65535;
+
+size_t up(size_t n) { return (n + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned(const void *p, size_t a) { return ((uintptr_t)p % a) == 0; }
+
+mtpv_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return MTPV_OK;
+    cudaGetLastError();  // clear a sticky launch error so later calls can proceed
+    return MTPV_ERR_CUDA;
+}
+
+// --- workspace layouts -----------------------------------------------------
+struct VerifyWs {
+    size_t counters, stats, total;
+};
+VerifyWs verify_layout(int B, int K) {
+    VerifyWs l;
+    l.counters = 0;
+    l.stats = up(sizeof(unsigned int) * (size_t)B);
+    l.total = l.stats + up(sizeof(mtpv::RowStats) * (size_t)B * (2 * K + 1));
+    return l;
+}
+
+struct StepWs {
+    size_t tl, dl, verify, total;
+};
+StepWs step_layout(int B, int K, int V) {
+    StepWs l;
+    l.tl = 0;
+    l.dl = l.tl + up(sizeof(float) * (size_t)B * (K + 1) * V);
+    l.verify = l.dl + up(sizeof(float) * (size_t)B * K * V);
+    l.total = l.verify + verify_layout(B, K).total;
+    return l;
+}
+
+struct HostWs {
+    size_t step, ht, hd, drafts, ua, us, tok, acc, rs, total;
+};
+HostWs host_layout(int B, int K, int V, int h) {
+    HostWs l;
+    l.step = 0;
+    l.ht = step_layout(B, K, V).total;
+    l.hd = l.ht + up((size_t)B * (K + 1) * h * 2);
+    l.drafts = l.hd + up((size_t)B * K * h * 2);
+    l.ua = l.drafts + up(sizeof(int32_t) * (size_t)B * K);
+    l.us = l.ua + up(sizeof(float) * (size_t)B * K);
+    l.tok = l.us + up(sizeof(float) * (size_t)B * (K + 1));
+    l.acc = l.tok + up(sizeof(int32_t) * (size_t)B * (K + 1));
+    l.rs = l.acc + up(sizeof(int32_t) * (size_t)B);
+    l.total = l.rs + up(sizeof(int32_t) * (size_t)B);
+    return l;
+}
+
+bool verify_shape_ok(int B, int K, int V) {
+    return B >= 1 && K >= 1 && K <= kMaxK && V >= 1 && V <= kMaxV &&
+           (long long)B * (2 * K + 1) <= kMaxRows;
+}
+
+bool sampling_params_ok(float T, float top_p) {
+    return isfinite(T) && T >= 0.0f && !isnan(top_p) && top_p > 0.0f;
+}
+
+bool lm_head_shape_ok(int M, int Kd, int N) {
+    return M >= 1 && M <= 64 && Kd >= 64 && Kd % 64 == 0 && N >= 1 &&
+           mtpv::lm_head_max_smem_rows(Kd) >= 1;
+}
+
+char *at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
+
+mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *drafts, const float *ua,
+                          const float *us, int B, int K, int V, float T, float top_p,
+                          int32_t *out_tokens, int32_t *out_acc, int32_t *row_status, void *ws,
+                          cudaStream_t s) {
+    const VerifyWs l = verify_layout(B, K);
+    unsigned int *counters = reinterpret_cast<unsigned int *>(at(ws, l.counters));
+    cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(unsigned int) * (size_t)B, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    mtpv::SamplerParams p;
+    p.tl = tl;
+    p.dl = dl;
+    p.drafts = drafts;
+    p.u_acc = ua;
+    p.u_samp = us;
+    p.B = B;
+    p.K = K;
+    p.V = V;
+    p.T = T;
+    p.top_p = top_p;
+    p.verify = 1;
+    p.out_tokens = out_tokens;
+    p.out_acc = out_acc;
+    p.row_status = row_status;
+    p.stats = reinterpret_cast<mtpv::RowStats *>(at(ws, l.stats));
+    p.counters = counters;
+    return cuda_status(mtpv::launch_sampler(p, B * (2 * K + 1), s));
+}
+
+}  // namespace
+
+extern "C" {
+
+int mtpv_version(void) { return 100; }
+
+const char *mtpv_status_string(mtpv_status st) {
+    switch (st) {
+        case MTPV_OK: return "ok";
+        case MTPV_ERR_INVALID_ARG: return "invalid argument";
+        case MTPV_ERR_UNSUPPORTED: return "unsupported";
+        case MTPV_ERR_WORKSPACE: return "workspace missing or too small";
+        case MTPV_ERR_CUDA: return "CUDA error";
+        case MTPV_ERR_TIMEOUT: return "device wait timed out";
+    }
+    return "unknown status";
+}
+
+size_t mtpv_lm_head_workspace_bytes(int M, int Kd, int N, mtpv_wfmt fmt) {
+    (void)M; (void)Kd; (void)N; (void)fmt;
+    return 0;
+}
+
+mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, const void *w,
+                                const void *scales, mtpv_wfmt fmt, float *y, void *ws,
+                                size_t ws_bytes, mtpv_stream stream) {
+    (void)ws; (void)ws_bytes;
+    if (!x || !w || !y || !lm_head_shape_ok(M, Kd, N)) return MTPV_ERR_INVALID_ARG;
+    if (fmt != MTPV_W_BF16 && fmt != MTPV_W_INT4_G64) return MTPV_ERR_INVALID_ARG;
+    if (fmt == MTPV_W_INT4_G64 && (!scales || !aligned(scales, 2))) return MTPV_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 4)) return MTPV_ERR_INVALID_ARG;
+    return cuda_status(mtpv::launch_lm_head(x, M, Kd, N, w, scales, (int)fmt, y, (cudaStream_t)stream));
+}
+
+size_t mtpv_verify_workspace_bytes(int B, int K, int V) {
+    if (!verify_shape_ok(B, K, V)) return 0;
+    return verify_layout(B, K).total;
+}
+
+mtpv_status mtpv_verify(const float *target_logits, const float *draft_logits,
+                        const int32_t *draft_tokens, const float *u_accept, const float *u_sample,
+                        int B, int K, int V, float temperature, float top_p, int32_t *out_tokens,
+                        int32_t *out_accepted, int32_t *row_status, void *ws, size_t ws_bytes,
+                        mtpv_stream stream) {
+    if (!target_logits || !draft_logits || !draft_tokens || !u_accept || !u_sample || !out_tokens ||
+        !out_accepted)
+        return MTPV_ERR_INVALID_ARG;
+    if (!verify_shape_ok(B, K, V) || !sampling_params_ok(temperature, top_p))
+        return MTPV_ERR_INVALID_ARG;
+    if (!aligned(target_logits, 4) || !aligned(draft_logits, 4)) return MTPV_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < verify_layout(B, K).total) return MTPV_ERR_WORKSPACE;
+    return launch_verify(target_logits, draft_logits, draft_tokens, u_accept, u_sample, B, K, V,
+                         temperature, top_p, out_tokens, out_accepted, row_status, ws,
+                         (cudaStream_t)stream);
+}
+
+size_t mtpv_sample_workspace_bytes(int R, int V) {
+    if (R < 1 || R > kMaxRows || V < 1 || V > kMaxV) return 0;
+    return up(sizeof(mtpv::RowStats) * (size_t)R);
+}
+
+mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, float top_p,
+                        const float *u, int32_t *out, int32_t *row_status, void *ws,
+                        size_t ws_bytes, mtpv_stream stream) {
+    if (!logits || !u || !out) return MTPV_ERR_INVALID_ARG;
+    if (R < 1 || R > kMaxRows || V < 1 || V > kMaxV || !sampling_params_ok(temperature, top_p))
+        return MTPV_ERR_INVALID_ARG;
+    if (!aligned(logits, 4)) return MTPV_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < mtpv_sample_workspace_bytes(R, V))
+        return MTPV_ERR_WORKSPACE;
+    mtpv::SamplerParams p = {};
+    p.tl = logits;
+    p.dl = nullptr;
+    p.u_samp = u;
+    p.B = R;
+    p.K = 0;
+    p.V = V;
+    p.T = temperature;
+    p.top_p = top_p;
+    p.verify = 0;
+    p.out_tokens = out;
+    p.row_status = row_status;
+    p.stats = reinterpret_cast<mtpv::RowStats *>(ws);
+    p.counters = nullptr;
+    return cuda_status(mtpv::launch_sampler(p, R, (cudaStream_t)stream));
+}
+
+size_t mtpv_verify_step_workspace_bytes(int B, int K, int V, int h) {
+    if (!verify_shape_ok(B, K, V) || B * (K + 1) > 64 || h < 64 || h % 64) return 0;
+    return step_layout(B, K, V).total;
+}
+
+mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const void *s_draft,
+                             const void *h_target, const void *h_draft,
+                             const int32_t *draft_tokens, const float *u_accept,
+                             const float *u_sample, int B, int K, int V, int h, float temperature,
+                             float top_p, int32_t *out_tokens, int32_t *out_accepted,
+                             int32_t *row_status, float *target_logits, float *draft_logits,
+                             void *ws, size_t ws_bytes, mtpv_stream stream) {
+    if (!w_target || !w_draft || !s_draft || !h_target || !h_draft || !draft_tokens || !u_accept ||
+        !u_sample || !out_tokens || !out_accepted)
+        return MTPV_ERR_INVALID_ARG;
+    if (!verify_shape_ok(B, K, V) || B * (K + 1) > 64 || !lm_head_shape_ok(B * (K + 1), h, V) ||
+        !sampling_params_ok(temperature, top_p))
+        return MTPV_ERR_INVALID_ARG;
+    if (!aligned(w_target, 16) || !aligned(w_draft, 16) || !aligned(s_draft, 2) ||
+        !aligned(h_target, 16) || !aligned(h_draft, 16))
+        return MTPV_ERR_INVALID_ARG;
+    if ((target_logits && !aligned(target_logits, 4)) || (draft_logits && !aligned(draft_logits, 4)))
+        return MTPV_ERR_INVALID_ARG;
+    const StepWs l = step_layout(B, K, V);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MTPV_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    float *tl = target_logits ? target_logits : reinterpret_cast<float *>(at(ws, l.tl));
+    float *dl = draft_logits ? draft_logits : reinterpret_cast<float *>(at(ws, l.dl));
+    cudaError_t e = mtpv::launch_lm_head(h_target, B * (K + 1), h, V, w_target, nullptr, MTPV_W_BF16, tl, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    e = mtpv::launch_lm_head(h_draft, B * K, h, V, w_draft, s_draft, MTPV_W_INT4_G64, dl, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    return launch_verify(tl, dl, draft_tokens, u_accept, u_sample, B, K, V, temperature, top_p,
+                         out_tokens, out_accepted, row_status, at(ws, l.verify), s);
+}
+
+size_t mtpv_verify_step_host_workspace_bytes(int B, int K, int V, int h) {
+    if (mtpv_verify_step_workspace_bytes(B, K, V, h) == 0) return 0;
+    return host_layout(B, K, V, h).total;
+}
+
+mtpv_status mtpv_verify_step_host(const void *w_target, const void *w_draft, const void *s_draft,
+                                  const void *h_target_host, const void *h_draft_host,
+                                  const int32_t *draft_tokens_host, const float *u_accept_host,
+                                  const float *u_sample_host, int B, int K, int V, int h,
+                                  float temperature, float top_p, int32_t *out_tokens_host,
+                                  int32_t *out_accepted_host, int32_t *row_status_host, void *ws,
+                                  size_t ws_bytes, mtpv_stream stream) {
+    if (!h_target_host || !h_draft_host || !draft_tokens_host || !u_accept_host || !u_sample_host ||
+        !out_tokens_host || !out_accepted_host)
+        return MTPV_ERR_INVALID_ARG;
+    if (mtpv_verify_step_workspace_bytes(B, K, V, h) == 0) return MTPV_ERR_INVALID_ARG;
+    const HostWs l = host_layout(B, K, V, h);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MTPV_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const size_t nt = (size_t)B * (K + 1), nd = (size_t)B * K;
+    struct Copy { void *dst; const void *src; size_t bytes; };
+    const Copy in[] = {
+        {at(ws, l.ht), h_target_host, nt * h * 2},
+        {at(ws, l.hd), h_draft_host, nd * h * 2},
+        {at(ws, l.drafts), draft_tokens_host, nd * sizeof(int32_t)},
+        {at(ws, l.ua), u_accept_host, nd * sizeof(float)},
+        {at(ws, l.us), u_sample_host, nt * sizeof(float)},
+    };
+    for (const Copy &c : in) {
+        cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
+    int32_t *tok = reinterpret_cast<int32_t *>(at(ws, l.tok));
+    int32_t *acc = reinterpret_cast<int32_t *>(at(ws, l.acc));
+    int32_t *rs = reinterpret_cast<int32_t *>(at(ws, l.rs));
+    mtpv_status st = mtpv_verify_step(
+        w_target, w_draft, s_draft, at(ws, l.ht), at(ws, l.hd),
+        reinterpret_cast<const int32_t *>(at(ws, l.drafts)), reinterpret_cast<const float *>(at(ws, l.ua)),
+        reinterpret_cast<const float *>(at(ws, l.us)), B, K, V, h, temperature, top_p, tok, acc, rs,
+        nullptr, nullptr, at(ws, l.step), l.ht, stream);
+    if (st != MTPV_OK) return st;
+    cudaError_t e = cudaMemcpyAsync(out_tokens_host, tok, nt * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(out_accepted_host, acc, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess && row_status_host)
+        e = cudaMemcpyAsync(row_status_host, rs, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    return cuda_status(e);
+}
+
+}  // extern "C"
