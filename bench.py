@@ -1,0 +1,418 @@
+"""Benchmark of the speculative-decoding verify step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+                    [--impl {mtpv,reference}] [--no-cpu-baseline] [--no-e2e]
+
+One step = the whole verify step of one batch: the K+1 target rows through
+the bf16 LM head, the K draft rows through the int4 group-64 head, and the
+Leviathan-Chen verification (acceptance, residual / bonus draw).  Inputs are
+seeded synthetic tensors with the shapes of a Qwen-class 27B model (hidden
+5120, vocabulary 151936; random-init heads W ~ N(0, 0.02^2)), resident in HBM
+before timing.  The heads (1.98 GB per step) are far larger than L2, so every
+step streams them from HBM.
+
+Multi-GPU: the verify step does not shard; N ranks run N independent
+replicas (weak scaling) and the time is the max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from verify_step_lm_b200 import synth  # noqa: E402
+
+CONFIGS = {
+    # name: B, K, V, h, T, top_p, draft noise sigma, head std
+    "qwen27b": dict(B=1, K=3, V=151936, h=5120, T=0.6, top_p=0.95, sigma=0.3, wstd=0.02),
+    "qwen27b_k1": dict(B=1, K=1, V=151936, h=5120, T=0.6, top_p=0.95, sigma=0.3, wstd=0.02),
+    "qwen27b_k2": dict(B=1, K=2, V=151936, h=5120, T=0.6, top_p=0.95, sigma=0.3, wstd=0.02),
+    "qwen27b_greedy": dict(B=1, K=3, V=151936, h=5120, T=0.0, top_p=0.95, sigma=0.3, wstd=0.02),
+    "b8_v248k": dict(B=8, K=3, V=248320, h=5120, T=0.6, top_p=0.95, sigma=0.3, wstd=0.02),
+    "tiny": dict(B=1, K=3, V=4096, h=512, T=0.6, top_p=0.95, sigma=0.3, wstd=0.05),
+}
+POOL = 64
+METRIC = "verify steps/s (K=3, V=151936, h=5120) and achieved HBM GB/s vs roofline"
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def workload_name(c):
+    return (f"verify step B={c['B']} K={c['K']} hidden={c['h']} vocab={c['V']}: bf16 target head + "
+            f"int4 g64 draft head + Leviathan-Chen sampler, T={c['T']}, top_p={c['top_p']}")
+
+
+def step_bytes(c):
+    """Algorithmic HBM bytes of one step: both heads once, hidden states, the
+    fp32 logits written by the heads and read once by the sampler."""
+    B, K, V, h = c["B"], c["K"], c["V"], c["h"]
+    Mt, Md = B * (K + 1), B * K
+    w_bf16 = V * h * 2
+    w_int4 = V * h // 2 + V * (h // 64) * 2
+    hidden = (Mt + Md) * h * 2
+    logits = (Mt + Md) * V * 4
+    return {"w_bf16": w_bf16, "w_int4": w_int4, "hidden": hidden, "logits_rw": 2 * logits,
+            "bf16_launch": w_bf16 + Mt * h * 2 + Mt * V * 4,
+            "int4_launch": w_int4 + Md * h * 2 + Md * V * 4,
+            "sampler_launch": logits,
+            "total": w_bf16 + w_int4 + hidden + 2 * logits}
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        rows = []
+        try:
+            for line in open(self.path):
+                f = [x.strip() for x in line.split(",")]
+                if len(f) >= 9 and f[1].replace(".", "").isdigit():
+                    rows.append(f)
+        except Exception:
+            pass
+        finally:
+            try:
+                os.unlink(self.path)
+            except Exception:
+                pass
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": float(rows[0][2]),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w_max": max(float(r[3]) for r in rows if r[3].replace(".", "").isdigit())}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (baseline / reference arm)
+# ---------------------------------------------------------------------------
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def oracle_steps(c, seconds: float, min_steps: int, max_steps: int, heads=None):
+    """Time the CPU oracle on whole verify steps of workload c (host cores).
+
+    ``heads`` = (W, Wq, S) CPU tensors to reuse; generated here otherwise.
+    """
+    import oracle  # test infrastructure: used here only for the CPU baseline
+
+    B, K, V, h = c["B"], c["K"], c["V"], c["h"]
+    T32, P32 = float(np.float32(c["T"])), float(np.float32(c["top_p"]))
+    cores = host_cores()
+    if heads is None:
+        W = synth.make_head(V, h, c["wstd"], seed=12345)
+        Wq, S = synth.quantize_int4_g64(W)
+    else:
+        W, Wq, S = heads
+    Wb, Wqn, Sb = synth.bf16_bits(W), Wq.numpy(), synth.bf16_bits(S)
+    elapsed, steps = 0.0, 0
+    while steps < max_steps and (steps < min_steps or elapsed < seconds):
+        Ht, Hd = synth.make_hidden(B, K, h, c["sigma"], seed=1000 + steps)
+        u = synth.step_uniforms(1000 + steps, 0, B, K)
+        # drafts from the oracle's own q' (input preparation, not timed)
+        dl0 = oracle.lm_head_int4g64(synth.bf16_bits(Hd), Wqn, Sb, threads=cores)
+        d, _, _ = oracle.sample_rows(dl0, T32, P32, u["u_draft"].reshape(-1), threads=cores)
+        t0 = time.perf_counter()
+        tl = oracle.lm_head_bf16(synth.bf16_bits(Ht), Wb, threads=cores)
+        dl = oracle.lm_head_int4g64(synth.bf16_bits(Hd), Wqn, Sb, threads=cores)
+        oracle.verify(tl.reshape(B, K + 1, V), dl.reshape(B, K, V), d.reshape(B, K), u["u_accept"],
+                      u["u_sample"], T32, P32, threads=min(cores, B))
+        elapsed += time.perf_counter() - t0
+        steps += 1
+    return steps, elapsed, cores
+
+
+def run_reference(args, c, rank):
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        oracle_steps(c, 0.0, 1, 1)
+    steps, elapsed, cores = oracle_steps(c, 0.0, args.steps, args.steps)
+    v = steps / elapsed
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": workload_name(c), "parallelism": "replicas"},
+        "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
+                         "sample": f"{steps} whole verify steps of the workload, fp64 C oracle"},
+        "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the GPU arm
+# ---------------------------------------------------------------------------
+def build_pool(c, dev, mtpv):
+    B, K, V, h = c["B"], c["K"], c["V"], c["h"]
+    W = synth.make_head(V, h, c["wstd"], seed=12345, device=dev)
+    Wq, S = synth.quantize_int4_g64(W)
+    ht, hd, dr, ua, us = [], [], [], [], []
+    dl = torch.empty((B * K, V), dtype=torch.float32, device=dev)
+    for i in range(POOL):
+        Ht, Hd = synth.make_hidden(B, K, h, c["sigma"], seed=i, device=dev)
+        u = synth.step_uniforms(i, 0, B, K)
+        # drafts: the draft phase's own sampling from q' (library kernels)
+        mtpv.lm_head_smallm(Hd, Wq, S, mtpv.W_INT4_G64, dl)
+        d = torch.empty((B * K,), dtype=torch.int32, device=dev)
+        mtpv.sample(dl, c["T"], c["top_p"], torch.as_tensor(u["u_draft"].reshape(-1)).to(dev), d)
+        ht.append(Ht)
+        hd.append(Hd)
+        dr.append(d.view(B, K))
+        ua.append(torch.as_tensor(u["u_accept"]).to(dev))
+        us.append(torch.as_tensor(u["u_sample"]).to(dev))
+    torch.cuda.synchronize()
+    return W, Wq, S, ht, hd, dr, ua, us
+
+
+def run_gpu(args, c, rank, world, local_rank):
+    import verify_step_lm_b200 as mtpv
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    mtpv.load()
+    B, K, V, h = c["B"], c["K"], c["V"], c["h"]
+    T, top_p = c["T"], c["top_p"]
+    W, Wq, S, ht, hd, dr, ua, us = build_pool(c, dev, mtpv)
+    tl = torch.empty((B, K + 1, V), dtype=torch.float32, device=dev)
+    dl = torch.empty((B, K, V), dtype=torch.float32, device=dev)
+    ot = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+    oa = torch.empty((B,), dtype=torch.int32, device=dev)
+    rs = torch.empty((B,), dtype=torch.int32, device=dev)
+    ws = mtpv.workspace(mtpv.verify_step_workspace_bytes(B, K, V, h), dev)
+    vws = mtpv.workspace(mtpv.verify_workspace_bytes(B, K, V), dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(i):
+        j = i % POOL
+        mtpv.verify_step(W, Wq, S, ht[j], hd[j], dr[j], ua[j], us[j], B, K, T, top_p, ot, oa, rs,
+                         tl, dl, ws)
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    # --- warm-up
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+
+    # --- timed region: K whole steps through the product entry point
+    with ClockSampler(dev.index) as clk:
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(args.steps):
+            step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        step_ms = e0.elapsed_time(e1) / args.steps
+
+        # --- per-kernel breakdown: the same three launches the step makes,
+        # with events between them (same stream, same count of steps)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            j = i % POOL
+            ev = evs[i]
+            ev[0].record(stream)
+            mtpv.lm_head_smallm(ht[j], W, None, mtpv.W_BF16, tl.view(B * (K + 1), V))
+            ev[1].record(stream)
+            mtpv.lm_head_smallm(hd[j], Wq, S, mtpv.W_INT4_G64, dl.view(B * K, V))
+            ev[2].record(stream)
+            mtpv.verify(tl, dl, dr[j], ua[j], us[j], T, top_p, ot, oa, rs, ws=vws)
+            ev[3].record(stream)
+        torch.cuda.synchronize()
+        barrier()
+    clocks = clk.summary()
+    k_bf16 = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    k_int4 = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    k_samp = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    comp_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in evs)
+
+    step_ms = max_over_ranks(step_ms)
+    value = world * 1e3 / step_ms
+
+    # --- end to end: host buffers through mtpv_verify_step_host
+    e2e = None
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().contiguous().pin_memory()
+        hht = [pin(x) for x in ht]
+        hhd = [pin(x) for x in hd]
+        hdr = [pin(x) for x in dr]
+        hua = [pin(x) for x in ua]
+        hus = [pin(x) for x in us]
+        hot = torch.empty((B, K + 1), dtype=torch.int32).pin_memory()
+        hoa = torch.empty((B,), dtype=torch.int32).pin_memory()
+        hrs = torch.empty((B,), dtype=torch.int32).pin_memory()
+        hws = mtpv.workspace(mtpv.verify_step_host_workspace_bytes(B, K, V, h), dev)
+
+        def hstep(i):
+            j = i % POOL
+            mtpv.verify_step_host(W, Wq, S, hht[j], hhd[j], hdr[j], hua[j], hus[j], B, K, T, top_p,
+                                  hot, hoa, hrs, hws)
+
+        for i in range(args.warmup):
+            hstep(i)
+        barrier()
+        torch.cuda.synchronize()
+        f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        f0.record(stream)
+        for i in range(args.steps):
+            hstep(i)
+        f1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps)
+        h2d = (B * (K + 1) * h + B * K * h) * 2 + B * K * 4 + B * K * 4 + B * (K + 1) * 4
+        d2h = B * (K + 1) * 4 + B * 4 + B * 4
+        e2e = {"value": world * 1e3 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "api": "mtpv_verify_step_host (pinned host inputs/outputs)"}
+
+    if rank != 0:
+        return
+    peak, peak_kind = measured_peaks()
+    sb = step_bytes(c)
+    achieved = sb["bf16_launch"] / (k_bf16 * 1e-3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "steps/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16/int4 weights, fp32 accumulate, f64 sampler",
+        "data": "synthetic",
+        "config": {"workload": workload_name(c), "global_batch": B * world, "seq_len": K + 1,
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                   "l2": "inputs larger than L2: 1.98 GB of head weights streamed per step",
+                   "config_name": args.config},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "traffic": None, "kernel": "lm_head_bf16_kernel",
+                     "algorithmic_bytes_per_launch": sb["bf16_launch"], "peak_source": peak_kind},
+        "step_roofline": {"achieved": sb["total"] / (step_ms * 1e-3) / 1e9, "peak": peak,
+                          "unit": "GB/s", "frac": sb["total"] / (step_ms * 1e-3) / 1e9 / peak,
+                          "frac_of_8tbs": sb["total"] / (step_ms * 1e-3) / 8e12,
+                          "algorithmic_bytes_per_step": sb["total"]},
+        "kernels_ms": {"lm_head_bf16": k_bf16, "lm_head_int4": k_int4, "sampler_with_memset": k_samp,
+                       "sum": comp_ms},
+        "kernels_gbs": {"lm_head_bf16": sb["bf16_launch"] / (k_bf16 * 1e-3) / 1e9,
+                        "lm_head_int4": sb["int4_launch"] / (k_int4 * 1e-3) / 1e9},
+        "acceptance_last_step": oa.cpu().tolist(),
+        "gpu_launches": 3 * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        steps, elapsed, cores = oracle_steps(c, seconds=10.0, min_steps=2, max_steps=30,
+                                             heads=(W.cpu(), Wq.cpu(), S.cpu()))
+        line["cpu_baseline"] = {"value": steps / elapsed, "unit": "steps/s", "cores": cores,
+                                "kind": "oracle",
+                                "sample": f"{steps} whole verify steps of the workload (fp64 C oracle, "
+                                          f"{cores} threads), {elapsed:.1f} s"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--config", default="qwen27b", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="mtpv", choices=["mtpv", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    c = CONFIGS[args.config]
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        run_reference(args, c, rank)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_gpu(args, c, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
