@@ -167,6 +167,42 @@ MTPV_API mtpv_status mtpv_verify(const float *target_logits, const float *draft_
                         int32_t *row_status, void *ws, size_t ws_bytes, mtpv_stream stream);
 
 /* ------------------------------------------------------------------------
+ * mtpv_verify_noalloc -- mtpv_verify without a caller-supplied workspace.
+ * (The pages have no counterpart to this call; it is a convenience of this
+ * library.)
+ *
+ * Some callers cannot hand us device scratch memory: a decode loop that must
+ * never allocate once it runs (an allocation can synchronise the device and
+ * stall the loop), a plug-in whose host framework owns all device memory and
+ * forbids private cudaMalloc calls, or a hook that runs while a stream is
+ * being captured, where an allocation would break the capture.  This entry
+ * point takes exactly the inputs and outputs of mtpv_verify, with the same
+ * meaning, layout and results, and allocates nothing: the kernel's scratch
+ * (B ticket counters and one 40-byte statistics record per row) lives in a
+ * fixed 64 KiB array compiled into the library, which every GPU that loads the
+ * library keeps until the process exits.
+ *
+ *   Limit: round_up(4*B, 256) + round_up(40*B*(2K+1), 256) <= 65536 bytes
+ *   (for K = 3, up to B = 230 sequences); larger requests return
+ *   MTPV_ERR_UNSUPPORTED and launch nothing.  Other argument errors return
+ *   MTPV_ERR_INVALID_ARG as in mtpv_verify.
+ *   First call on a device: it looks up the array's device address once
+ *   (cudaGetSymbolAddress, which may load the library's GPU code); make that
+ *   first call before any stream capture.
+ *   Every call shares the one array and leaves its contents behind; each call
+ *   clears the counters it needs on `stream` first.  Calls whose GPU work can
+ *   overlap in time (different streams without ordering) race on the array
+ *   and give wrong results: order them on one stream.
+ *   It calls no cudaMalloc, cudaFree or allocating library routine.
+ * ---------------------------------------------------------------------- */
+MTPV_API mtpv_status mtpv_verify_noalloc(const float *target_logits, const float *draft_logits,
+                                         const int32_t *draft_tokens, const float *u_accept,
+                                         const float *u_sample, int B, int K, int V,
+                                         float temperature, float top_p, int32_t *out_tokens,
+                                         int32_t *out_accepted, int32_t *row_status,
+                                         mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
  * mtpv_sample -- one draw from the warped distribution of each of R rows
  * (temperature + top-p exactly as in mtpv_verify, inverse CDF with u[r]).
  * This is the draft phase's own sampling step (hazakura.dev notes, Layer 2
