@@ -25,14 +25,18 @@ mtpv_status cuda_status(cudaError_t e) {
 }
 
 // --- workspace layouts -----------------------------------------------------
+// verify: ticket counters, per-row statistics, then the per-row e-cache
+// (exp((l - m)/T) of every token, fp64) that lets the draw skip recomputing.
 struct VerifyWs {
-    size_t counters, stats, total;
+    size_t counters, stats, ecache, total;
 };
-VerifyWs verify_layout(int B, int K) {
+VerifyWs verify_layout(int B, int K, int V) {
+    const size_t rows = (size_t)B * (2 * K + 1);
     VerifyWs l;
     l.counters = 0;
     l.stats = up(sizeof(unsigned int) * (size_t)B);
-    l.total = l.stats + up(sizeof(mtpv::RowStats) * (size_t)B * (2 * K + 1));
+    l.ecache = l.stats + up(sizeof(mtpv::RowStats) * rows);
+    l.total = l.ecache + up(sizeof(double) * rows * (size_t)V);
     return l;
 }
 
@@ -44,7 +48,7 @@ StepWs step_layout(int B, int K, int V) {
     l.tl = 0;
     l.dl = l.tl + up(sizeof(float) * (size_t)B * (K + 1) * V);
     l.verify = l.dl + up(sizeof(float) * (size_t)B * K * V);
-    l.total = l.verify + verify_layout(B, K).total;
+    l.total = l.verify + verify_layout(B, K, V).total;
     return l;
 }
 
@@ -86,7 +90,7 @@ mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *draft
                           const float *us, int B, int K, int V, float T, float top_p,
                           int32_t *out_tokens, int32_t *out_acc, int32_t *row_status, void *ws,
                           cudaStream_t s) {
-    const VerifyWs l = verify_layout(B, K);
+    const VerifyWs l = verify_layout(B, K, V);
     unsigned int *counters = reinterpret_cast<unsigned int *>(at(ws, l.counters));
     cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(unsigned int) * (size_t)B, s);
     if (e != cudaSuccess) return cuda_status(e);
@@ -107,6 +111,7 @@ mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *draft
     p.row_status = row_status;
     p.stats = reinterpret_cast<mtpv::RowStats *>(at(ws, l.stats));
     p.counters = counters;
+    p.ecache = reinterpret_cast<double *>(at(ws, l.ecache));
     return cuda_status(mtpv::launch_sampler(p, B * (2 * K + 1), s));
 }
 
@@ -146,7 +151,7 @@ mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, const void 
 
 size_t mtpv_verify_workspace_bytes(int B, int K, int V) {
     if (!verify_shape_ok(B, K, V)) return 0;
-    return verify_layout(B, K).total;
+    return verify_layout(B, K, V).total;
 }
 
 mtpv_status mtpv_verify(const float *target_logits, const float *draft_logits,
@@ -160,7 +165,7 @@ mtpv_status mtpv_verify(const float *target_logits, const float *draft_logits,
     if (!verify_shape_ok(B, K, V) || !sampling_params_ok(temperature, top_p))
         return MTPV_ERR_INVALID_ARG;
     if (!aligned(target_logits, 4) || !aligned(draft_logits, 4)) return MTPV_ERR_INVALID_ARG;
-    if (!ws || !aligned(ws, kAlign) || ws_bytes < verify_layout(B, K).total) return MTPV_ERR_WORKSPACE;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < verify_layout(B, K, V).total) return MTPV_ERR_WORKSPACE;
     return launch_verify(target_logits, draft_logits, draft_tokens, u_accept, u_sample, B, K, V,
                          temperature, top_p, out_tokens, out_accepted, row_status, ws,
                          (cudaStream_t)stream);
@@ -168,7 +173,7 @@ mtpv_status mtpv_verify(const float *target_logits, const float *draft_logits,
 
 size_t mtpv_sample_workspace_bytes(int R, int V) {
     if (R < 1 || R > kMaxRows || V < 1 || V > kMaxV) return 0;
-    return up(sizeof(mtpv::RowStats) * (size_t)R);
+    return up(sizeof(mtpv::RowStats) * (size_t)R) + up(sizeof(double) * (size_t)R * V);
 }
 
 mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, float top_p,
@@ -194,6 +199,7 @@ mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, fl
     p.row_status = row_status;
     p.stats = reinterpret_cast<mtpv::RowStats *>(ws);
     p.counters = nullptr;
+    p.ecache = reinterpret_cast<double *>(at(ws, up(sizeof(mtpv::RowStats) * (size_t)R)));
     return cuda_status(mtpv::launch_sampler(p, R, (cudaStream_t)stream));
 }
 

@@ -6,7 +6,7 @@
 
 namespace mtpv {
 
-// Rows of bf16 activations of length Kd that one launch can stage in shared memory.
+// Rows of activations of length Kd that one launch can stage (as fp32) in shared memory.
 size_t lm_head_max_smem_rows(int Kd);
 
 // y[M, N] = x[M, Kd] . Wd[N, Kd]^T; fmt is an mtpv_wfmt.  Arguments are

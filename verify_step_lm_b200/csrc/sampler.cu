@@ -14,11 +14,14 @@
 //
 // Design for sm_100a.  One thread-block cluster of C CTAs (16, or 8 when a
 // 16-CTA cluster cannot be resident) owns one row; each CTA owns a contiguous
-// slice of the vocabulary.  Cross-CTA reductions go through distributed shared
-// memory and hardware cluster barriers (no global flags, no spin loops):
-//   P1  max / min / argmax / finiteness of the row
-//   P2  e_j = exp((l_j - m)/T) in fp64, Z, and a 2048-bin mass histogram on
-//       (m - l_j), binned linearly over the row's own range
+// slice of the vocabulary and keeps it in shared memory.  Cross-CTA steps go
+// through distributed shared memory and hardware cluster barriers (no global
+// flags, no spin loops):
+//   P1  the slice is read once (coalesced) into shared memory; max / min /
+//       argmax / finiteness of the row
+//   P2  e_j = exp((l_j - m)/T) in fp64 for every token, once: Z, a 2048-bin
+//       mass histogram on (m - l_j) over the row's own range, and (when the
+//       workspace has room) the e_j themselves for the draw
 //   P3  the bin where the descending cumulative mass reaches top_p * Z; its
 //       tokens are gathered into CTA 0, sorted on a (logit desc, index asc)
 //       64-bit key and scanned for the exact cut token.  A crossing bin with
@@ -27,10 +30,11 @@
 //   P4  verify: the last cluster of a sequence to finish its row (a global
 //       ticket counter; nobody waits) runs the acceptance tests and the
 //       residual / bonus draw.  sample: every cluster draws from its own row.
-// The draw is a cluster-wide inverse CDF whose partial sums are formed in one
-// fixed nested order (CTA slices, warp chunks, 32-wide steps), so the total,
-// the prefix that picks the CTA and the prefix used inside it agree bit for
-// bit.  All probability arithmetic is fp64 on the fp32 logits.
+// The draw is a cluster-wide inverse CDF.  Its partial sums are formed in one
+// fixed nested order (CTA slice -> warp -> thread's contiguous sub-chunk ->
+// token, every level a sequential chain), so the total, the prefix that picks
+// the CTA, the warp, the thread and the token agree bit for bit.  All
+// probability arithmetic is fp64 on the fp32 logits.
 #include <cooperative_groups.h>
 #include <float.h>
 #include <limits.h>
@@ -48,12 +52,22 @@ constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCandCap = 4096;
 constexpr int kMaxK = 16;
+constexpr int kCacheFloats = 16384;  // logits slice kept in shared memory (64 KB)
+constexpr int kBatch = 8;            // loads in flight per thread in streaming loops
+
+// Dynamic shared memory: a large region reused phase by phase, then the
+// small bookkeeping struct.
+//   region: [logits slice cache: kCacheFloats fp32][hist_mass: kBins fp64]
+//           [hist_cnt: kBins int][cand: kCandCap u64][cand_e: kCandCap fp64]
+//   during the draw the whole region is the weight buffer (fp64).
+constexpr size_t kOffHistMass = kCacheFloats * sizeof(float);
+constexpr size_t kOffHistCnt = kOffHistMass + kBins * sizeof(double);
+constexpr size_t kOffCand = kOffHistCnt + kBins * sizeof(int);
+constexpr size_t kOffCandE = kOffCand + kCandCap * sizeof(unsigned long long);
+constexpr size_t kRegionBytes = kOffCandE + kCandCap * sizeof(double);
+constexpr int kWBufDoubles = (int)(kRegionBytes / sizeof(double));
 
 struct SamplerSmem {
-    double hist_mass[kBins];
-    int hist_cnt[kBins];
-    unsigned long long cand[kCandCap];
-    double cand_e[kCandCap];
     double own_mass[kBins / 8];  // bins owned by this CTA (C >= 8), or radix digits
     int own_cnt[kBins / 8];
     double rad_mass[256];
@@ -73,6 +87,7 @@ struct SamplerSmem {
     int bc_bin, bc_cnt, bc_last;
     double bc_A;
     unsigned int cand_count;
+    unsigned int local_n, local_base;
     // derived by every CTA for itself
     float g_m, g_min;
     int g_arg, g_bad;
@@ -81,6 +96,17 @@ struct SamplerSmem {
     float cut_l;
     RowStats st[2 * kMaxK + 1];
     int seq_n, seq_status;
+};
+
+constexpr size_t kSmemBytes = kRegionBytes + sizeof(SamplerSmem);
+
+struct Region {
+    float *cache;
+    double *hist_mass;
+    int *hist_cnt;
+    unsigned long long *cand;
+    double *cand_e;
+    double *wbuf;
 };
 
 // ---------------------------------------------------------------------------
@@ -106,8 +132,45 @@ __device__ __forceinline__ int key_index(unsigned long long k) {
     return (int)(0xffffffffu - (unsigned)(k & 0xffffffffu));
 }
 
-__device__ __forceinline__ double e_of(float l, double m, double T) {
-    return exp(__dsub_rn((double)l, m) / T);
+// exp(x) in fp64 for x <= 0.  Cody-Waite range reduction (Cody and Waite,
+// "Software Manual for the Elementary Functions", 1980): k = rint(x / ln 2),
+// r = x - k ln 2 with ln 2 split into a 32-bit head (k * head is exact) and
+// the double nearest the remainder, |r| <= ln 2 / 2; exp(r) from its Taylor
+// series to degree 14 (truncation below 4e-18 relative); 2^k assembled in the
+// exponent field (two steps below 2^-1022).  Arguments below -745.2 give 0.
+__device__ __forceinline__ double exp_neg(double x) {
+    if (!(x > -745.2)) return 0.0;
+    const double kLog2e = 1.4426950408889634;
+    const double kLn2Head = 0x1.62e42ff000000p-1;
+    const double kLn2Tail = -0x1.718432a1b0e26p-35;
+    const double kRound = 6755399441055744.0;  // 1.5 * 2^52: adding it rounds to an integer
+    const double t = __fma_rn(x, kLog2e, kRound);
+    const double kd = __dsub_rn(t, kRound);
+    const int k = (int)__double2loint(t);
+    double r = __fma_rn(-kd, kLn2Head, x);
+    r = __fma_rn(-kd, kLn2Tail, r);
+    double q = 1.1470745597729725e-11;  // 1/14!
+    q = __fma_rn(q, r, 1.6059043836821613e-10);
+    q = __fma_rn(q, r, 2.08767569878681e-09);
+    q = __fma_rn(q, r, 2.505210838544172e-08);
+    q = __fma_rn(q, r, 2.755731922398589e-07);
+    q = __fma_rn(q, r, 2.7557319223985893e-06);
+    q = __fma_rn(q, r, 2.48015873015873e-05);
+    q = __fma_rn(q, r, 0.0001984126984126984);
+    q = __fma_rn(q, r, 0.001388888888888889);
+    q = __fma_rn(q, r, 0.008333333333333333);
+    q = __fma_rn(q, r, 0.041666666666666664);
+    q = __fma_rn(q, r, 0.16666666666666666);
+    q = __fma_rn(q, r, 0.5);
+    q = __fma_rn(q, r, 1.0);
+    q = __fma_rn(q, r, 1.0);
+    if (k >= -1022) return q * __hiloint2double((k + 1023) << 20, 0);
+    return (q * __hiloint2double((k + 1023 + 54) << 20, 0)) * 0x1p-54;
+}
+
+// e_j = exp((l_j - m) / T), with 1/T precomputed.
+__device__ __forceinline__ double e_of(float l, double m, double invT) {
+    return exp_neg(__dmul_rn(__dsub_rn((double)l, m), invT));
 }
 
 // Level-1 bin of a logit: linear in (m - l) over the row's range; monotone
@@ -120,12 +183,13 @@ __device__ __forceinline__ bool is_kept(const RowStats &st, float l, int j) {
     return (l > st.lstar) || (l == st.lstar && j <= st.idxstar);
 }
 
-// p'_j of one row given its statistics.
-__device__ __forceinline__ double warped_prob(const RowStats &st, const float *L, int j, double T) {
+// p'_j of one row given its statistics (logits read from global memory).
+__device__ __forceinline__ double warped_prob(const RowStats &st, const float *L, int j, double T,
+                                              double invT) {
     if (T == 0.0) return j == st.argmax ? 1.0 : 0.0;
-    float l = L[j];
+    const float l = L[j];
     if (!is_kept(st, l, j)) return 0.0;
-    return e_of(l, (double)st.m, T) / st.Zk;
+    return e_of(l, (double)st.m, invT) / st.Zk;
 }
 
 // Fixed-tree block sum (deterministic for a given launch shape).
@@ -146,15 +210,93 @@ __device__ double block_sum_d(double v, SamplerSmem &s) {
     return r;
 }
 
-// Inclusive warp scan (Kogge-Stone) in fp64.
-__device__ __forceinline__ double warp_incl_scan_d(double v) {
+// Sum over the CTAs of the cluster of the double at `addr` (one per CTA),
+// accumulated in rank order by every lane of the calling warp: lane r reads
+// rank r (the remote loads overlap), a broadcast shuffle chain adds them in a
+// fixed order.  *excl gets the sum of the ranks before `want`.
+__device__ __forceinline__ double cluster_sum_ordered(cg::cluster_group &cl, double *addr, int C,
+                                                      int want, double *excl) {
     const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        double t = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += t;
+    const double v = lane < C ? *cl.map_shared_rank(addr, lane) : 0.0;
+    double acc = 0.0, ex = 0.0;
+    for (int r = 0; r < C; ++r) {
+        const double vr = __shfl_sync(0xffffffffu, v, r);
+        if (r == want) ex = acc;
+        acc = __dadd_rn(acc, vr);
     }
-    return v;
+    if (excl) *excl = ex;
+    return acc;
+}
+
+// Warp-cooperative ordered prefix over a[0..n) (n a multiple of 32): lane l
+// sums a[l*q .. (l+1)*q) sequentially and the lane sums are chained in lane
+// order.  Returns the total.  With search, finds the first index i whose
+// inclusive prefix p_i satisfies base + p_i >= thr and returns it in *first
+// (-1 if none) with *before = base + (prefix before i).  Totals and searches
+// use the same additions, so a search started from a range's own base always
+// ends inside the range when base + total >= thr.
+__device__ double warp_prefix_search(const double *a, int n, double base, double thr, bool search,
+                                     int *first, double *before) {
+    const int lane = threadIdx.x & 31;
+    const int q = n / 32;
+    const double *my = a + lane * q;
+    double lt = 0.0;
+    for (int j = 0; j < q; ++j) lt = __dadd_rn(lt, my[j]);
+    double acc = 0.0, start = 0.0;
+    for (int r = 0; r < 32; ++r) {
+        const double v = __shfl_sync(0xffffffffu, lt, r);
+        if (r == lane) start = acc;
+        acc = __dadd_rn(acc, v);
+    }
+    if (search) {
+        int f = -1;
+        double bef = 0.0, loc = 0.0;
+        for (int j = 0; j < q; ++j) {
+            const double nl = __dadd_rn(loc, my[j]);
+            if (__dadd_rn(base, __dadd_rn(start, nl)) >= thr) {
+                f = lane * q + j;
+                bef = __dadd_rn(base, __dadd_rn(start, loc));
+                break;
+            }
+            loc = nl;
+        }
+        const unsigned hit = __ballot_sync(0xffffffffu, f >= 0);
+        if (hit) {
+            const int L = __ffs(hit) - 1;
+            *first = __shfl_sync(0xffffffffu, f, L);
+            *before = __shfl_sync(0xffffffffu, bef, L);
+        } else {
+            *first = -1;
+            *before = __dadd_rn(base, acc);
+        }
+    }
+    return acc;
+}
+
+// Bitonic sort of up to 512 keys held one per thread (block of 512), in
+// descending order; the stages that pair threads of the same warp use
+// shuffles, the rest go through `buf`.
+__device__ unsigned long long block_sort512_desc(unsigned long long key, unsigned long long *buf) {
+    const int tid = threadIdx.x;
+    for (int k = 2; k <= kThreads; k <<= 1) {
+        for (int jj = k >> 1; jj > 0; jj >>= 1) {
+            unsigned long long other;
+            if (jj >= 32) {
+                buf[tid] = key;
+                __syncthreads();
+                other = buf[tid ^ jj];
+                __syncthreads();
+            } else {
+                other = __shfl_xor_sync(0xffffffffu, key, jj);
+            }
+            const bool desc = (tid & k) == 0;
+            const bool lower = (tid & jj) == 0;
+            const unsigned long long mx = key > other ? key : other;
+            const unsigned long long mn = key > other ? other : key;
+            key = (desc == lower) ? mx : mn;
+        }
+    }
+    return key;
 }
 
 // Verify rows are ordered per sequence as K+1 target rows then K draft rows;
@@ -167,14 +309,66 @@ __device__ __forceinline__ const float *row_ptr(const SamplerParams &p, int row)
     return p.dl + ((size_t)b * p.K + (i - p.K - 1)) * p.V;
 }
 
-// Weight of token j in a draw.  kind 0: p'_t(j); kind 1: max(0, p'_t(j) - q'_d(j)).
-__device__ __forceinline__ double draw_weight(int kind, const RowStats &st_t, const float *Lt,
-                                              const RowStats &st_d, const float *Ld, int j,
-                                              double T) {
-    double pt = warped_prob(st_t, Lt, j, T);
-    if (kind == 0) return pt;
-    double w = __dsub_rn(pt, warped_prob(st_d, Ld, j, T));
+// What a draw sums over, in units of 1/Z'_t (the inverse CDF does not depend
+// on a common scale): kind 0 -> e_t[kept_t]  (= Z'_t p'_t);
+// kind 1 -> max(0, e_t[kept_t] - rho e_d[kept_d]) with rho = Z'_t / Z'_d
+// (= Z'_t max(0, p'_t - q'_d)).  The e arrays are the rows' cached
+// exp((l - m)/T) (null: recompute).
+struct DrawSrc {
+    RowStats st_t, st_d;
+    const float *Lt, *Ld;
+    const double *Et, *Ed;
+    double rho;
+    int kind;
+};
+
+__device__ __forceinline__ double draw_weight(const DrawSrc &d, int j, double invT) {
+    const float lt = d.Lt[j];
+    double wt = 0.0;
+    if (is_kept(d.st_t, lt, j)) wt = d.Et ? __ldcg(d.Et + j) : e_of(lt, (double)d.st_t.m, invT);
+    if (d.kind == 0) return wt;
+    const float ld = d.Ld[j];
+    double wd = 0.0;
+    if (is_kept(d.st_d, ld, j)) wd = d.Ed ? __ldcg(d.Ed + j) : e_of(ld, (double)d.st_d.m, invT);
+    const double w = __dsub_rn(wt, __dmul_rn(d.rho, wd));
     return w > 0.0 ? w : 0.0;
+}
+
+// draw_weight for the kBatch tokens j0, j0 + kThreads, ...: every load of the
+// batch is issued before the arithmetic (tokens at or past v1 get 0).
+__device__ __forceinline__ void draw_weights_batch(const DrawSrc &d, int v0, int v1, int j0,
+                                                   double invT, double (&w)[kBatch]) {
+    (void)v0;
+    float lt[kBatch], ld[kBatch];
+    double et[kBatch], ed[kBatch];
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+        const int j = j0 + q * kThreads;
+        lt[q] = j < v1 ? __ldg(d.Lt + j) : -INFINITY;
+        ld[q] = (d.kind == 1 && j < v1) ? __ldg(d.Ld + j) : -INFINITY;
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+        const int j = j0 + q * kThreads;
+        const bool kt = j < v1 && is_kept(d.st_t, lt[q], j);
+        const bool kd = d.kind == 1 && j < v1 && is_kept(d.st_d, ld[q], j);
+        et[q] = (kt && d.Et) ? __ldcg(d.Et + j) : 0.0;
+        ed[q] = (kd && d.Ed) ? __ldcg(d.Ed + j) : 0.0;
+    }
+#pragma unroll
+    for (int q = 0; q < kBatch; ++q) {
+        const int j = j0 + q * kThreads;
+        const bool kt = j < v1 && is_kept(d.st_t, lt[q], j);
+        const bool kd = d.kind == 1 && j < v1 && is_kept(d.st_d, ld[q], j);
+        double wt = kt ? (d.Et ? et[q] : e_of(lt[q], (double)d.st_t.m, invT)) : 0.0;
+        if (d.kind == 0) {
+            w[q] = wt;
+        } else {
+            const double wd = kd ? (d.Ed ? ed[q] : e_of(ld[q], (double)d.st_d.m, invT)) : 0.0;
+            const double x = __dsub_rn(wt, __dmul_rn(d.rho, wd));
+            w[q] = x > 0.0 ? x : 0.0;
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
@@ -182,88 +376,111 @@ __device__ __forceinline__ double draw_weight(int kind, const RowStats &st_t, co
 // Every CTA of the cluster calls it; the CTA holding the crossing writes
 // *x_out.  With allow_fallback, a residual whose total is exactly zero
 // (p' == q') is replaced by p'_t.
+// Summation order: each thread sums its contiguous sub-chunk sequentially
+// (tau), lanes are chained in lane order inside a warp (lp = prefix), warps in
+// warp order inside the CTA, CTAs in rank order.  Token j of thread t in warp
+// w has the cumulative value Pc + (Om_w + (lp_t + loc_j)), which at the end of
+// every thread, warp and CTA equals the prefix the next level starts from.
 // ---------------------------------------------------------------------------
-__device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, int kind,
-                             bool allow_fallback, const RowStats &st_t, const float *Lt,
-                             const RowStats &st_d, const float *Ld, double T, float u, int v0,
-                             int v1, int *x_out) {
+__device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double *wbuf, DrawSrc src,
+                             bool allow_fallback, double invT, float u, int v0, int v1, int *x_out) {
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
-    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
     const int n = v1 - v0;
-    const int chunk = ((n + kWarps - 1) / kWarps + 31) & ~31;
-    const int c0 = min(v1, v0 + w * chunk), c1 = min(v1, c0 + chunk);
+    const int ch = (n + kThreads - 1) / kThreads;
+    const int t0 = min(v1, v0 + tid * ch), t1 = min(v1, t0 + ch);
+    // weights computed once, coalesced, into shared memory; thread t's
+    // sub-chunk lives at wbuf[t * P ..] with an odd stride P (no bank conflicts)
+    const int P = ch | 1;
+    const bool buffered = ch > 0 && (size_t)kThreads * P <= (size_t)kWBufDoubles;
+    const double *mine = wbuf + (size_t)tid * P;
+    auto wat = [&](int j) -> double { return buffered ? mine[j - t0] : draw_weight(src, j, invT); };
 
     for (int attempt = 0; attempt < 2; ++attempt) {
-        // pass A: warp totals (sequential over 32-wide steps), CTA partial
-        double carry = 0.0;
-        for (int b = c0; b < c1; b += 32) {
-            const int j = b + lane;
-            double wj = (j < c1) ? draw_weight(kind, st_t, Lt, st_d, Ld, j, T) : 0.0;
-            double inc = warp_incl_scan_d(wj);
-            carry = __dadd_rn(carry, __shfl_sync(0xffffffffu, inc, 31));
+        if (buffered) {
+            __syncthreads();  // earlier users of the region are done
+            for (int i0 = tid; i0 < n; i0 += kBatch * kThreads) {
+                double wv[kBatch];
+                draw_weights_batch(src, v0, v1, v0 + i0, invT, wv);
+#pragma unroll
+                for (int q = 0; q < kBatch; ++q) {
+                    const int i = i0 + q * kThreads;
+                    if (i < n) {
+                        const int t = i / ch;
+                        wbuf[(size_t)t * P + (i - t * ch)] = wv[q];
+                    }
+                }
+            }
+            __syncthreads();
         }
-        if (lane == 0) s.warp_tot[w] = carry;
+        double tau = 0.0;
+        for (int j = t0; j < t1; ++j) tau = __dadd_rn(tau, wat(j));
+        double acc = 0.0, lp = 0.0;
+        for (int r = 0; r < 32; ++r) {
+            const double v = __shfl_sync(0xffffffffu, tau, r);
+            if (r == lane) lp = acc;
+            acc = __dadd_rn(acc, v);
+        }
+        if (lane == 0) s.warp_tot[w] = acc;
         __syncthreads();
-        if (threadIdx.x == 0) {
-            double acc = 0.0;
-            for (int i = 0; i < kWarps; ++i) acc = __dadd_rn(acc, s.warp_tot[i]);
-            s.pub_partial = acc;
+        if (tid == 0) {
+            double a = 0.0;
+            for (int i = 0; i < kWarps; ++i) a = __dadd_rn(a, s.warp_tot[i]);
+            s.pub_partial = a;
         }
         cluster.sync();
-        if (threadIdx.x == 0) {
-            double acc = 0.0, pc = 0.0;
-            for (int r = 0; r < C; ++r) {
-                double part = *cluster.map_shared_rank(&s.pub_partial, r);
-                if (r == rank) pc = acc;
-                acc = __dadd_rn(acc, part);
+        if (w == 0) {
+            double pc = 0.0;
+            const double tot = cluster_sum_ordered(cluster, &s.pub_partial, C, rank, &pc);
+            if (lane == 0) {
+                s.draw_Pc = pc;
+                s.draw_total = tot;
             }
-            s.draw_Pc = pc;
-            s.draw_total = acc;
         }
         cluster.sync();  // all peers have read pub_partial
         const double Pc = s.draw_Pc, total = s.draw_total;
-        if (total == 0.0 && allow_fallback && kind == 1) {
-            kind = 0;  // p' == q' exactly: draw from p'_n
+        if (total == 0.0 && allow_fallback && src.kind == 1) {
+            src.kind = 0;  // p' == q' exactly: draw from p'_n
             continue;
         }
         const double target = __dmul_rn((double)u, total);
         const double next = __dadd_rn(Pc, s.pub_partial);
-        if (!(Pc <= target && target < next)) return;  // crossing is in another CTA
-        if (threadIdx.x == 0) {
-            double acc = 0.0, Wst = 0.0;
-            int wst = kWarps - 1;
+        if (!(Pc <= target && target < next)) return;  // the crossing is in another CTA
+        if (tid == 0) {
+            double a = 0.0, om = 0.0;
+            int ws = kWarps - 1;
             for (int i = 0; i < kWarps; ++i) {
-                double nx = __dadd_rn(acc, s.warp_tot[i]);
-                if (__dadd_rn(Pc, nx) > target) { wst = i; Wst = acc; break; }
-                acc = nx;
+                const double nx = __dadd_rn(a, s.warp_tot[i]);
+                if (__dadd_rn(Pc, nx) > target) { ws = i; om = a; break; }
+                a = nx;
             }
-            s.wstar = wst;
-            s.draw_total = Wst;  // reused: prefix of the crossing warp
+            s.wstar = ws;
+            s.draw_total = om;  // reused: prefix of the crossing warp
             s.x_found = -1;
         }
         __syncthreads();
         if (w == s.wstar) {
-            const double Ww = s.draw_total;
-            double cr = 0.0;
-            int found = -1;
-            for (int b = c0; b < c1 && found < 0; b += 32) {
-                const int j = b + lane;
-                double wj = (j < c1) ? draw_weight(kind, st_t, Lt, st_d, Ld, j, T) : 0.0;
-                double inc = warp_incl_scan_d(wj);
-                double val = __dadd_rn(Pc, __dadd_rn(Ww, __dadd_rn(cr, inc)));
-                unsigned msk = __ballot_sync(0xffffffffu, (j < c1) && (val > target));
-                if (msk) found = b + __ffs(msk) - 1;
-                cr = __dadd_rn(cr, __shfl_sync(0xffffffffu, inc, 31));
+            const double om = s.draw_total;
+            const double end = __dadd_rn(Pc, __dadd_rn(om, __dadd_rn(lp, tau)));
+            const unsigned hit = __ballot_sync(0xffffffffu, end > target);
+            const int L = hit ? __ffs(hit) - 1 : 31;
+            if (lane == L) {
+                double loc = 0.0;
+                int found = -1;
+                for (int j = t0; j < t1; ++j) {
+                    loc = __dadd_rn(loc, wat(j));
+                    if (__dadd_rn(Pc, __dadd_rn(om, __dadd_rn(lp, loc))) > target) { found = j; break; }
+                }
+                s.x_found = found;
             }
-            if (lane == 0) s.x_found = found;
         }
         __syncthreads();
-        if (threadIdx.x == 0) {
+        if (tid == 0) {
             int x = s.x_found;
             if (x < 0) {  // not reachable with the consistent sums above; stay valid
                 for (int j = v1 - 1; j >= v0; --j)
-                    if (draw_weight(kind, st_t, Lt, st_d, Ld, j, T) > 0.0) { x = j; break; }
+                    if (draw_weight(src, j, invT) > 0.0) { x = j; break; }
             }
             *x_out = x;
         }
@@ -276,7 +493,15 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, int kin
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
-    SamplerSmem &s = *reinterpret_cast<SamplerSmem *>(smem_raw);
+    SamplerSmem &s = *reinterpret_cast<SamplerSmem *>(smem_raw + kRegionBytes);
+    Region rg;
+    rg.cache = reinterpret_cast<float *>(smem_raw);
+    rg.hist_mass = reinterpret_cast<double *>(smem_raw + kOffHistMass);
+    rg.hist_cnt = reinterpret_cast<int *>(smem_raw + kOffHistCnt);
+    rg.cand = reinterpret_cast<unsigned long long *>(smem_raw + kOffCand);
+    rg.cand_e = reinterpret_cast<double *>(smem_raw + kOffCandE);
+    rg.wbuf = reinterpret_cast<double *>(smem_raw);
+    float *cache = rg.cache;
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
@@ -286,19 +511,38 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
     const int V = p.V;
     const int slice = (V + C - 1) / C;
     const int v0 = min(V, rank * slice), v1 = min(V, v0 + slice);
+    const bool cached = (v1 - v0) <= kCacheFloats;
     const float *L = row_ptr(p, row);
     const double T = (double)p.T;
+    const double invT = T > 0.0 ? 1.0 / T : 0.0;
     const bool topp_all = !(p.top_p < 1.0f);
+    double *erow = p.ecache ? p.ecache + (size_t)row * V : nullptr;
+    auto lval = [&](int j) -> float { return cached ? cache[j - v0] : L[j]; };
 
-    // ---------------- P1: max, min, argmax, finiteness ----------------
+    // ---------------- P1: read the slice; max, min, argmax, finiteness ----------------
     {
         float mx = -INFINITY, mn = INFINITY;
         int arg = INT_MAX, bad = 0;
-        for (int j = v0 + tid; j < v1; j += kThreads) {
-            float l = L[j];
-            if (!isfinite(l)) bad = 1;
-            if (l > mx) { mx = l; arg = j; }
-            mn = fminf(mn, l);
+        // batches of kBatch loads are issued before any use or store, so the
+        // L2 round trips overlap
+        for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
+            float lv[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * kThreads;
+                lv[q] = j < v1 ? __ldg(L + j) : 0.0f;
+            }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * kThreads;
+                if (j < v1) {
+                    const float l = lv[q];
+                    if (cached) cache[j - v0] = l;
+                    if (!isfinite(l)) bad = 1;
+                    if (l > mx) { mx = l; arg = j; }
+                    mn = fminf(mn, l);
+                }
+            }
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
@@ -320,17 +564,20 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
             s.pub_max = mx; s.pub_min = mn; s.pub_arg = arg; s.pub_bad = bad;
         }
         cluster.sync();
-        if (tid == 0) {
-            float gm = -INFINITY, gn = INFINITY;
-            int ga = INT_MAX, gb = 0;
-            for (int r = 0; r < C; ++r) {
-                float rm = *cluster.map_shared_rank(&s.pub_max, r);
-                int ra = *cluster.map_shared_rank(&s.pub_arg, r);
-                if (rm > gm || (rm == gm && ra < ga)) { gm = rm; ga = ra; }
-                gn = fminf(gn, *cluster.map_shared_rank(&s.pub_min, r));
-                gb |= *cluster.map_shared_rank(&s.pub_bad, r);
+        if (wid == 0) {
+            float gm = lane < C ? *cluster.map_shared_rank(&s.pub_max, lane) : -INFINITY;
+            int ga = lane < C ? *cluster.map_shared_rank(&s.pub_arg, lane) : INT_MAX;
+            float gn = lane < C ? *cluster.map_shared_rank(&s.pub_min, lane) : INFINITY;
+            int gb = lane < C ? *cluster.map_shared_rank(&s.pub_bad, lane) : 0;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                const float om = __shfl_xor_sync(0xffffffffu, gm, o);
+                const int oa = __shfl_xor_sync(0xffffffffu, ga, o);
+                if (om > gm || (om == gm && oa < ga)) { gm = om; ga = oa; }
+                gn = fminf(gn, __shfl_xor_sync(0xffffffffu, gn, o));
+                gb |= __shfl_xor_sync(0xffffffffu, gb, o);
             }
-            s.g_m = gm; s.g_min = gn; s.g_arg = ga; s.g_bad = gb;
+            if (lane == 0) { s.g_m = gm; s.g_min = gn; s.g_arg = ga; s.g_bad = gb; }
         }
         __syncthreads();
     }
@@ -348,42 +595,46 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
     st.idxstar = INT_MAX;
 
     if (!bad && T > 0.0) {
-        // ---------------- P2: exps, Z, level-1 histogram ----------------
+        // ---------------- P2: exps, Z, level-1 histogram, e-cache ----------------
         const double md = (double)m;
         const float range = __fsub_rn(m, s.g_min);
         float inv_w = (range > 0.0f) ? __fdiv_rn((float)kBins, range) : 0.0f;
         if (!isfinite(inv_w)) inv_w = 0.0f;
         if (!topp_all) {
-            for (int b = tid; b < kBins; b += kThreads) { s.hist_mass[b] = 0.0; s.hist_cnt[b] = 0; }
+            for (int b = tid; b < kBins; b += kThreads) { rg.hist_mass[b] = 0.0; rg.hist_cnt[b] = 0; }
             __syncthreads();
         }
         double zt = 0.0;
-        {
-            int cur = -1, ccnt = 0;
-            double cacc = 0.0;
-            for (int j = v0 + tid; j < v1; j += kThreads) {
-                float l = L[j];
-                double e = e_of(l, md, T);
-                zt += e;
-                if (!topp_all) {
-                    int b = bin_of(l, m, inv_w);
-                    if (b != cur) {
-                        if (cur >= 0) { atomicAdd(&s.hist_mass[cur], cacc); atomicAdd(&s.hist_cnt[cur], ccnt); }
-                        cur = b; cacc = 0.0; ccnt = 0;
+        for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
+            float lv[kBatch];
+            double ev[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * kThreads;
+                lv[q] = j < v1 ? lval(j) : m;
+            }
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) ev[q] = e_of(lv[q], md, invT);
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * kThreads;
+                if (j < v1) {
+                    zt += ev[q];
+                    if (erow) erow[j] = ev[q];
+                    if (!topp_all) {
+                        const int b = bin_of(lv[q], m, inv_w);
+                        atomicAdd(&rg.hist_mass[b], ev[q]);
+                        atomicAdd(&rg.hist_cnt[b], 1);
                     }
-                    cacc += e;
-                    ++ccnt;
                 }
             }
-            if (cur >= 0) { atomicAdd(&s.hist_mass[cur], cacc); atomicAdd(&s.hist_cnt[cur], ccnt); }
         }
-        double zc = block_sum_d(zt, s);
+        const double zc = block_sum_d(zt, s);
         if (tid == 0) { s.pub_Z = zc; s.cand_count = 0u; }
         cluster.sync();
-        if (tid == 0) {
-            double z = 0.0;
-            for (int r = 0; r < C; ++r) z = __dadd_rn(z, *cluster.map_shared_rank(&s.pub_Z, r));
-            s.g_Z = z;
+        if (wid == 0) {
+            const double z = cluster_sum_ordered(cluster, &s.pub_Z, C, 0, nullptr);
+            if (lane == 0) s.g_Z = z;
         }
         __syncthreads();
         st.Z = s.g_Z;
@@ -394,54 +645,70 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
             const double thr = __dmul_rn((double)p.top_p, st.Z);
             const int per = kBins / C;
             const int base = rank * per;
-            for (int b = tid; b < per; b += kThreads) {
-                double ms = 0.0;
-                int cn = 0;
-                for (int r = 0; r < C; ++r) {
-                    ms = __dadd_rn(ms, cluster.map_shared_rank(s.hist_mass, r)[base + b]);
-                    cn += cluster.map_shared_rank(s.hist_cnt, r)[base + b];
+            // merge the cluster's histograms for the bins this CTA owns: C
+            // lanes per bin, one remote load each (all issued together), a
+            // fixed shuffle tree
+            {
+                constexpr int kPasses = kBins / kThreads;
+                const int bpp = kThreads / C, r = tid % C;
+                double vv[kPasses];
+                int cc[kPasses];
+#pragma unroll
+                for (int q = 0; q < kPasses; ++q) {
+                    const int b = q * bpp + tid / C;
+                    vv[q] = cluster.map_shared_rank(rg.hist_mass, r)[base + b];
+                    cc[q] = cluster.map_shared_rank(rg.hist_cnt, r)[base + b];
                 }
-                s.own_mass[b] = ms;
-                s.own_cnt[b] = cn;
+#pragma unroll
+                for (int q = 0; q < kPasses; ++q) {
+                    double v = vv[q];
+                    int cn = cc[q];
+                    for (int o = C >> 1; o > 0; o >>= 1) {
+                        v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+                        cn += __shfl_xor_sync(0xffffffffu, cn, o);
+                    }
+                    if (r == 0) {
+                        const int b = q * bpp + tid / C;
+                        s.own_mass[b] = v;
+                        s.own_cnt[b] = cn;
+                    }
+                }
             }
             __syncthreads();
-            if (tid == 0) {
-                double t = 0.0;
-                for (int b = 0; b < per; ++b) t = __dadd_rn(t, s.own_mass[b]);
-                s.pub_range_total = t;
+            if (wid == 0) {
+                int f;
+                double bef;
+                const double t = warp_prefix_search(s.own_mass, per, 0.0, 0.0, false, &f, &bef);
+                if (lane == 0) s.pub_range_total = t;
             }
             cluster.sync();
-            if (tid == 0) {
-                // first range whose inclusive prefix reaches thr, then the bin
+            if (wid == 0) {
+                // first range whose inclusive prefix reaches thr (same order everywhere)
+                const double v = lane < C ? *cluster.map_shared_rank(&s.pub_range_total, lane) : 0.0;
                 double P = 0.0, Pstar = 0.0;
                 int cstar = -1;
                 for (int r = 0; r < C; ++r) {
-                    double nxt = __dadd_rn(P, *cluster.map_shared_rank(&s.pub_range_total, r));
-                    if (cstar < 0 && nxt >= thr) { cstar = r; Pstar = P; }
-                    P = nxt;
+                    const double nx = __dadd_rn(P, __shfl_sync(0xffffffffu, v, r));
+                    if (cstar < 0 && nx >= thr) { cstar = r; Pstar = P; }
+                    P = nx;
                 }
+                int bstar = -2, cnt = 0;
+                double A = P;
                 if (cstar == rank) {
-                    double loc = 0.0, A = Pstar;
-                    int bstar = -1;
-                    for (int b = 0; b < per; ++b) {
-                        double nl = __dadd_rn(loc, s.own_mass[b]);
-                        if (__dadd_rn(Pstar, nl) >= thr) { bstar = base + b; A = __dadd_rn(Pstar, loc); break; }
-                        loc = nl;
-                    }
-                    if (bstar < 0) bstar = base + per - 1;  // unreachable: sums agree
-                    const int cnt = s.own_cnt[bstar - base];
-                    for (int r = 0; r < C; ++r) {
-                        *cluster.map_shared_rank(&s.bc_bin, r) = bstar;
-                        *cluster.map_shared_rank(&s.bc_cnt, r) = cnt;
-                        *cluster.map_shared_rank(&s.bc_A, r) = A;
-                    }
+                    int f;
+                    double bef;
+                    warp_prefix_search(s.own_mass, per, Pstar, thr, true, &f, &bef);
+                    if (f < 0) f = per - 1;  // not reachable: the range total reached thr
+                    bstar = base + f;
+                    cnt = s.own_cnt[f];
+                    A = bef;
                 } else if (cstar < 0 && rank == 0) {
-                    // thr above the histogram total (top_p within rounding of 1): keep all
-                    for (int r = 0; r < C; ++r) {
-                        *cluster.map_shared_rank(&s.bc_bin, r) = -1;
-                        *cluster.map_shared_rank(&s.bc_cnt, r) = 0;
-                        *cluster.map_shared_rank(&s.bc_A, r) = P;
-                    }
+                    bstar = -1;  // thr above the histogram total (top_p within rounding of 1)
+                }
+                if (bstar != -2 && lane < C) {
+                    *cluster.map_shared_rank(&s.bc_bin, lane) = bstar;
+                    *cluster.map_shared_rank(&s.bc_cnt, lane) = cnt;
+                    *cluster.map_shared_rank(&s.bc_A, lane) = A;
                 }
             }
             cluster.sync();
@@ -451,44 +718,63 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
             if (bstar < 0 || cnt == 0) {
                 st.Zk = st.Z;  // nothing to cut (top_p within rounding of 1): keep all
             } else if (cnt <= kCandCap) {
-                // gather the crossing bin's tokens into CTA 0
-                unsigned int *cc = cluster.map_shared_rank(&s.cand_count, 0);
-                unsigned long long *ck = cluster.map_shared_rank(s.cand, 0);
+                // gather the crossing bin's tokens into CTA 0: stage them
+                // locally, reserve a range with one remote atomic, copy
+                unsigned long long *stage = reinterpret_cast<unsigned long long *>(rg.cand_e);
+                if (tid == 0) s.local_n = 0u;
+                __syncthreads();
                 for (int j = v0 + tid; j < v1; j += kThreads) {
-                    float l = L[j];
+                    const float l = lval(j);
                     if (bin_of(l, m, inv_w) == bstar) {
-                        unsigned slot = atomicAdd(cc, 1u);
-                        if (slot < (unsigned)kCandCap) ck[slot] = rank_key(l, j);
+                        const unsigned slot = atomicAdd(&s.local_n, 1u);
+                        if (slot < (unsigned)kCandCap) stage[slot] = rank_key(l, j);
                     }
+                }
+                __syncthreads();
+                const unsigned nloc = min(s.local_n, (unsigned)kCandCap);
+                if (tid == 0)
+                    s.local_base = nloc ? atomicAdd(cluster.map_shared_rank(&s.cand_count, 0), nloc) : 0u;
+                __syncthreads();
+                {
+                    unsigned long long *ck = cluster.map_shared_rank(rg.cand, 0);
+                    const unsigned b0 = s.local_base;
+                    for (unsigned i = tid; i < nloc; i += kThreads)
+                        if (b0 + i < (unsigned)kCandCap) ck[b0 + i] = stage[i];
                 }
                 cluster.sync();
                 if (rank == 0) {
                     const int n = min((int)s.cand_count, kCandCap);
                     int n2 = 1;
                     while (n2 < n) n2 <<= 1;
-                    for (int i = n + tid; i < n2; i += kThreads) s.cand[i] = 0ull;
+                    if (n2 <= kThreads) {
+                        unsigned long long key = tid < n ? rg.cand[tid] : 0ull;
+                        key = block_sort512_desc(key, reinterpret_cast<unsigned long long *>(rg.hist_mass));
+                        rg.cand[tid] = key;
+                        n2 = 1;  // sorted: skip the shared-memory network below
+                    }
+                    for (int i = n + tid; i < n2; i += kThreads) rg.cand[i] = 0ull;
                     __syncthreads();
                     for (int k = 2; k <= n2; k <<= 1) {  // bitonic sort, descending
                         for (int jj = k >> 1; jj > 0; jj >>= 1) {
                             for (int i = tid; i < n2; i += kThreads) {
                                 const int ix = i ^ jj;
                                 if (ix > i) {
-                                    unsigned long long a = s.cand[i], b = s.cand[ix];
+                                    unsigned long long a = rg.cand[i], b = rg.cand[ix];
                                     const bool desc = (i & k) == 0;
-                                    if (desc ? (a < b) : (a > b)) { s.cand[i] = b; s.cand[ix] = a; }
+                                    if (desc ? (a < b) : (a > b)) { rg.cand[i] = b; rg.cand[ix] = a; }
                                 }
                             }
                             __syncthreads();
                         }
                     }
-                    for (int i = tid; i < n; i += kThreads) s.cand_e[i] = e_of(key_logit(s.cand[i]), md, T);
+                    for (int i = tid; i < n; i += kThreads) rg.cand_e[i] = e_of(key_logit(rg.cand[i]), md, invT);
                     // exclusive prefix over the sorted candidates: sequential
-                    // chunks per thread, thread totals scanned by warp 0
+                    // chunks per thread, thread totals chained by warp 0
                     const int ch = (n + kThreads - 1) / kThreads;
                     const int i0 = min(n, tid * ch), i1 = min(n, i0 + ch);
                     __syncthreads();
                     double tt = 0.0;
-                    for (int i = i0; i < i1; ++i) tt = __dadd_rn(tt, s.cand_e[i]);
+                    for (int i = i0; i < i1; ++i) tt = __dadd_rn(tt, rg.cand_e[i]);
                     s.thr_excl[tid] = tt;
                     if (tid == 0) s.first_fail = INT_MAX;
                     __syncthreads();
@@ -496,13 +782,16 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                         constexpr int per_lane = kThreads / 32;
                         double lt = 0.0;
                         for (int q = 0; q < per_lane; ++q) lt = __dadd_rn(lt, s.thr_excl[lane * per_lane + q]);
-                        double inc = warp_incl_scan_d(lt);
-                        double prev = __shfl_up_sync(0xffffffffu, inc, 1);
-                        double acc = (lane == 0) ? 0.0 : prev;
-                        for (int q = 0; q < per_lane; ++q) {
-                            double v = s.thr_excl[lane * per_lane + q];
-                            s.thr_excl[lane * per_lane + q] = acc;
+                        double acc = 0.0, start = 0.0;
+                        for (int r = 0; r < 32; ++r) {
+                            const double v = __shfl_sync(0xffffffffu, lt, r);
+                            if (r == lane) start = acc;
                             acc = __dadd_rn(acc, v);
+                        }
+                        for (int q = 0; q < per_lane; ++q) {
+                            const double v = s.thr_excl[lane * per_lane + q];
+                            s.thr_excl[lane * per_lane + q] = start;
+                            start = __dadd_rn(start, v);
                         }
                     }
                     __syncthreads();
@@ -510,7 +799,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                         double ex = s.thr_excl[tid];
                         for (int i = i0; i < i1; ++i) {
                             if (__dadd_rn(A, ex) >= thr) { atomicMin(&s.first_fail, i); break; }
-                            ex = __dadd_rn(ex, s.cand_e[i]);
+                            ex = __dadd_rn(ex, rg.cand_e[i]);
                         }
                     }
                     __syncthreads();
@@ -518,10 +807,10 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                     if (cut < 0) cut = 0;  // A < thr by construction: the first is kept
                     if (cut >= i0 && cut < i1) {
                         double ex = s.thr_excl[tid];
-                        for (int i = i0; i < cut; ++i) ex = __dadd_rn(ex, s.cand_e[i]);
-                        s.cut_Zk = __dadd_rn(A, __dadd_rn(ex, s.cand_e[cut]));
-                        s.cut_idx = key_index(s.cand[cut]);
-                        s.cut_l = key_logit(s.cand[cut]);
+                        for (int i = i0; i < cut; ++i) ex = __dadd_rn(ex, rg.cand_e[i]);
+                        s.cut_Zk = __dadd_rn(A, __dadd_rn(ex, rg.cand_e[cut]));
+                        s.cut_idx = key_index(rg.cand[cut]);
+                        s.cut_l = key_logit(rg.cand[cut]);
                     }
                     __syncthreads();
                     st.Zk = s.cut_Zk;
@@ -540,11 +829,11 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                         int cur = -1, ccnt = 0;
                         double cacc = 0.0;
                         for (int j = v0 + tid; j < v1; j += kThreads) {
-                            float l = L[j];
-                            unsigned long long key = rank_key(l, j);
+                            const float l = lval(j);
+                            const unsigned long long key = rank_key(l, j);
                             if ((key & mask) != prefix) continue;
                             const int d = (int)((key >> shift) & 255ull);
-                            double e = e_of(l, md, T);
+                            const double e = erow ? erow[j] : e_of(l, md, invT);
                             if (d != cur) {
                                 if (cur >= 0) { atomicAdd(&s.rad_mass[cur], cacc); atomicAdd(&s.rad_cnt[cur], ccnt); }
                                 cur = d; cacc = 0.0; ccnt = 0;
@@ -573,7 +862,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                             if (s.own_cnt[d] == 0) continue;
                             dlast = d;
                             Alast = acc;
-                            double nx = __dadd_rn(acc, s.own_mass[d]);
+                            const double nx = __dadd_rn(acc, s.own_mass[d]);
                             if (nx >= thr) { dsel = d; Asel = acc; break; }
                             acc = nx;
                         }
@@ -588,16 +877,16 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                 }
                 st.lstar = key_logit(prefix);
                 st.idxstar = key_index(prefix);
-                st.Zk = __dadd_rn(above, e_of(st.lstar, md, T));
+                st.Zk = __dadd_rn(above, e_of(st.lstar, md, invT));
             }
         }
     }
 
-    // publish the row statistics (CTA 0 of the cluster)
-    if (rank == 0 && tid == 0) {
-        p.stats[row] = st;
-        __threadfence();
-    }
+    // publish the row statistics (CTA 0) and make this CTA's e-cache writes
+    // visible device-wide before the cluster barrier
+    if (rank == 0 && tid == 0) p.stats[row] = st;
+    __syncthreads();
+    if (tid == 0) __threadfence();
     cluster.sync();
 
     if (!p.verify) {
@@ -620,7 +909,16 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                 if (p.row_status) p.row_status[row] = MTPV_ROW_OK;
             }
         } else {
-            cluster_draw(cluster, s, 0, false, sr, L, sr, L, T, p.u_samp[row], v0, v1, &p.out_tokens[row]);
+            DrawSrc src;
+            src.st_t = sr;
+            src.st_d = sr;
+            src.Lt = L;
+            src.Ld = L;
+            src.Et = erow;
+            src.Ed = erow;
+            src.rho = 1.0;
+            src.kind = 0;
+            cluster_draw(cluster, s, rg.wbuf, src, false, invT, p.u_samp[row], v0, v1, &p.out_tokens[row]);
             if (rank == 0 && tid == 0 && p.row_status) p.row_status[row] = MTPV_ROW_OK;
         }
         cluster.sync();
@@ -658,27 +956,26 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
     __syncthreads();
     const float *Lt0 = p.tl + (size_t)b * (K + 1) * V;
     const float *Ld0 = p.dl + (size_t)b * K * V;
-    if (tid == 0) {
+    if (wid == 0) {
+        // one lane per draft position: range check, acceptance ratio
+        const int d = lane < K ? p.drafts[b * K + lane] : 0;
+        const bool bad_d = lane < K && (d < 0 || d >= V);
+        const bool bad_r = lane < S && s.st[lane].status != MTPV_ROW_OK;
         int status = MTPV_ROW_OK;
-        for (int i = 0; i < K; ++i) {
-            const int d = p.drafts[b * K + i];
-            if (d < 0 || d >= V) status = MTPV_ROW_BAD_DRAFT;
+        if (__any_sync(0xffffffffu, bad_d)) status = MTPV_ROW_BAD_DRAFT;
+        else if (__any_sync(0xffffffffu, bad_r)) status = MTPV_ROW_NONFINITE;
+        bool reject = false;
+        if (status == MTPV_ROW_OK && lane < K) {
+            const double pt = warped_prob(s.st[lane], Lt0 + (size_t)lane * V, d, T, invT);
+            const double qd = warped_prob(s.st[K + 1 + lane], Ld0 + (size_t)lane * V, d, T, invT);
+            const double r = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
+            reject = !((double)p.u_acc[b * K + lane] < r);
         }
-        if (status == MTPV_ROW_OK)
-            for (int i = 0; i < S; ++i)
-                if (s.st[i].status != MTPV_ROW_OK) status = MTPV_ROW_NONFINITE;
-        int n = K;
-        if (status == MTPV_ROW_OK) {
-            for (int i = 0; i < K; ++i) {
-                const int d = p.drafts[b * K + i];
-                const double pt = warped_prob(s.st[i], Lt0 + (size_t)i * V, d, T);
-                const double qd = warped_prob(s.st[K + 1 + i], Ld0 + (size_t)i * V, d, T);
-                const double r = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
-                if (!((double)p.u_acc[b * K + i] < r)) { n = i; break; }
-            }
+        const unsigned rej = __ballot_sync(0xffffffffu, reject);
+        if (lane == 0) {
+            s.seq_n = rej ? __ffs(rej) - 1 : K;
+            s.seq_status = status;
         }
-        s.seq_n = n;
-        s.seq_status = status;
     }
     __syncthreads();
     const int n = s.seq_n;
@@ -702,16 +999,24 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
         if (T == 0.0) {
             if (rank == 0 && tid == 0) ot[n] = s.st[n].argmax;
         } else {
-            const float *Lt = Lt0 + (size_t)n * V;
-            const RowStats stt = s.st[n];
+            DrawSrc src;
+            src.st_t = s.st[n];
+            src.Lt = Lt0 + (size_t)n * V;
+            src.Et = p.ecache ? p.ecache + (size_t)(b * S + n) * V : nullptr;
             if (n < K) {
-                const RowStats std_ = s.st[K + 1 + n];
-                cluster_draw(cluster, s, 1, true, stt, Lt, std_, Ld0 + (size_t)n * V, T,
-                             p.u_samp[b * (K + 1) + n], v0, v1, &ot[n]);
+                src.st_d = s.st[K + 1 + n];
+                src.Ld = Ld0 + (size_t)n * V;
+                src.Ed = p.ecache ? p.ecache + (size_t)(b * S + K + 1 + n) * V : nullptr;
+                src.rho = src.st_t.Zk / src.st_d.Zk;
+                src.kind = 1;
             } else {
-                cluster_draw(cluster, s, 0, false, stt, Lt, stt, Lt, T, p.u_samp[b * (K + 1) + n],
-                             v0, v1, &ot[n]);
+                src.st_d = src.st_t;
+                src.Ld = src.Lt;
+                src.Ed = src.Et;
+                src.rho = 1.0;
+                src.kind = 0;
             }
+            cluster_draw(cluster, s, rg.wbuf, src, n < K, invT, p.u_samp[b * (K + 1) + n], v0, v1, &ot[n]);
         }
     }
     if (rank == 0 && tid == 0) p.counters[b] = 0u;
@@ -721,20 +1026,19 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t sampler_smem_bytes() { return sizeof(SamplerSmem); }
+size_t sampler_smem_bytes() { return kSmemBytes; }
 
 int sampler_cluster_size() {
     static int cached = 0;
     if (cached) return cached;
-    const size_t smem = sizeof(SamplerSmem);
-    cudaFuncSetAttribute(sampler_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(sampler_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     cudaFuncSetAttribute(sampler_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int best = 8;
     for (int c : {16, 8}) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(c, 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem;
+        cfg.dynamicSmemBytes = kSmemBytes;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeClusterDimension;
         at[0].val.clusterDim.x = c;
@@ -759,7 +1063,7 @@ cudaError_t launch_sampler(const SamplerParams &p, int rows, cudaStream_t stream
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(C, rows, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = sizeof(SamplerSmem);
+    cfg.dynamicSmemBytes = kSmemBytes;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;

@@ -32,6 +32,7 @@ struct SamplerParams {
     int32_t *row_status;  // verify: [B]; sample: [R]; may be null
     RowStats *stats;      // [rows]
     unsigned int *counters;  // verify: [B], zero on entry
+    double *ecache;       // [rows][V]: exp((l_j - m)/T) of every row (T > 0), or null
 };
 
 size_t sampler_smem_bytes();
