@@ -6,18 +6,23 @@
 // dequantise inside the inner loop, one kernel per storage format
 // (gist.science BaseRT explainer, methodology: specialisation).
 //
-// At M <= 8 every weight is used M times: the kernel is an HBM stream.  Design
-// for sm_100a:
-//   - the M activation rows are staged once per CTA in shared memory (bf16);
-//   - each warp owns RW consecutive weight rows at a time and sweeps the whole
-//     reduction length with 16-byte non-allocating loads (U chunks per lane
-//     in flight per row), so every byte of the head is read exactly once;
-//   - fp32 accumulation in registers, one warp-shuffle reduction per row;
-//   - int4 rows are dequantised in registers: each nibble n becomes the fp32
-//     value (n - 8) through the exponent trick 0x4B000000 | n = 2^23 + n
-//     (exact), the group scale multiplies the 32-weight partial sum once;
-//   - a persistent grid of (SMs x resident CTAs) walks the row groups.
+// At M <= 8 every weight is used M times, so the work is an HBM stream and the
+// kernels are built around keeping enough bytes in flight:
+//   bf16 head   CUDA cores.  Each warp owns RW consecutive weight rows and
+//               sweeps the whole reduction with 16-byte non-allocating loads,
+//               U chunks per row in flight; activations staged once per CTA
+//               as fp32 in an XOR-swizzled shared-memory layout; fp32
+//               accumulation, one warp-shuffle reduction per row.
+//   int4 head   tensor cores (mma.sync m16n8k16, fp32 accumulate).  On CUDA
+//               cores the dequantisation plus M FMAs per weight left the ALU
+//               and FMA pipes as the limit at a third of HBM bandwidth, so the
+//               weights are dequantised straight into MMA A registers and the
+//               activations are the B operand.  Each warp streams 16-row
+//               tiles through its own cp.async ring in shared memory.
+// A persistent grid of (SMs x resident CTAs) walks the row blocks.
 #include <algorithm>
+
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 #include "lm_head.cuh"
@@ -27,358 +32,13 @@ namespace mtpv {
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
 
-template <int M>
-__device__ __forceinline__ void load_x8(const uint4 *xs, int nch, int c, float (&xf)[M][8]) {
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-        const uint4 v = xs[m * nch + c];
-        xf[m][0] = bf16_lo(v.x); xf[m][1] = bf16_hi(v.x);
-        xf[m][2] = bf16_lo(v.y); xf[m][3] = bf16_hi(v.y);
-        xf[m][4] = bf16_lo(v.z); xf[m][5] = bf16_hi(v.z);
-        xf[m][6] = bf16_lo(v.w); xf[m][7] = bf16_hi(v.w);
-    }
-}
-
-// ---------------------------------------------------------------------------
-// bf16 weights: 16-byte chunk = 8 weights
-// ---------------------------------------------------------------------------
-template <int M, int RW, int U>
-__global__ void __launch_bounds__(kGemvThreads) lm_head_bf16_kernel(
-    const uint16_t *__restrict__ x, int Kd, int N, const uint16_t *__restrict__ W,
-    float *__restrict__ y, int ldy) {
-    extern __shared__ uint4 xs[];  // [M][Kd/8]
-    const int nch = Kd >> 3;
-    const uint4 *xg = reinterpret_cast<const uint4 *>(x);
-    for (int i = threadIdx.x; i < M * nch; i += kGemvThreads) xs[i] = xg[i];
-    __syncthreads();
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int groups = (N + RW - 1) / RW;
-    for (int g = blockIdx.x * kGemvWarps + warp; g < groups; g += gridDim.x * kGemvWarps) {
-        const int r0 = g * RW;
-        const uint4 *wr[RW];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-            wr[r] = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + r, N - 1) * Kd);
-        float acc[RW][M];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
-
-        for (int c0 = lane; c0 < nch; c0 += 32 * U) {
-            uint4 wv[U][RW];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-#pragma unroll
-                for (int r = 0; r < RW; ++r)
-                    wv[u][r] = (c < nch) ? ld_stream16(wr[r] + c) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-                if (c < nch) {
-                    float xf[M][8];
-                    load_x8<M>(xs, nch, c, xf);
-#pragma unroll
-                    for (int r = 0; r < RW; ++r) {
-                        const uint4 w = wv[u][r];
-                        const float wf[8] = {bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y),
-                                             bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w)};
-#pragma unroll
-                        for (int m = 0; m < M; ++m) {
-                            float a = acc[r][m];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) a = fmaf(xf[m][i], wf[i], a);
-                            acc[r][m] = a;
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                const float v = warp_sum(acc[r][m]);
-                if (lane == 0 && r0 + r < N) y[(size_t)m * ldy + r0 + r] = v;
-            }
-    }
-}
-
-// ---------------------------------------------------------------------------
-// int4 group-64 weights: 16-byte chunk = 32 weights = half a group
-// ---------------------------------------------------------------------------
-__device__ __forceinline__ float nib_minus8(uint32_t word, int i) {
-    // 2^23 + n exactly, minus (2^23 + 8)
-    return __uint_as_float(0x4B000000u | ((word >> (4 * i)) & 0xFu)) - 8388616.0f;
-}
-
-// In-place nibble dequantisation.  Nibble i of a 32-bit word sits at bits
-// 4i..4i+3; OR-ing it (unshifted, for i <= 4) into the mantissa of 2^23 gives
-// the float 2^23 + n*16^i exactly, and subtracting 2^23 + 8*16^i leaves
-// (n - 8)*16^i exactly.  Nibbles 5..7 are taken from the word shifted right by
-// 12 (positions 2..4).  The activations are stored pre-multiplied by 16^-p,
-// so every product equals (n - 8) * x exactly, as in the plain definition.
-__device__ __forceinline__ float nib_at(uint32_t w, uint32_t mask, float offset) {
-    return __fsub_rn(__uint_as_float(0x4B000000u | (w & mask)), offset);
-}
-
-// Shared-memory layouts of fp32 activations, XOR-swizzled so that a warp's
-// 128-bit loads (one chunk per lane, consecutive chunks in consecutive lanes)
-// spread over all 32 banks.
-//   int4 kernels: a chunk is 32 weights = 8 float4; float4 j of chunk c is
-//   stored at position j ^ (c & 7).
-//   bf16 kernel:  a chunk is 8 weights = 2 float4; float4 j of chunk c is
-//   stored at position j ^ ((c >> 2) & 1).
-__device__ __forceinline__ int swz32(int k) {
-    const int c = k >> 5, j = (k >> 2) & 7;
-    return (c << 5) | ((j ^ (c & 7)) << 2) | (k & 3);
-}
+// Shared-memory layout of the bf16 kernel's fp32 activations, XOR-swizzled so
+// that a warp's 128-bit loads (one 8-weight chunk per lane, consecutive chunks
+// in consecutive lanes) spread over all 32 banks: float4 j of chunk c is
+// stored at position j ^ ((c >> 2) & 1).
 __device__ __forceinline__ int swz8(int k) {
     const int c = k >> 3, j = (k >> 2) & 1;
     return (c << 3) | ((j ^ ((c >> 2) & 1)) << 2) | (k & 3);
-}
-
-// Activations for the int4 kernel: fp32, weight k of each group of 8 scaled by
-// 16^-p with p = k%8 for k%8 <= 4, k%8 - 3 otherwise (see nib_at).
-__device__ __forceinline__ float int4_x_scale(int k) {
-    const int i = k & 7;
-    const int p = i <= 4 ? i : i - 3;
-    return __uint_as_float((uint32_t)(127 - 4 * p) << 23);  // 2^(-4p)
-}
-
-// Eight dequantised weights (n - 8) * 16^p of one 32-bit word.
-__device__ __forceinline__ void int4_word_dequant(uint32_t w, float (&f)[8]) {
-    const uint32_t w2 = w >> 12;
-    f[0] = nib_at(w, 0xFu, 8388616.0f);
-    f[1] = nib_at(w, 0xF0u, 8388736.0f);
-    f[2] = nib_at(w, 0xF00u, 8390656.0f);
-    f[3] = nib_at(w, 0xF000u, 8421376.0f);
-    f[4] = nib_at(w, 0xF0000u, 8912896.0f);
-    f[5] = nib_at(w2, 0xF00u, 8390656.0f);
-    f[6] = nib_at(w2, 0xF000u, 8421376.0f);
-    f[7] = nib_at(w2, 0xF0000u, 8912896.0f);
-}
-
-__device__ __forceinline__ uint32_t word_of(const uint4 &v, int q) {
-    return q == 0 ? v.x : q == 1 ? v.y : q == 2 ? v.z : v.w;
-}
-
-template <int M, int RW, int U>
-__global__ void __launch_bounds__(kGemvThreads) lm_head_int4_v2_kernel(
-    const uint16_t *__restrict__ x, int Kd, int N, const uint8_t *__restrict__ Wq,
-    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
-    extern __shared__ float xsf[];  // [M][Kd] fp32, pre-scaled
-    for (int i = threadIdx.x; i < M * Kd; i += kGemvThreads) {
-        const int m = i / Kd, k = i - m * Kd;
-        xsf[m * Kd + swz32(k)] = __uint_as_float((uint32_t)x[i] << 16) * int4_x_scale(k);
-    }
-    __syncthreads();
-
-    const int nch = Kd >> 5;   // 16-byte chunks (32 weights) per row
-    const int ng = Kd >> 6;    // scales per row
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int groups = (N + RW - 1) / RW;
-    for (int g = blockIdx.x * kGemvWarps + warp; g < groups; g += gridDim.x * kGemvWarps) {
-        const int r0 = g * RW;
-        const uint4 *wr[RW];
-        const uint16_t *sr[RW];
-#pragma unroll
-        for (int r = 0; r < RW; ++r) {
-            const int rr = min(r0 + r, N - 1);
-            wr[r] = reinterpret_cast<const uint4 *>(Wq + (size_t)rr * (Kd >> 1));
-            sr[r] = S + (size_t)rr * ng;
-        }
-        float acc[RW][M];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
-
-        for (int c0 = lane; c0 < nch; c0 += 32 * U) {
-            uint4 wv[U][RW];
-            float sc[U][RW];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-#pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    wv[u][r] = (c < nch) ? ld_stream16(wr[r] + c) : make_uint4(0, 0, 0, 0);
-                    sc[u][r] = (c < nch) ? __uint_as_float((uint32_t)__ldg(sr[r] + (c >> 1)) << 16) : 0.0f;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-                if (c < nch) {
-                    float part[RW][M];
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < M; ++m) part[r][m] = 0.0f;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float4 xa[M], xb[M];
-#pragma unroll
-                        for (int m = 0; m < M; ++m) {
-                            xa[m] = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 32 + (((2 * q) ^ (c & 7)) << 2));
-                            xb[m] = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 32 + (((2 * q + 1) ^ (c & 7)) << 2));
-                        }
-#pragma unroll
-                        for (int r = 0; r < RW; ++r) {
-                            float f[8];
-                            int4_word_dequant(word_of(wv[u][r], q), f);
-#pragma unroll
-                            for (int m = 0; m < M; ++m) {
-                                float t = part[r][m];
-                                t = fmaf(f[0], xa[m].x, t); t = fmaf(f[1], xa[m].y, t);
-                                t = fmaf(f[2], xa[m].z, t); t = fmaf(f[3], xa[m].w, t);
-                                t = fmaf(f[4], xb[m].x, t); t = fmaf(f[5], xb[m].y, t);
-                                t = fmaf(f[6], xb[m].z, t); t = fmaf(f[7], xb[m].w, t);
-                                part[r][m] = t;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < M; ++m) acc[r][m] = fmaf(sc[u][r], part[r][m], acc[r][m]);
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                const float v = warp_sum(acc[r][m]);
-                if (lane == 0 && r0 + r < N) y[(size_t)m * ldy + r0 + r] = v;
-            }
-    }
-}
-
-// Paired fp32 arithmetic of sm_100 (two lanes of work per instruction).
-__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
-    float2 d;
-    asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(*reinterpret_cast<unsigned long long *>(&d))
-        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)));
-    return d;
-}
-__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
-    float2 d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(*reinterpret_cast<unsigned long long *>(&d))
-        : "l"(*reinterpret_cast<unsigned long long *>(&a)), "l"(*reinterpret_cast<unsigned long long *>(&b)),
-          "l"(*reinterpret_cast<unsigned long long *>(&c)));
-    return d;
-}
-
-// As lm_head_int4_v2_kernel with the dequantising subtractions and the FMAs
-// issued as f32x2 pairs; each (row, activation) keeps an even and an odd
-// partial sum.
-template <int M, int RW, int U>
-__global__ void __launch_bounds__(kGemvThreads) lm_head_int4_v3_kernel(
-    const uint16_t *__restrict__ x, int Kd, int N, const uint8_t *__restrict__ Wq,
-    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
-    extern __shared__ float xsf[];  // [M][Kd] fp32, pre-scaled
-    for (int i = threadIdx.x; i < M * Kd; i += kGemvThreads) {
-        const int m = i / Kd, k = i - m * Kd;
-        xsf[m * Kd + swz32(k)] = __uint_as_float((uint32_t)x[i] << 16) * int4_x_scale(k);
-    }
-    __syncthreads();
-
-    const int nch = Kd >> 5;
-    const int ng = Kd >> 6;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int groups = (N + RW - 1) / RW;
-    const float2 off01 = make_float2(8388616.0f, 8388736.0f);
-    const float2 off23 = make_float2(8390656.0f, 8421376.0f);
-    const float2 off45 = make_float2(8912896.0f, 8390656.0f);
-    const float2 off67 = make_float2(8421376.0f, 8912896.0f);
-    for (int g = blockIdx.x * kGemvWarps + warp; g < groups; g += gridDim.x * kGemvWarps) {
-        const int r0 = g * RW;
-        const uint4 *wr[RW];
-        const uint16_t *sr[RW];
-#pragma unroll
-        for (int r = 0; r < RW; ++r) {
-            const int rr = min(r0 + r, N - 1);
-            wr[r] = reinterpret_cast<const uint4 *>(Wq + (size_t)rr * (Kd >> 1));
-            sr[r] = S + (size_t)rr * ng;
-        }
-        float acc[RW][M];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
-
-        for (int c0 = lane; c0 < nch; c0 += 32 * U) {
-            uint4 wv[U][RW];
-            float sc[U][RW];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-#pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    wv[u][r] = (c < nch) ? ld_stream16(wr[r] + c) : make_uint4(0, 0, 0, 0);
-                    sc[u][r] = (c < nch) ? __uint_as_float((uint32_t)__ldg(sr[r] + (c >> 1)) << 16) : 0.0f;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-                if (c < nch) {
-                    float2 part[RW][M];
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < M; ++m) part[r][m] = make_float2(0.0f, 0.0f);
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {
-                        float4 xa[M], xb[M];
-#pragma unroll
-                        for (int m = 0; m < M; ++m) {
-                            xa[m] = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 32 + (((2 * q) ^ (c & 7)) << 2));
-                            xb[m] = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 32 + (((2 * q + 1) ^ (c & 7)) << 2));
-                        }
-#pragma unroll
-                        for (int r = 0; r < RW; ++r) {
-                            const uint32_t w = word_of(wv[u][r], q);
-                            const uint32_t w2 = w >> 12;
-                            const float2 f01 = sub2(make_float2(__uint_as_float(0x4B000000u | (w & 0xFu)),
-                                                                __uint_as_float(0x4B000000u | (w & 0xF0u))), off01);
-                            const float2 f23 = sub2(make_float2(__uint_as_float(0x4B000000u | (w & 0xF00u)),
-                                                                __uint_as_float(0x4B000000u | (w & 0xF000u))), off23);
-                            const float2 f45 = sub2(make_float2(__uint_as_float(0x4B000000u | (w & 0xF0000u)),
-                                                                __uint_as_float(0x4B000000u | (w2 & 0xF00u))), off45);
-                            const float2 f67 = sub2(make_float2(__uint_as_float(0x4B000000u | (w2 & 0xF000u)),
-                                                                __uint_as_float(0x4B000000u | (w2 & 0xF0000u))), off67);
-#pragma unroll
-                            for (int m = 0; m < M; ++m) {
-                                float2 t = part[r][m];
-                                t = fma2(f01, make_float2(xa[m].x, xa[m].y), t);
-                                t = fma2(f23, make_float2(xa[m].z, xa[m].w), t);
-                                t = fma2(f45, make_float2(xb[m].x, xb[m].y), t);
-                                t = fma2(f67, make_float2(xb[m].z, xb[m].w), t);
-                                part[r][m] = t;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < M; ++m)
-                            acc[r][m] = fmaf(sc[u][r], part[r][m].x + part[r][m].y, acc[r][m]);
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                const float v = warp_sum(acc[r][m]);
-                if (lane == 0 && r0 + r < N) y[(size_t)m * ldy + r0 + r] = v;
-            }
-    }
 }
 
 // bf16 weights with the activations staged as fp32 (no per-use widening).
@@ -448,98 +108,10 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_bf16_xf32_kernel(
     }
 }
 
-template <int M, int RW, int U>
-__global__ void __launch_bounds__(kGemvThreads) lm_head_int4_kernel(
-    const uint16_t *__restrict__ x, int Kd, int N, const uint8_t *__restrict__ Wq,
-    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
-    extern __shared__ uint4 xs[];  // [M][Kd/8] bf16
-    const int nx = Kd >> 3;
-    const uint4 *xg = reinterpret_cast<const uint4 *>(x);
-    for (int i = threadIdx.x; i < M * nx; i += kGemvThreads) xs[i] = xg[i];
-    __syncthreads();
-
-    const int nch = Kd >> 5;   // 16-byte chunks per row
-    const int ng = Kd >> 6;    // scales per row
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int groups = (N + RW - 1) / RW;
-    for (int g = blockIdx.x * kGemvWarps + warp; g < groups; g += gridDim.x * kGemvWarps) {
-        const int r0 = g * RW;
-        const uint4 *wr[RW];
-        const uint16_t *sr[RW];
-#pragma unroll
-        for (int r = 0; r < RW; ++r) {
-            const int rr = min(r0 + r, N - 1);
-            wr[r] = reinterpret_cast<const uint4 *>(Wq + (size_t)rr * (Kd >> 1));
-            sr[r] = S + (size_t)rr * ng;
-        }
-        float acc[RW][M];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
-
-        for (int c0 = lane; c0 < nch; c0 += 32 * U) {
-            uint4 wv[U][RW];
-            float sc[U][RW];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-#pragma unroll
-                for (int r = 0; r < RW; ++r) {
-                    wv[u][r] = (c < nch) ? ld_stream16(wr[r] + c) : make_uint4(0, 0, 0, 0);
-                    sc[u][r] = (c < nch) ? __uint_as_float((uint32_t)__ldg(sr[r] + (c >> 1)) << 16) : 0.0f;
-                }
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-                if (c < nch) {
-                    float part[RW][M];
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < M; ++m) part[r][m] = 0.0f;
-#pragma unroll
-                    for (int q = 0; q < 4; ++q) {  // 4 words of 8 weights
-                        float xf[M][8];
-                        load_x8<M>(xs, nx, c * 4 + q, xf);
-#pragma unroll
-                        for (int r = 0; r < RW; ++r) {
-                            const uint32_t word = q == 0 ? wv[u][r].x : q == 1 ? wv[u][r].y : q == 2 ? wv[u][r].z : wv[u][r].w;
-                            float wf[8];
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) wf[i] = nib_minus8(word, i);
-#pragma unroll
-                            for (int m = 0; m < M; ++m) {
-                                float a = part[r][m];
-#pragma unroll
-                                for (int i = 0; i < 8; ++i) a = fmaf(xf[m][i], wf[i], a);
-                                part[r][m] = a;
-                            }
-                        }
-                    }
-#pragma unroll
-                    for (int r = 0; r < RW; ++r)
-#pragma unroll
-                        for (int m = 0; m < M; ++m) acc[r][m] = fmaf(sc[u][r], part[r][m], acc[r][m]);
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                const float v = warp_sum(acc[r][m]);
-                if (lane == 0 && r0 + r < N) y[(size_t)m * ldy + r0 + r] = v;
-            }
-    }
-}
-
 // ---------------------------------------------------------------------------
 // int4 group-64 weights on the tensor cores (mma.sync m16n8k16, bf16 in,
-// fp32 accumulate).  At M <= 8 the CUDA-core form above is bound by its
-// dequantisation and FMA issue (ncu: ALU and FMA pipes both busy, DRAM far
-// from peak), so the draft head uses this form: the weights are the A
+// fp32 accumulate), direct-load form: the fallback for shapes the fp16 ring
+// kernel below does not take.  The weights are the A
 // operand (16 vocabulary rows x 16 k), the activations the B operand (k x 8
 // activation rows).  Dequantisation writes the A registers directly: one
 // LOP3 per two weights, ((w >> 4j) & 0x000F000F) | 0x43004300 is the bf16
@@ -689,6 +261,232 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_int4_mma_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// cp.async ring used by the fp16 int4 kernel: every warp owns NST
+// shared-memory stages, each a 16-row x GPS-group tile of the head (and its
+// scales), filled with 16-byte cp.async copies while the warp computes on an
+// earlier stage.  Tile rows are XOR-swizzled in 16-byte chunks (chunk c of row
+// r at c ^ (r & 7)), so the per-lane 8-byte fragment reads hit every bank pair
+// once.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+    const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem));
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+
+template <int GPS, int NST>
+struct Int4Ring {
+    static constexpr int kTileBytes = 16 * GPS * 32;   // 16 rows x GPS groups of 32 bytes
+    static constexpr int kScaleBytes = 16 * GPS * 2;   // 16 rows x GPS bf16 scales
+    static constexpr int kStageBytes = kTileBytes + kScaleBytes;
+    static constexpr int kWarpBytes = NST * kStageBytes;
+};
+
+// fp16 form of the ring kernel.  A word's nibbles become fp16 pairs with one
+// shift and four LOP3 (Kim et al., "Who Says Elephants Can't Run", 2022; the
+// Marlin kernel, Frantar et al., 2024): the fp16 mantissa holds a nibble at
+// bit 0 or bit 4 of each half, so
+//   (w & 0x000F000F) | 0x64006400 = (1024 + n_j, 1024 + n_{j+4})      j = 0
+//   (w & 0x00F000F0) | 0x64006400 = (1024 + 16 n_j, 1024 + 16 n_{j+4}) j = 1
+// and j = 2, 3 the same on w >> 8.  The activations paired with the j = 1, 3
+// halves are stored divided by 16, and every group's offset term
+// (1032 x or 1152 x/16 per weight) is removed with a precomputed sum.  The
+// activations are fp16, exact after a per-row power-of-two prescale that
+// keeps |x| <= 2^14 (undone on the output).  Layouts as in the bf16 kernels.
+__device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void mma_f16_16816_zc(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%10,%10,%10,%10};"
+        : "=f"(c[0]), "=f"(c[1]), "=f"(c[2]), "=f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
+}
+
+// the four fp16 pairs of one word (pair j = weights (j, j + 4) of the word)
+__device__ __forceinline__ void nib_pairs_f16(uint32_t w, uint32_t (&p)[4]) {
+    const uint32_t w8 = w >> 8;
+    p[0] = (w & 0x000F000Fu) | 0x64006400u;
+    p[1] = (w & 0x00F000F0u) | 0x64006400u;
+    p[2] = (w8 & 0x000F000Fu) | 0x64006400u;
+    p[3] = (w8 & 0x00F000F0u) | 0x64006400u;
+}
+
+template <int GPS, int NST, int NT>
+__global__ void __launch_bounds__(NT) lm_head_int4_f16_kernel(
+    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint8_t *__restrict__ Wq,
+    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
+    using R = Int4Ring<GPS, NST>;
+    static_assert(GPS % 8 == 0, "scale rows are copied in 16-byte chunks");
+    constexpr int NW = NT / 32;
+    extern __shared__ uint4 smem_mma[];
+    __shared__ unsigned int row_amax[8];
+    __shared__ float row_unscale[8];
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    uint16_t *xb = reinterpret_cast<uint16_t *>(smem_mma);                   // [M + 1][rowc * 8] fp16
+    float *xs = reinterpret_cast<float *>(smem_mma + (M + 1) * rowc);        // [Gt][8] offset sums
+    unsigned char *rings = reinterpret_cast<unsigned char *>(xs + Gt * 8);   // [warps][NST][stage]
+
+    // --- stage the activations: per-row power-of-two prescale, fp16, permuted
+    if (threadIdx.x < 8) row_amax[threadIdx.x] = 0u;
+    __syncthreads();
+    for (int i = threadIdx.x; i < M * Kd; i += NT)
+        atomicMax(&row_amax[i / Kd], ((uint32_t)x[i] << 16) & 0x7fffffffu);
+    for (int i = threadIdx.x; i < rowc * 8; i += NT) xb[M * rowc * 8 + i] = 0;
+    __syncthreads();
+    if (threadIdx.x < 8) {
+        // largest exponent e with 2^e <= max|x|; shift rows above 2^14 down
+        const int e = (int)(row_amax[threadIdx.x] >> 23) - 127;
+        const int sh = e > 13 ? e - 13 : 0;
+        row_unscale[threadIdx.x] = __uint_as_float((uint32_t)(127 + sh) << 23);
+        row_amax[threadIdx.x] = (uint32_t)sh;
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < M * Kd; i += NT) {
+        const int m = i / Kd, k = i - m * Kd;
+        const int j = (k & 15) & 3;
+        const int sh = (int)row_amax[m] + ((j & 1) ? 4 : 0);
+        const float v = __uint_as_float((uint32_t)x[i] << 16) * __uint_as_float((uint32_t)(127 - sh) << 23);
+        xb[m * rowc * 8 + mma_x_pos(k)] = __half_as_ushort(__float2half_rn(v));
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < Gt * 8; i += NT) {
+        const int G = i >> 3, m = i & 7;
+        float sum = 0.0f;
+        if (m < M)
+            for (int k = G * 64; k < G * 64 + 64; ++k) {
+                const float b = __half2float(__ushort_as_half(xb[m * rowc * 8 + mma_x_pos(k)]));
+                sum = fmaf((((k & 15) & 3) & 1) ? 1152.0f : 1032.0f, b, sum);
+            }
+        xs[i] = sum;
+    }
+    __syncthreads();
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const size_t rowbytes = (size_t)(Kd >> 1);
+    const uint4 *xrow = smem_mma + (g < M ? g : M) * rowc + 2 * t;
+    const float *xsl = xs + 2 * t;
+    unsigned char *ring = rings + (size_t)warp * R::kWarpBytes;
+    const int nblk = (N + 15) / 16;
+    const int nst = Gt / GPS;
+    const int first = blockIdx.x * NW + warp, stride = gridDim.x * NW;
+
+    // per-lane copy pattern of a stage: chunk q = lane + 32 i of the 16 x (2 GPS) tile
+    constexpr int kCp = GPS;  // 16-byte weight chunks per lane per stage
+    int cp_row[kCp], cp_soff[kCp], cp_goff[kCp];
+#pragma unroll
+    for (int i = 0; i < kCp; ++i) {
+        const int q = lane + 32 * i;
+        const int r = q / (2 * GPS), c = q % (2 * GPS);
+        cp_row[i] = r;
+        cp_soff[i] = r * (GPS * 32) + ((c ^ (r & 7)) << 4);
+        cp_goff[i] = c * 16;
+    }
+    const int sc_r = lane / (GPS / 8), sc_c = lane % (GPS / 8);
+
+    int it_task = first, it_st = 0, it_slot = 0;  // next tile to issue
+    auto issue = [&]() {
+        if (it_task < nblk) {
+            unsigned char *slot = ring + it_slot * R::kStageBytes;
+            const uint8_t *base = Wq + (size_t)it_st * GPS * 32;
+#pragma unroll
+            for (int i = 0; i < kCp; ++i) {
+                const int row = min(it_task * 16 + cp_row[i], N - 1);
+                cp_async16(slot + cp_soff[i], base + row * rowbytes + cp_goff[i]);
+            }
+            if (lane < 2 * GPS) {
+                const int row = min(it_task * 16 + sc_r, N - 1);
+                cp_async16(slot + R::kTileBytes + sc_r * (GPS * 2) + sc_c * 16,
+                           S + (size_t)row * Gt + (size_t)it_st * GPS + sc_c * 8);
+            }
+            if (++it_st == nst) { it_st = 0; it_task += stride; }
+            if (++it_slot == NST) it_slot = 0;
+        }
+        cp_async_commit();
+    };
+
+#pragma unroll
+    for (int k = 0; k < NST - 1; ++k) issue();
+    int slot_i = 0;
+    for (int task = first; task < nblk; task += stride) {
+        float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+        for (int st = 0; st < nst; ++st) {
+            issue();
+            cp_async_wait<NST - 1>();
+            __syncwarp();
+            const unsigned char *slot = ring + slot_i * R::kStageBytes;
+            if (++slot_i == NST) slot_i = 0;
+            const uint16_t *ssl = reinterpret_cast<const uint16_t *>(slot + R::kTileBytes);
+            const unsigned char *rowg = slot + g * (GPS * 32) + 8 * (t & 1);
+            const unsigned char *rowg8 = rowg + 8 * (GPS * 32);
+            const uint4 *xr = xrow + st * GPS * 8;
+            const float *xc = xsl + st * GPS * 8;
+#pragma unroll
+            for (int gq = 0; gq < GPS; ++gq) {
+                const int sw = ((2 * gq + (t >> 1)) ^ g) << 4;
+                const uint2 w0 = *reinterpret_cast<const uint2 *>(rowg + sw);
+                const uint2 w1 = *reinterpret_cast<const uint2 *>(rowg8 + sw);
+                const float s0 = __uint_as_float((uint32_t)ssl[g * GPS + gq] << 16);
+                const float s1 = __uint_as_float((uint32_t)ssl[(g + 8) * GPS + gq] << 16);
+                const uint4 bA = xr[gq * 8];
+                const uint4 bB = xr[gq * 8 + 1];
+                const float2 corr = *reinterpret_cast<const float2 *>(xc + gq * 8);
+                uint32_t p0x[4], p1x[4], p0y[4], p1y[4];
+                nib_pairs_f16(w0.x, p0x);
+                nib_pairs_f16(w1.x, p1x);
+                nib_pairs_f16(w0.y, p0y);
+                nib_pairs_f16(w1.y, p1y);
+                float c[4];
+                {
+                    const uint32_t a[4] = {p0x[0], p1x[0], p0y[0], p1y[0]};
+                    mma_f16_16816_zc(c, a, bA.x, bA.y);
+                }
+                {
+                    const uint32_t a[4] = {p0x[1], p1x[1], p0y[1], p1y[1]};
+                    mma_f16_16816(c, a, bA.z, bA.w);
+                }
+                {
+                    const uint32_t a[4] = {p0x[2], p1x[2], p0y[2], p1y[2]};
+                    mma_f16_16816(c, a, bB.x, bB.y);
+                }
+                {
+                    const uint32_t a[4] = {p0x[3], p1x[3], p0y[3], p1y[3]};
+                    mma_f16_16816(c, a, bB.z, bB.w);
+                }
+                acc[0] = fmaf(s0, c[0] - corr.x, acc[0]);
+                acc[1] = fmaf(s0, c[1] - corr.y, acc[1]);
+                acc[2] = fmaf(s1, c[2] - corr.x, acc[2]);
+                acc[3] = fmaf(s1, c[3] - corr.y, acc[3]);
+            }
+            __syncwarp();  // every lane is done with this slot before it is refilled
+        }
+        const int r0 = task * 16;
+        const int m0 = 2 * t, m1 = 2 * t + 1;
+        const int ra = r0 + g, rbw = r0 + g + 8;
+        if (m0 < M) {
+            const float us = row_unscale[m0];
+            if (ra < N) y[(size_t)m0 * ldy + ra] = acc[0] * us;
+            if (rbw < N) y[(size_t)m0 * ldy + rbw] = acc[2] * us;
+        }
+        if (m1 < M) {
+            const float us = row_unscale[m1];
+            if (ra < N) y[(size_t)m1 * ldy + ra] = acc[1] * us;
+            if (rbw < N) y[(size_t)m1 * ldy + rbw] = acc[3] * us;
+        }
+    }
+    cp_async_wait<0>();
+}
+
+// ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
 template <typename Kern>
@@ -705,7 +503,7 @@ template <int M>
 static cudaError_t launch_bf16(const uint16_t *x, int Kd, int N, const uint16_t *W, float *y,
                                int ldy, cudaStream_t s) {
     constexpr int RW = M <= 4 ? 4 : 2;
-    constexpr int U = 4;
+    constexpr int U = M <= 4 ? 4 : 2;
     auto k = lm_head_bf16_xf32_kernel<M, RW, U>;
     const size_t smem = (size_t)M * Kd * sizeof(float);
     if (smem > 48 * 1024) {
@@ -719,28 +517,39 @@ static cudaError_t launch_bf16(const uint16_t *x, int Kd, int N, const uint16_t 
     return cudaGetLastError();
 }
 
-template <int M>
-static cudaError_t launch_int4(const uint16_t *x, int Kd, int N, const uint8_t *Wq,
-                               const uint16_t *S, float *y, int ldy, cudaStream_t s) {
-    constexpr int RW = M <= 4 ? 4 : 2;
-    constexpr int U = 2;
-    auto k = lm_head_int4_v3_kernel<M, RW, U>;
-    const size_t smem = (size_t)M * Kd * sizeof(float);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
-    const int groups = (N + RW - 1) / RW;
-    const int need = (groups + kGemvWarps - 1) / kGemvWarps;
-    const int grid = std::min(need, kSMs * resident_ctas(k, smem));
-    k<<<grid, kGemvThreads, smem, s>>>(x, Kd, N, Wq, S, y, ldy);
-    return cudaGetLastError();
-}
-
-// Shared memory of the tensor-core int4 kernel for M (<= 8) activation rows.
+// Shared memory of the direct-load tensor-core int4 kernel for M (<= 8) rows.
 static size_t int4_mma_smem(int M, int Kd) {
     const size_t Gt = (size_t)Kd / 64;
     return (size_t)M * (Gt * 8 + 1) * 16 + Gt * 8 * sizeof(float);
+}
+
+// The fp16 ring kernel: 3-stage rings of 8 groups in 12 warps per CTA.
+constexpr int kF16Gps = 8, kF16Nst = 3, kF16Threads = 384;
+static size_t int4_f16_smem(int M, int Kd) {
+    const size_t Gt = (size_t)Kd / 64;
+    return (size_t)(M + 1) * (Gt * 8 + 1) * 16 + Gt * 8 * sizeof(float) +
+           (size_t)(kF16Threads / 32) * Int4Ring<kF16Gps, kF16Nst>::kWarpBytes;
+}
+static bool int4_f16_ok(int M, int Kd) {
+    return M <= 8 && Kd % (64 * kF16Gps) == 0 && int4_f16_smem(M, Kd) <= (size_t)227 * 1024;
+}
+
+static cudaError_t launch_int4_f16(const uint16_t *x, int M, int Kd, int N, const uint8_t *Wq,
+                                   const uint16_t *S, float *y, int ldy, cudaStream_t s) {
+    auto k = lm_head_int4_f16_kernel<kF16Gps, kF16Nst, kF16Threads>;
+    const size_t smem = int4_f16_smem(M, Kd);
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int occ = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kF16Threads, smem) != cudaSuccess || occ < 1) {
+        cudaGetLastError();
+        occ = 1;
+    }
+    const int nblk = (N + 15) / 16;
+    const int need = (nblk + kF16Threads / 32 - 1) / (kF16Threads / 32);
+    const int grid = std::min(need, kSMs * occ);
+    k<<<grid, kF16Threads, smem, s>>>(x, M, Kd, N, Wq, S, y, ldy);
+    return cudaGetLastError();
 }
 
 static cudaError_t launch_int4_mma(const uint16_t *x, int M, int Kd, int N, const uint8_t *Wq,
@@ -789,21 +598,17 @@ cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, c
         } else {
             const uint8_t *Wq = static_cast<const uint8_t *>(w);
             const uint16_t *S = static_cast<const uint16_t *>(scales);
+            if (int4_f16_ok(mm, Kd)) {
+                e = launch_int4_f16(xm, mm, Kd, N, Wq, S, ym, N, s);
+                if (e != cudaSuccess) return e;
+                continue;
+            }
             if (int4_mma_smem(mm, Kd) <= (size_t)227 * 1024) {
                 e = launch_int4_mma(xm, mm, Kd, N, Wq, S, ym, N, s);
                 if (e != cudaSuccess) return e;
                 continue;
             }
-            switch (mm) {
-                case 1: e = launch_int4<1>(xm, Kd, N, Wq, S, ym, N, s); break;
-                case 2: e = launch_int4<2>(xm, Kd, N, Wq, S, ym, N, s); break;
-                case 3: e = launch_int4<3>(xm, Kd, N, Wq, S, ym, N, s); break;
-                case 4: e = launch_int4<4>(xm, Kd, N, Wq, S, ym, N, s); break;
-                case 5: e = launch_int4<5>(xm, Kd, N, Wq, S, ym, N, s); break;
-                case 6: e = launch_int4<6>(xm, Kd, N, Wq, S, ym, N, s); break;
-                case 7: e = launch_int4<7>(xm, Kd, N, Wq, S, ym, N, s); break;
-                default: e = launch_int4<8>(xm, Kd, N, Wq, S, ym, N, s); break;
-            }
+            return cudaErrorInvalidValue;  // no int4 kernel for this shape
         }
         if (e != cudaSuccess) return e;
     }
