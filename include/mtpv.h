@@ -91,9 +91,16 @@ MTPV_API const char *mtpv_status_string(mtpv_status st);
  *   y[m][n] = sum_k x[m][k] * Wd[n][k],  0 <= m < M, 0 <= n < N   (fp32 out)
  *
  *   x       device, bf16 [M, Kd] row-major (activations / hidden states).
- *   M       rows, 1 <= M <= 64.  The kernel is built for M <= 8; larger M is
- *           processed in groups of 8 rows (the weights are re-read per group).
- *   Kd      reduction length, a positive multiple of 64.
+ *   M       rows, 1 <= M <= 64.  The kernels are built for M <= 8; larger M is
+ *           processed in groups of min(8, floor(232448 / (4 Kd))) rows (the
+ *           weights are re-read per group).
+ *   Kd      reduction length, a positive multiple of 64, at most 58112 (the
+ *           kernels stage each activation row in shared memory as fp32).
+ *           MTPV_W_INT4_G64 with Kd a multiple of 512 and
+ *           (M + 1)(2 Kd + 16) + Kd/2 <= 75776 bytes of staged activations
+ *           (M <= 6 at Kd = 5120) runs on the tensor cores (fp16 MMA, exact fp16 dequantisation, fp32
+ *           accumulation per 64-weight group); other int4 shapes use a bf16
+ *           MMA form with the same accumulation order per group.
  *   N       output columns (vocabulary rows of the head), N >= 1.
  *   w       device weights, layout per fmt:
  *             MTPV_W_BF16:     bf16 [N, Kd] (nn.Linear out x in layout);
