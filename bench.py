@@ -1,7 +1,7 @@
 """Benchmark of the speculative-decoding verify step on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
-                    [--impl {mtpv,reference}] [--no-cpu-baseline] [--no-e2e]
+                    [--impl {mtpv,reference}] [--no-cpu-baseline] [--no-e2e] [--no-graph]
 
 One step = the whole verify step of one batch: the K+1 target rows through
 the bf16 LM head, the K draft rows through the int4 group-64 head, and the
@@ -306,6 +306,33 @@ def run_gpu(args, c, rank, world, local_rank):
     step_ms = max_over_ranks(step_ms)
     value = world * 1e3 / step_ms
 
+    # --- the same steps replayed from CUDA graphs (one captured graph per
+    # pool entry; the library makes no allocation or host sync inside a step)
+    graph = None
+    if not args.no_graph:
+        graphs = []
+        for j in range(POOL):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                step(j)
+            graphs.append(g)
+        torch.cuda.synchronize()
+        for i in range(args.warmup):
+            graphs[i % POOL].replay()
+        barrier()
+        torch.cuda.synchronize()
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for i in range(args.steps):
+            graphs[i % POOL].replay()
+        g1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        graph_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
+        graph = {"value": world * 1e3 / graph_ms, "unit": "steps/s", "ms_per_step": graph_ms,
+                 "graphs": POOL, "nodes_per_step": "4 kernels"}
+        del graphs
+
     # --- end to end: host buffers through mtpv_verify_step_host
     e2e = None
     if not args.no_e2e:
@@ -358,20 +385,21 @@ def run_gpu(args, c, rank, world, local_rank):
                    "l2": "inputs larger than L2: 1.98 GB of head weights streamed per step",
                    "config_name": args.config},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None, "kernel": "lm_head_bf16_kernel",
+                     "frac": achieved / peak, "traffic": None, "kernel": "lm_head_bf16_xf32_kernel",
                      "algorithmic_bytes_per_launch": sb["bf16_launch"], "peak_source": peak_kind},
         "step_roofline": {"achieved": sb["total"] / (step_ms * 1e-3) / 1e9, "peak": peak,
                           "unit": "GB/s", "frac": sb["total"] / (step_ms * 1e-3) / 1e9 / peak,
                           "frac_of_8tbs": sb["total"] / (step_ms * 1e-3) / 8e12,
                           "algorithmic_bytes_per_step": sb["total"]},
-        "kernels_ms": {"lm_head_bf16": k_bf16, "lm_head_int4": k_int4, "sampler_with_memset": k_samp,
+        "kernels_ms": {"lm_head_bf16": k_bf16, "lm_head_int4": k_int4, "sampler": k_samp,
                        "sum": comp_ms},
         "kernels_gbs": {"lm_head_bf16": sb["bf16_launch"] / (k_bf16 * 1e-3) / 1e9,
                         "lm_head_int4": sb["int4_launch"] / (k_int4 * 1e-3) / 1e9},
         "acceptance_last_step": oa.cpu().tolist(),
-        "gpu_launches": 3 * args.steps,
+        "gpu_launches": 4 * args.steps,
         "clocks": clocks,
         "e2e": e2e,
+        "graph": graph,
     }
     if not args.no_cpu_baseline and world == 1:
         steps, elapsed, cores = oracle_steps(c, seconds=10.0, min_steps=2, max_steps=30,
@@ -392,6 +420,7 @@ def main():
     ap.add_argument("--impl", default="mtpv", choices=["mtpv", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")

@@ -25,8 +25,9 @@ mtpv_status cuda_status(cudaError_t e) {
 }
 
 // --- workspace layouts -----------------------------------------------------
-// verify: ticket counters, per-row statistics, then the per-row e-cache
-// (exp((l - m)/T) of every token, fp64) that lets the draw skip recomputing.
+// verify: ticket counters, per-row statistics slots, then the per-row
+// weights (exp((l - m)/T) of kept tokens, 0 elsewhere; fp64) that the draw
+// kernel reads instead of recomputing.
 struct VerifyWs {
     size_t counters, stats, ecache, total;
 };
@@ -35,7 +36,7 @@ VerifyWs verify_layout(int B, int K, int V) {
     VerifyWs l;
     l.counters = 0;
     l.stats = up(sizeof(unsigned int) * (size_t)B);
-    l.ecache = l.stats + up(sizeof(mtpv::RowStats) * rows);
+    l.ecache = l.stats + up(sizeof(mtpv::RowSlot) * rows);
     l.total = l.ecache + up(sizeof(double) * rows * (size_t)V);
     return l;
 }
@@ -92,8 +93,6 @@ mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *draft
                           cudaStream_t s) {
     const VerifyWs l = verify_layout(B, K, V);
     unsigned int *counters = reinterpret_cast<unsigned int *>(at(ws, l.counters));
-    cudaError_t e = cudaMemsetAsync(counters, 0, sizeof(unsigned int) * (size_t)B, s);
-    if (e != cudaSuccess) return cuda_status(e);
     mtpv::SamplerParams p;
     p.tl = tl;
     p.dl = dl;
@@ -109,7 +108,7 @@ mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *draft
     p.out_tokens = out_tokens;
     p.out_acc = out_acc;
     p.row_status = row_status;
-    p.stats = reinterpret_cast<mtpv::RowStats *>(at(ws, l.stats));
+    p.slots = reinterpret_cast<mtpv::RowSlot *>(at(ws, l.stats));
     p.counters = counters;
     p.ecache = reinterpret_cast<double *>(at(ws, l.ecache));
     return cuda_status(mtpv::launch_sampler(p, B * (2 * K + 1), s));
@@ -173,7 +172,7 @@ mtpv_status mtpv_verify(const float *target_logits, const float *draft_logits,
 
 size_t mtpv_sample_workspace_bytes(int R, int V) {
     if (R < 1 || R > kMaxRows || V < 1 || V > kMaxV) return 0;
-    return up(sizeof(mtpv::RowStats) * (size_t)R) + up(sizeof(double) * (size_t)R * V);
+    return up(sizeof(mtpv::RowSlot) * (size_t)R) + up(sizeof(double) * (size_t)R * V);
 }
 
 mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, float top_p,
@@ -197,9 +196,9 @@ mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, fl
     p.verify = 0;
     p.out_tokens = out;
     p.row_status = row_status;
-    p.stats = reinterpret_cast<mtpv::RowStats *>(ws);
+    p.slots = reinterpret_cast<mtpv::RowSlot *>(ws);
     p.counters = nullptr;
-    p.ecache = reinterpret_cast<double *>(at(ws, up(sizeof(mtpv::RowStats) * (size_t)R)));
+    p.ecache = reinterpret_cast<double *>(at(ws, up(sizeof(mtpv::RowSlot) * (size_t)R)));
     return cuda_status(mtpv::launch_sampler(p, R, (cudaStream_t)stream));
 }
 

@@ -270,11 +270,11 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_int4_mma_kernel(
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(sa), "l"(gmem) : "memory");
 }
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;"); }
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N)); }
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 template <int GPS, int NST>
 struct Int4Ring {
@@ -489,16 +489,6 @@ __global__ void __launch_bounds__(NT) lm_head_int4_f16_kernel(
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <typename Kern>
-static int resident_ctas(Kern k, size_t smem) {
-    int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kGemvThreads, smem) != cudaSuccess) {
-        cudaGetLastError();
-        occ = 1;
-    }
-    return std::max(1, occ);
-}
-
 template <int M>
 static cudaError_t launch_bf16(const uint16_t *x, int Kd, int N, const uint16_t *W, float *y,
                                int ldy, cudaStream_t s) {
@@ -506,13 +496,12 @@ static cudaError_t launch_bf16(const uint16_t *x, int Kd, int N, const uint16_t 
     constexpr int U = M <= 4 ? 4 : 2;
     auto k = lm_head_bf16_xf32_kernel<M, RW, U>;
     const size_t smem = (size_t)M * Kd * sizeof(float);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
+    int occ = 0;
+    cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ);
+    if (e != cudaSuccess) return e;
     const int groups = (N + RW - 1) / RW;
     const int need = (groups + kGemvWarps - 1) / kGemvWarps;
-    const int grid = std::min(need, kSMs * resident_ctas(k, smem));
+    const int grid = std::min(need, kSMs * occ);
     k<<<grid, kGemvThreads, smem, s>>>(x, Kd, N, W, y, ldy);
     return cudaGetLastError();
 }
@@ -530,21 +519,18 @@ static size_t int4_f16_smem(int M, int Kd) {
     return (size_t)(M + 1) * (Gt * 8 + 1) * 16 + Gt * 8 * sizeof(float) +
            (size_t)(kF16Threads / 32) * Int4Ring<kF16Gps, kF16Nst>::kWarpBytes;
 }
-static bool int4_f16_ok(int M, int Kd) {
-    return M <= 8 && Kd % (64 * kF16Gps) == 0 && int4_f16_smem(M, Kd) <= (size_t)227 * 1024;
+static bool int4_f16_ok(int M, int Kd, const void *S) {
+    return M <= 8 && Kd % (64 * kF16Gps) == 0 && ((uintptr_t)S & 15) == 0 &&
+           int4_f16_smem(M, Kd) <= (size_t)227 * 1024;
 }
 
 static cudaError_t launch_int4_f16(const uint16_t *x, int M, int Kd, int N, const uint8_t *Wq,
                                    const uint16_t *S, float *y, int ldy, cudaStream_t s) {
     auto k = lm_head_int4_f16_kernel<kF16Gps, kF16Nst, kF16Threads>;
     const size_t smem = int4_f16_smem(M, Kd);
-    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
     int occ = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k, kF16Threads, smem) != cudaSuccess || occ < 1) {
-        cudaGetLastError();
-        occ = 1;
-    }
+    cudaError_t e = kernel_setup((const void *)k, kF16Threads, smem, &occ);
+    if (e != cudaSuccess) return e;
     const int nblk = (N + 15) / 16;
     const int need = (nblk + kF16Threads / 32 - 1) / (kF16Threads / 32);
     const int grid = std::min(need, kSMs * occ);
@@ -557,13 +543,12 @@ static cudaError_t launch_int4_mma(const uint16_t *x, int M, int Kd, int N, cons
     constexpr int RB = 2, U = 4;
     auto k = lm_head_int4_mma_kernel<RB, U>;
     const size_t smem = int4_mma_smem(M, Kd);
-    if (smem > 48 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return e;
-    }
+    int occ = 0;
+    cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ);
+    if (e != cudaSuccess) return e;
     const int ntask = ((N + 15) / 16 + RB - 1) / RB;
     const int need = (ntask + kGemvWarps - 1) / kGemvWarps;
-    const int grid = std::min(need, kSMs * resident_ctas(k, smem));
+    const int grid = std::min(need, kSMs * occ);
     k<<<grid, kGemvThreads, smem, s>>>(x, M, Kd, N, Wq, S, y, ldy);
     return cudaGetLastError();
 }
@@ -598,7 +583,7 @@ cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, c
         } else {
             const uint8_t *Wq = static_cast<const uint8_t *>(w);
             const uint16_t *S = static_cast<const uint16_t *>(scales);
-            if (int4_f16_ok(mm, Kd)) {
+            if (int4_f16_ok(mm, Kd, S)) {
                 e = launch_int4_f16(xm, mm, Kd, N, Wq, S, ym, N, s);
                 if (e != cudaSuccess) return e;
                 continue;

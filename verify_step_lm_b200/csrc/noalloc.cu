@@ -16,6 +16,7 @@ constexpr int kMaxDevices = 64;
 constexpr int kMaxK = 16;
 constexpr int kMaxV = 1 << 24;
 constexpr int kMaxRows = 65535;
+static_assert(sizeof(mtpv::RowSlot) == 40, "the documented limit counts 40 bytes per row");
 
 // The library's own scratch.  In host code this name is only a stand-in for
 // the device object; its device address comes from cudaGetSymbolAddress.
@@ -64,7 +65,7 @@ extern "C" mtpv_status mtpv_verify_noalloc(const float *target_logits, const flo
     // scratch layout: B ticket counters, then one statistics record per row
     const size_t rows = (size_t)B * (2 * K + 1);
     const size_t stats_off = round_up(sizeof(unsigned int) * (size_t)B);
-    const size_t need = stats_off + round_up(sizeof(mtpv::RowStats) * rows);
+    const size_t need = stats_off + round_up(sizeof(mtpv::RowSlot) * rows);
     if (need > kScratchBytes) return MTPV_ERR_UNSUPPORTED;  // beyond the fixed scratch
 
     void *scratch = nullptr;
@@ -75,12 +76,7 @@ extern "C" mtpv_status mtpv_verify_noalloc(const float *target_logits, const flo
     }
     cudaStream_t s = (cudaStream_t)stream;
     unsigned int *counters = static_cast<unsigned int *>(scratch);
-    // the counters must start at zero; the statistics are written before use
-    e = cudaMemsetAsync(counters, 0, sizeof(unsigned int) * (size_t)B, s);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        return MTPV_ERR_CUDA;
-    }
+    // the statistics kernel clears the counters; the slots are written before use
     mtpv::SamplerParams p = {};
     p.tl = target_logits;
     p.dl = draft_logits;
@@ -96,7 +92,7 @@ extern "C" mtpv_status mtpv_verify_noalloc(const float *target_logits, const flo
     p.out_tokens = out_tokens;
     p.out_acc = out_accepted;
     p.row_status = row_status;
-    p.stats = reinterpret_cast<mtpv::RowStats *>(static_cast<unsigned char *>(scratch) + stats_off);
+    p.slots = reinterpret_cast<mtpv::RowSlot *>(static_cast<unsigned char *>(scratch) + stats_off);
     p.counters = counters;
     e = mtpv::launch_sampler(p, (int)rows, s);
     if (e != cudaSuccess) {

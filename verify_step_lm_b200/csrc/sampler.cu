@@ -12,33 +12,42 @@
 //                 (p'_n if that is all zero), else the bonus from p'_K; the
 //                 draw is the inverse CDF in vocabulary order.
 //
-// Design for sm_100a.  One thread-block cluster of C CTAs (16, or 8 when a
-// 16-CTA cluster cannot be resident) owns one row; each CTA owns a contiguous
-// slice of the vocabulary and keeps it in shared memory.  Cross-CTA steps go
-// through distributed shared memory and hardware cluster barriers (no global
-// flags, no spin loops):
-//   P1  the slice is read once (coalesced) into shared memory; max / min /
-//       argmax / finiteness of the row
-//   P2  e_j = exp((l_j - m)/T) in fp64 for every token, once: Z, a 2048-bin
-//       mass histogram on (m - l_j) over the row's own range, and (when the
-//       workspace has room) the e_j themselves for the draw
+// Design for sm_100a: two kernels, each a grid of thread-block clusters of C
+// CTAs (16, or 8 when a 16-CTA cluster cannot be resident); every cross-CTA
+// step goes through distributed shared memory and hardware cluster barriers
+// (no global flags, no spin loops).
+// Statistics kernel, one cluster per logits row; each CTA owns a contiguous
+// slice of the vocabulary and keeps it in shared memory:
+//   P1  the slice is read once (coalesced); max / min / argmax / finiteness
+//   P2  e_j = exp((l_j - m)/T) in fp64 for every token: Z and a 2048-bin mass
+//       histogram on (m - l_j) over the row's own range
 //   P3  the bin where the descending cumulative mass reaches top_p * Z; its
 //       tokens are gathered into CTA 0, sorted on a (logit desc, index asc)
 //       64-bit key and scanned for the exact cut token.  A crossing bin with
 //       more than kCandCap tokens (massive ties, degenerate ranges) falls back
 //       to an 8-pass weighted radix select on the same key.
-//   P4  verify: the last cluster of a sequence to finish its row (a global
-//       ticket counter; nobody waits) runs the acceptance tests and the
-//       residual / bonus draw.  sample: every cluster draws from its own row.
-// The draw is a cluster-wide inverse CDF.  Its partial sums are formed in one
-// fixed nested order (CTA slice -> warp -> thread's contiguous sub-chunk ->
-// token, every level a sequential chain), so the total, the prefix that picks
-// the CTA, the warp, the thread and the token agree bit for bit.  All
-// probability arithmetic is fp64 on the fp32 logits.
+//   out the row's statistics, and (workspace permitting) the row's weights
+//       e_j of kept tokens, 0 elsewhere: p'_j = e_j / Z' with no further test
+// Draw kernel, one cluster per draft position i of a sequence (sampling: per
+// row).  The acceptance test of d_i reads two weights; the cluster then draws
+// position i's residual token (the bonus at i == K) with u_samp[i], as if the
+// first rejection were at i, by a cluster-wide inverse CDF over the weights:
+// every load is independent of the others, nothing is recomputed.  The last
+// cluster of a sequence to finish (a global ticket counter; nobody waits)
+// reads the K+1 position records, finds n and writes the outputs.  Drawing
+// every position in parallel gives the same tokens as drawing only at n,
+// since each draw uses its own uniform.
+// The draw's partial sums are formed in one fixed nested order (CTA slice ->
+// warp -> thread's contiguous sub-chunk -> token, every level a sequential
+// chain), so the total, the prefix that picks the CTA, the warp, the thread
+// and the token agree bit for bit.  All probability arithmetic is fp64 on the
+// fp32 logits.
 #include <cooperative_groups.h>
 #include <float.h>
 #include <limits.h>
 #include <math.h>
+
+#include <mutex>
 
 #include "common.cuh"
 #include "sampler.cuh"
@@ -51,7 +60,6 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCandCap = 4096;
-constexpr int kMaxK = 16;
 constexpr int kCacheFloats = 16384;  // logits slice kept in shared memory (64 KB)
 constexpr int kBatch = 8;            // loads in flight per thread in streaming loops
 
@@ -65,7 +73,8 @@ constexpr size_t kOffHistCnt = kOffHistMass + kBins * sizeof(double);
 constexpr size_t kOffCand = kOffHistCnt + kBins * sizeof(int);
 constexpr size_t kOffCandE = kOffCand + kCandCap * sizeof(unsigned long long);
 constexpr size_t kRegionBytes = kOffCandE + kCandCap * sizeof(double);
-constexpr int kWBufDoubles = (int)(kRegionBytes / sizeof(double));
+constexpr int kDrawBufDoubles = 16384;  // the draw kernel's weight buffer (128 KB)
+constexpr size_t kDrawBufBytes = kDrawBufDoubles * sizeof(double);
 
 struct SamplerSmem {
     double own_mass[kBins / 8];  // bins owned by this CTA (C >= 8), or radix digits
@@ -94,11 +103,11 @@ struct SamplerSmem {
     double g_Z, draw_Pc, draw_total, cut_Zk;
     int wstar, x_found, first_fail, cut_idx;
     float cut_l;
-    RowStats st[2 * kMaxK + 1];
-    int seq_n, seq_status;
+    int res_x, res_acc;  // draw kernel: the position's token and acceptance, in CTA 0
 };
 
-constexpr size_t kSmemBytes = kRegionBytes + sizeof(SamplerSmem);
+constexpr size_t kStatsSmemBytes = kRegionBytes + sizeof(SamplerSmem);
+constexpr size_t kDrawSmemBytes = kDrawBufBytes + sizeof(SamplerSmem);
 
 struct Region {
     float *cache;
@@ -106,7 +115,6 @@ struct Region {
     int *hist_cnt;
     unsigned long long *cand;
     double *cand_e;
-    double *wbuf;
 };
 
 // ---------------------------------------------------------------------------
@@ -312,8 +320,9 @@ __device__ __forceinline__ const float *row_ptr(const SamplerParams &p, int row)
 // What a draw sums over, in units of 1/Z'_t (the inverse CDF does not depend
 // on a common scale): kind 0 -> e_t[kept_t]  (= Z'_t p'_t);
 // kind 1 -> max(0, e_t[kept_t] - rho e_d[kept_d]) with rho = Z'_t / Z'_d
-// (= Z'_t max(0, p'_t - q'_d)).  The e arrays are the rows' cached
-// exp((l - m)/T) (null: recompute).
+// (= Z'_t max(0, p'_t - q'_d)).  With the statistics kernel's weights (Et,
+// Ed: e of kept tokens, 0 elsewhere) a weight is two independent loads;
+// without them (null) it is recomputed from the logits and the statistics.
 struct DrawSrc {
     RowStats st_t, st_d;
     const float *Lt, *Ld;
@@ -322,25 +331,39 @@ struct DrawSrc {
     int kind;
 };
 
-__device__ __forceinline__ double draw_weight(const DrawSrc &d, int j, double invT) {
-    const float lt = d.Lt[j];
-    double wt = 0.0;
-    if (is_kept(d.st_t, lt, j)) wt = d.Et ? __ldcg(d.Et + j) : e_of(lt, (double)d.st_t.m, invT);
+__device__ __forceinline__ double draw_combine(const DrawSrc &d, double wt, double wd) {
     if (d.kind == 0) return wt;
-    const float ld = d.Ld[j];
-    double wd = 0.0;
-    if (is_kept(d.st_d, ld, j)) wd = d.Ed ? __ldcg(d.Ed + j) : e_of(ld, (double)d.st_d.m, invT);
     const double w = __dsub_rn(wt, __dmul_rn(d.rho, wd));
     return w > 0.0 ? w : 0.0;
 }
 
+__device__ __forceinline__ double draw_weight(const DrawSrc &d, int j, double invT) {
+    if (d.Et) return draw_combine(d, d.Et[j], d.kind == 1 ? d.Ed[j] : 0.0);
+    const float lt = d.Lt[j];
+    const double wt = is_kept(d.st_t, lt, j) ? e_of(lt, (double)d.st_t.m, invT) : 0.0;
+    if (d.kind == 0) return wt;
+    const float ld = d.Ld[j];
+    const double wd = is_kept(d.st_d, ld, j) ? e_of(ld, (double)d.st_d.m, invT) : 0.0;
+    return draw_combine(d, wt, wd);
+}
+
 // draw_weight for the kBatch tokens j0, j0 + kThreads, ...: every load of the
 // batch is issued before the arithmetic (tokens at or past v1 get 0).
-__device__ __forceinline__ void draw_weights_batch(const DrawSrc &d, int v0, int v1, int j0,
-                                                   double invT, double (&w)[kBatch]) {
-    (void)v0;
+__device__ __forceinline__ void draw_weights_batch(const DrawSrc &d, int v1, int j0, double invT,
+                                                   double (&w)[kBatch]) {
+    if (d.Et) {
+        double et[kBatch], ed[kBatch];
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) {
+            const int j = j0 + q * kThreads;
+            et[q] = j < v1 ? d.Et[j] : 0.0;
+            ed[q] = (d.kind == 1 && j < v1) ? d.Ed[j] : 0.0;
+        }
+#pragma unroll
+        for (int q = 0; q < kBatch; ++q) w[q] = draw_combine(d, et[q], ed[q]);
+        return;
+    }
     float lt[kBatch], ld[kBatch];
-    double et[kBatch], ed[kBatch];
 #pragma unroll
     for (int q = 0; q < kBatch; ++q) {
         const int j = j0 + q * kThreads;
@@ -350,24 +373,10 @@ __device__ __forceinline__ void draw_weights_batch(const DrawSrc &d, int v0, int
 #pragma unroll
     for (int q = 0; q < kBatch; ++q) {
         const int j = j0 + q * kThreads;
-        const bool kt = j < v1 && is_kept(d.st_t, lt[q], j);
-        const bool kd = d.kind == 1 && j < v1 && is_kept(d.st_d, ld[q], j);
-        et[q] = (kt && d.Et) ? __ldcg(d.Et + j) : 0.0;
-        ed[q] = (kd && d.Ed) ? __ldcg(d.Ed + j) : 0.0;
-    }
-#pragma unroll
-    for (int q = 0; q < kBatch; ++q) {
-        const int j = j0 + q * kThreads;
-        const bool kt = j < v1 && is_kept(d.st_t, lt[q], j);
-        const bool kd = d.kind == 1 && j < v1 && is_kept(d.st_d, ld[q], j);
-        double wt = kt ? (d.Et ? et[q] : e_of(lt[q], (double)d.st_t.m, invT)) : 0.0;
-        if (d.kind == 0) {
-            w[q] = wt;
-        } else {
-            const double wd = kd ? (d.Ed ? ed[q] : e_of(ld[q], (double)d.st_d.m, invT)) : 0.0;
-            const double x = __dsub_rn(wt, __dmul_rn(d.rho, wd));
-            w[q] = x > 0.0 ? x : 0.0;
-        }
+        const double wt = (j < v1 && is_kept(d.st_t, lt[q], j)) ? e_of(lt[q], (double)d.st_t.m, invT) : 0.0;
+        const double wd = (d.kind == 1 && j < v1 && is_kept(d.st_d, ld[q], j))
+                              ? e_of(ld[q], (double)d.st_d.m, invT) : 0.0;
+        w[q] = draw_combine(d, wt, wd);
     }
 }
 
@@ -393,7 +402,7 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
     // weights computed once, coalesced, into shared memory; thread t's
     // sub-chunk lives at wbuf[t * P ..] with an odd stride P (no bank conflicts)
     const int P = ch | 1;
-    const bool buffered = ch > 0 && (size_t)kThreads * P <= (size_t)kWBufDoubles;
+    const bool buffered = ch > 0 && (size_t)kThreads * P <= (size_t)kDrawBufDoubles;
     const double *mine = wbuf + (size_t)tid * P;
     auto wat = [&](int j) -> double { return buffered ? mine[j - t0] : draw_weight(src, j, invT); };
 
@@ -402,7 +411,7 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
             __syncthreads();  // earlier users of the region are done
             for (int i0 = tid; i0 < n; i0 += kBatch * kThreads) {
                 double wv[kBatch];
-                draw_weights_batch(src, v0, v1, v0 + i0, invT, wv);
+                draw_weights_batch(src, v1, v0 + i0, invT, wv);
 #pragma unroll
                 for (int q = 0; q < kBatch; ++q) {
                     const int i = i0 + q * kThreads;
@@ -489,9 +498,9 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
 }
 
 // ---------------------------------------------------------------------------
-// the kernel: one cluster per row
+// statistics kernel: one cluster per logits row
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
+__global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SamplerSmem &s = *reinterpret_cast<SamplerSmem *>(smem_raw + kRegionBytes);
     Region rg;
@@ -500,7 +509,6 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
     rg.hist_cnt = reinterpret_cast<int *>(smem_raw + kOffHistCnt);
     rg.cand = reinterpret_cast<unsigned long long *>(smem_raw + kOffCand);
     rg.cand_e = reinterpret_cast<double *>(smem_raw + kOffCandE);
-    rg.wbuf = reinterpret_cast<double *>(smem_raw);
     float *cache = rg.cache;
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
@@ -517,6 +525,8 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
     const double invT = T > 0.0 ? 1.0 / T : 0.0;
     const bool topp_all = !(p.top_p < 1.0f);
     double *erow = p.ecache ? p.ecache + (size_t)row * V : nullptr;
+    if (p.verify && row == 0 && rank == 0)  // ticket counters of the draw kernel
+        for (int k = tid; k < p.B; k += kThreads) p.counters[k] = 0u;
     auto lval = [&](int j) -> float { return cached ? cache[j - v0] : L[j]; };
 
     // ---------------- P1: read the slice; max, min, argmax, finiteness ----------------
@@ -620,7 +630,6 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                 const int j = j0 + q * kThreads;
                 if (j < v1) {
                     zt += ev[q];
-                    if (erow) erow[j] = ev[q];
                     if (!topp_all) {
                         const int b = bin_of(lv[q], m, inv_w);
                         atomicAdd(&rg.hist_mass[b], ev[q]);
@@ -813,10 +822,16 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                         s.cut_l = key_logit(rg.cand[cut]);
                     }
                     __syncthreads();
-                    st.Zk = s.cut_Zk;
-                    st.idxstar = s.cut_idx;
-                    st.lstar = s.cut_l;
+                    if (wid == 0 && lane < C) {  // the cut, into every CTA of the cluster
+                        *cluster.map_shared_rank(&s.cut_Zk, lane) = s.cut_Zk;
+                        *cluster.map_shared_rank(&s.cut_idx, lane) = s.cut_idx;
+                        *cluster.map_shared_rank(&s.cut_l, lane) = s.cut_l;
+                    }
                 }
+                cluster.sync();
+                st.Zk = s.cut_Zk;
+                st.idxstar = s.cut_idx;
+                st.lstar = s.cut_l;
             } else {
                 // weighted radix select on the 64-bit key, 8 bits per pass
                 unsigned long long prefix = 0ull, mask = 0ull;
@@ -833,7 +848,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
                             const unsigned long long key = rank_key(l, j);
                             if ((key & mask) != prefix) continue;
                             const int d = (int)((key >> shift) & 255ull);
-                            const double e = erow ? erow[j] : e_of(l, md, invT);
+                            const double e = e_of(l, md, invT);
                             if (d != cur) {
                                 if (cur >= 0) { atomicAdd(&s.rad_mass[cur], cacc); atomicAdd(&s.rad_cnt[cur], ccnt); }
                                 cur = d; cacc = 0.0; ccnt = 0;
@@ -882,163 +897,170 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_kernel(SamplerParams p) {
         }
     }
 
-    // publish the row statistics (CTA 0) and make this CTA's e-cache writes
-    // visible device-wide before the cluster barrier
-    if (rank == 0 && tid == 0) p.stats[row] = st;
-    __syncthreads();
-    if (tid == 0) __threadfence();
-    cluster.sync();
-
-    if (!p.verify) {
-        // ---------------- P4 (sample): draw from this row ----------------
-        RowStats sr;
-        sr.m = __ldcg(&p.stats[row].m);
-        sr.Zk = __ldcg(&p.stats[row].Zk);
-        sr.lstar = __ldcg(&p.stats[row].lstar);
-        sr.idxstar = __ldcg(&p.stats[row].idxstar);
-        sr.argmax = __ldcg(&p.stats[row].argmax);
-        sr.status = __ldcg(&p.stats[row].status);
-        if (sr.status != MTPV_ROW_OK) {
-            if (rank == 0 && tid == 0) {
-                p.out_tokens[row] = -1;
-                if (p.row_status) p.row_status[row] = sr.status;
+    // the row's statistics, then its weights: e_j of kept tokens, 0 elsewhere
+    if (rank == 0 && tid == 0) p.slots[row].st = st;
+    if (erow && !bad && T > 0.0) {
+        const double md = (double)m;
+        for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
+            float lv[kBatch];
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * kThreads;
+                lv[q] = j < v1 ? lval(j) : -INFINITY;
             }
-        } else if (T == 0.0) {
-            if (rank == 0 && tid == 0) {
-                p.out_tokens[row] = sr.argmax;
-                if (p.row_status) p.row_status[row] = MTPV_ROW_OK;
+#pragma unroll
+            for (int q = 0; q < kBatch; ++q) {
+                const int j = j0 + q * kThreads;
+                if (j < v1) erow[j] = is_kept(st, lv[q], j) ? e_of(lv[q], md, invT) : 0.0;
             }
-        } else {
-            DrawSrc src;
-            src.st_t = sr;
-            src.st_d = sr;
-            src.Lt = L;
-            src.Ld = L;
-            src.Et = erow;
-            src.Ed = erow;
-            src.rho = 1.0;
-            src.kind = 0;
-            cluster_draw(cluster, s, rg.wbuf, src, false, invT, p.u_samp[row], v0, v1, &p.out_tokens[row]);
-            if (rank == 0 && tid == 0 && p.row_status) p.row_status[row] = MTPV_ROW_OK;
         }
-        cluster.sync();
-        return;
     }
+    cluster.sync();  // no CTA exits while a peer may still read its shared memory
+}
 
-    // ---------------- P4 (verify): the last cluster of the sequence ----------------
-    const int S = 2 * p.K + 1;
-    const int b = row / S;
+// ---------------------------------------------------------------------------
+// draw kernel: one cluster per draft position (verify) or per row (sample)
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams p) {
+    extern __shared__ __align__(16) unsigned char smem_raw[];
+    SamplerSmem &s = *reinterpret_cast<SamplerSmem *>(smem_raw + kDrawBufBytes);
+    double *wbuf = reinterpret_cast<double *>(smem_raw);
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
+    const int tid = threadIdx.x;
+    const int V = p.V, K = p.K;
+    const int slice = (V + C - 1) / C;
+    const int v0 = min(V, rank * slice), v1 = min(V, v0 + slice);
+    const double T = (double)p.T;
+    const double invT = T > 0.0 ? 1.0 / T : 0.0;
+
+    // this cluster's rows: verify position i of sequence b -> target row i and
+    // (i < K) draft row i; sample -> one row
+    const int c = blockIdx.y;
+    int b = c, i = 0, rt = c, rd = c;
+    if (p.verify) {
+        const int S = 2 * K + 1;
+        b = c / (K + 1);
+        i = c - b * (K + 1);
+        rt = b * S + i;
+        rd = i < K ? b * S + K + 1 + i : rt;
+    }
+    const bool residual = p.verify && i < K;
     if (rank == 0 && tid == 0) {
-        const unsigned old = atomicAdd(&p.counters[b], 1u);
-        const int last = (old == (unsigned)(S - 1));
-        for (int r = 0; r < C; ++r) *cluster.map_shared_rank(&s.bc_last, r) = last;
+        s.res_x = -1;
+        s.res_acc = 0;
     }
-    cluster.sync();
-    if (!s.bc_last) {
-        cluster.sync();
-        return;
-    }
-    __threadfence();
-    const int K = p.K;
-    if (tid < S) {
-        const RowStats *g = &p.stats[b * S + tid];
-        RowStats r;
-        r.Z = __ldcg(&g->Z);
-        r.Zk = __ldcg(&g->Zk);
-        r.m = __ldcg(&g->m);
-        r.lmin = __ldcg(&g->lmin);
-        r.lstar = __ldcg(&g->lstar);
-        r.idxstar = __ldcg(&g->idxstar);
-        r.argmax = __ldcg(&g->argmax);
-        r.status = __ldcg(&g->status);
-        s.st[tid] = r;
-    }
-    __syncthreads();
-    const float *Lt0 = p.tl + (size_t)b * (K + 1) * V;
-    const float *Ld0 = p.dl + (size_t)b * K * V;
-    if (wid == 0) {
-        // one lane per draft position: range check, acceptance ratio
-        const int d = lane < K ? p.drafts[b * K + lane] : 0;
-        const bool bad_d = lane < K && (d < 0 || d >= V);
-        const bool bad_r = lane < S && s.st[lane].status != MTPV_ROW_OK;
-        int status = MTPV_ROW_OK;
-        if (__any_sync(0xffffffffu, bad_d)) status = MTPV_ROW_BAD_DRAFT;
-        else if (__any_sync(0xffffffffu, bad_r)) status = MTPV_ROW_NONFINITE;
-        bool reject = false;
-        if (status == MTPV_ROW_OK && lane < K) {
-            const double pt = warped_prob(s.st[lane], Lt0 + (size_t)lane * V, d, T, invT);
-            const double qd = warped_prob(s.st[K + 1 + lane], Ld0 + (size_t)lane * V, d, T, invT);
-            const double r = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
-            reject = !((double)p.u_acc[b * K + lane] < r);
-        }
-        const unsigned rej = __ballot_sync(0xffffffffu, reject);
-        if (lane == 0) {
-            s.seq_n = rej ? __ffs(rej) - 1 : K;
-            s.seq_status = status;
-        }
-    }
-    __syncthreads();
-    const int n = s.seq_n;
-    const int status = s.seq_status;
-    int32_t *ot = p.out_tokens + (size_t)b * (K + 1);
-    if (status != MTPV_ROW_OK) {
-        if (rank == 0 && tid <= K) ot[tid] = -1;
-        if (rank == 0 && tid == 0) {
-            p.out_acc[b] = -1;
-            if (p.row_status) p.row_status[b] = status;
-        }
-    } else {
-        if (rank == 0 && tid <= K) {
-            if (tid < n) ot[tid] = p.drafts[b * K + tid];
-            else if (tid > n) ot[tid] = -1;
-        }
-        if (rank == 0 && tid == 0) {
-            p.out_acc[b] = n;
-            if (p.row_status) p.row_status[b] = MTPV_ROW_OK;
-        }
-        if (T == 0.0) {
-            if (rank == 0 && tid == 0) ot[n] = s.st[n].argmax;
-        } else {
-            DrawSrc src;
-            src.st_t = s.st[n];
-            src.Lt = Lt0 + (size_t)n * V;
-            src.Et = p.ecache ? p.ecache + (size_t)(b * S + n) * V : nullptr;
-            if (n < K) {
-                src.st_d = s.st[K + 1 + n];
-                src.Ld = Ld0 + (size_t)n * V;
-                src.Ed = p.ecache ? p.ecache + (size_t)(b * S + K + 1 + n) * V : nullptr;
-                src.rho = src.st_t.Zk / src.st_d.Zk;
-                src.kind = 1;
+    const RowStats st_t = p.slots[rt].st;
+    const RowStats st_d = p.slots[rd].st;
+    const float *Lt = row_ptr(p, rt), *Ld = row_ptr(p, rd);
+    const double *Et = p.ecache ? p.ecache + (size_t)rt * V : nullptr;
+    const double *Ed = p.ecache ? p.ecache + (size_t)rd * V : nullptr;
+
+    // ---------------- acceptance test of d_i ----------------
+    int status = st_t.status;
+    if (residual) {
+        const int d = p.drafts[(size_t)b * K + i];
+        if (d < 0 || d >= V) status = MTPV_ROW_BAD_DRAFT;
+        else if (st_d.status != MTPV_ROW_OK) status = MTPV_ROW_NONFINITE;
+        if (status == MTPV_ROW_OK && rank == 0 && tid == 0) {
+            double pt, qd;  // p'_i(d_i), q'_i(d_i)
+            if (Et && T > 0.0) {
+                pt = Et[d] / st_t.Zk;
+                qd = Ed[d] / st_d.Zk;
             } else {
-                src.st_d = src.st_t;
-                src.Ld = src.Lt;
-                src.Ed = src.Et;
-                src.rho = 1.0;
-                src.kind = 0;
+                pt = warped_prob(st_t, Lt, d, T, invT);
+                qd = warped_prob(st_d, Ld, d, T, invT);
             }
-            cluster_draw(cluster, s, rg.wbuf, src, n < K, invT, p.u_samp[b * (K + 1) + n], v0, v1, &ot[n]);
+            const double ratio = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
+            s.res_acc = (double)p.u_acc[(size_t)b * K + i] < ratio ? 1 : 0;
         }
     }
-    if (rank == 0 && tid == 0) p.counters[b] = 0u;
-    cluster.sync();
+
+    // ---------------- this position's residual / bonus draw ----------------
+    int *x_dst = p.verify ? cluster.map_shared_rank(&s.res_x, 0) : &p.out_tokens[c];
+    if (status != MTPV_ROW_OK) {
+        if (rank == 0 && tid == 0) *x_dst = -1;
+    } else if (T == 0.0) {
+        if (rank == 0 && tid == 0) *x_dst = st_t.argmax;
+    } else {
+        DrawSrc src;
+        src.st_t = st_t;
+        src.st_d = residual ? st_d : st_t;
+        src.Lt = Lt;
+        src.Ld = residual ? Ld : Lt;
+        src.Et = Et;
+        src.Ed = residual ? Ed : Et;
+        src.rho = residual ? st_t.Zk / st_d.Zk : 1.0;
+        src.kind = residual ? 1 : 0;
+        const float u = p.verify ? p.u_samp[(size_t)b * (K + 1) + i] : p.u_samp[c];
+        cluster_draw(cluster, s, wbuf, src, residual, invT, u, v0, v1, x_dst);
+    }
+    if (rank == 0 && tid == 0 && !p.verify && p.row_status) p.row_status[c] = status;
+    cluster.sync();  // verify: res_x and res_acc are in CTA 0; no CTA exits while a peer reads it
+    if (!p.verify || rank != 0 || tid != 0) return;
+
+    // ---------------- record, ticket, and (last cluster) the sequence's outputs ----------------
+    const int S = 2 * K + 1;
+    PosRecord rec;
+    rec.x = s.res_x;
+    rec.accept = s.res_acc;
+    rec.status = status;
+    rec.pad = 0;
+    p.slots[rt].rec = rec;  // target row i's statistics are not read again
+    __threadfence();
+    const unsigned old = atomicAdd(&p.counters[b], 1u);
+    if (old != (unsigned)K) return;  // another position of sequence b finishes last
+    __threadfence();
+    int seq_status = MTPV_ROW_OK, n = K;
+    for (int k = 0; k <= K; ++k) {
+        const int sk = __ldcg(&p.slots[b * S + k].rec.status);
+        if (sk == MTPV_ROW_BAD_DRAFT) seq_status = MTPV_ROW_BAD_DRAFT;
+        else if (sk != MTPV_ROW_OK && seq_status == MTPV_ROW_OK) seq_status = sk;
+    }
+    for (int k = 0; k < K; ++k)
+        if (!__ldcg(&p.slots[b * S + k].rec.accept)) { n = k; break; }
+    int32_t *ot = p.out_tokens + (size_t)b * (K + 1);
+    if (seq_status != MTPV_ROW_OK) {
+        for (int k = 0; k <= K; ++k) ot[k] = -1;
+        p.out_acc[b] = -1;
+    } else {
+        for (int k = 0; k < n; ++k) ot[k] = p.drafts[(size_t)b * K + k];
+        ot[n] = __ldcg(&p.slots[b * S + n].rec.x);
+        for (int k = n + 1; k <= K; ++k) ot[k] = -1;
+        p.out_acc[b] = n;
+    }
+    if (p.row_status) p.row_status[b] = seq_status;
+    p.counters[b] = 0u;
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-size_t sampler_smem_bytes() { return kSmemBytes; }
+namespace {
 
-int sampler_cluster_size() {
-    static int cached = 0;
-    if (cached) return cached;
-    cudaFuncSetAttribute(sampler_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
-    cudaFuncSetAttribute(sampler_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+// Cluster size of each sampler kernel per device (16 when a 16-CTA cluster
+// can be resident, else 8), found once; 0 = not yet known.
+int g_cluster_size[2][64];
+std::mutex g_cluster_mu;
+
+template <typename Kern>
+int cluster_size_for(int which, Kern kernel, size_t smem) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 8;
+    }
+    std::lock_guard<std::mutex> lock(g_cluster_mu);
+    if (g_cluster_size[which][dev]) return g_cluster_size[which][dev];
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
     int best = 8;
     for (int c : {16, 8}) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(c, 1, 1);
         cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = kSmemBytes;
+        cfg.dynamicSmemBytes = smem;
         cudaLaunchAttribute at[1];
         at[0].id = cudaLaunchAttributeClusterDimension;
         at[0].val.clusterDim.x = c;
@@ -1047,23 +1069,23 @@ int sampler_cluster_size() {
         cfg.attrs = at;
         cfg.numAttrs = 1;
         int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, sampler_kernel, &cfg) == cudaSuccess &&
-            nclusters > 0) {
+        if (cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg) == cudaSuccess && nclusters > 0) {
             best = c;
             break;
         }
         cudaGetLastError();
     }
-    cached = best;
+    g_cluster_size[which][dev] = best;
     return best;
 }
 
-cudaError_t launch_sampler(const SamplerParams &p, int rows, cudaStream_t stream) {
-    const int C = sampler_cluster_size();
+template <typename Kern>
+cudaError_t launch_clusters(Kern kernel, int C, int clusters, size_t smem, const SamplerParams &p,
+                            cudaStream_t stream) {
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(C, rows, 1);
+    cfg.gridDim = dim3(C, clusters, 1);
     cfg.blockDim = dim3(kThreads, 1, 1);
-    cfg.dynamicSmemBytes = kSmemBytes;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute at[1];
     at[0].id = cudaLaunchAttributeClusterDimension;
@@ -1072,7 +1094,18 @@ cudaError_t launch_sampler(const SamplerParams &p, int rows, cudaStream_t stream
     at[0].val.clusterDim.z = 1;
     cfg.attrs = at;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, sampler_kernel, p);
+    return cudaLaunchKernelEx(&cfg, kernel, p);
+}
+
+}  // namespace
+
+cudaError_t launch_sampler(const SamplerParams &p, int rows, cudaStream_t stream) {
+    const int C1 = cluster_size_for(0, sampler_stats_kernel, kStatsSmemBytes);
+    cudaError_t e = launch_clusters(sampler_stats_kernel, C1, rows, kStatsSmemBytes, p, stream);
+    if (e != cudaSuccess) return e;
+    const int C2 = cluster_size_for(1, sampler_draw_kernel, kDrawSmemBytes);
+    const int clusters = p.verify ? p.B * (p.K + 1) : rows;
+    return launch_clusters(sampler_draw_kernel, C2, clusters, kDrawSmemBytes, p, stream);
 }
 
 }  // namespace mtpv

@@ -18,6 +18,22 @@ struct RowStats {
     int status;   // MTPV_ROW_OK or MTPV_ROW_NONFINITE
 };
 
+// Result of one draft position (verify): the token drawn there as if the
+// first rejection were at that position, whether its draft token was
+// accepted, and its status.
+struct PosRecord {
+    int x, accept, status, pad;
+};
+
+// One workspace slot per logits row.  The statistics kernel writes the row's
+// RowStats; in verify mode the draw kernel then replaces the slot of target
+// row i with position i's PosRecord (no one reads that row's statistics
+// afterwards).
+union RowSlot {
+    RowStats st;
+    PosRecord rec;
+};
+
 struct SamplerParams {
     const float *tl;        // verify: target logits [B, K+1, V]; sample: logits [R, V]
     const float *dl;        // verify: draft logits [B, K, V]
@@ -30,13 +46,13 @@ struct SamplerParams {
     int32_t *out_tokens;  // verify: [B, K+1]; sample: [R]
     int32_t *out_acc;     // verify: [B]
     int32_t *row_status;  // verify: [B]; sample: [R]; may be null
-    RowStats *stats;      // [rows]
-    unsigned int *counters;  // verify: [B], zero on entry
-    double *ecache;       // [rows][V]: exp((l_j - m)/T) of every row (T > 0), or null
+    RowSlot *slots;       // [rows]
+    unsigned int *counters;  // verify: [B]; zeroed by the statistics kernel
+    double *ecache;       // [rows][V]: exp((l_j - m)/T) of kept tokens, 0 elsewhere (T > 0), or null
 };
 
-size_t sampler_smem_bytes();
-int sampler_cluster_size();
+// Launches the statistics kernel over `rows` logits rows, then the draw
+// kernel (one cluster per draft position in verify mode, per row otherwise).
 cudaError_t launch_sampler(const SamplerParams &p, int rows, cudaStream_t stream);
 
 }  // namespace mtpv
