@@ -96,11 +96,12 @@ MTPV_API const char *mtpv_status_string(mtpv_status st);
  *           weights are re-read per group).
  *   Kd      reduction length, a positive multiple of 64, at most 58112 (the
  *           kernels stage each activation row in shared memory as fp32).
- *           MTPV_W_INT4_G64 with Kd a multiple of 512 and
- *           (M + 1)(2 Kd + 16) + Kd/2 <= 75776 bytes of staged activations
- *           (M <= 6 at Kd = 5120) runs on the tensor cores (fp16 MMA, exact fp16 dequantisation, fp32
- *           accumulation per 64-weight group); other int4 shapes use a bf16
- *           MMA form with the same accumulation order per group.
+ *           MTPV_W_INT4_G64 runs on the tensor cores (fp16 MMA of exactly
+ *           dequantised nibbles, fp32 accumulation per 64-weight group):
+ *           through per-warp shared-memory rings when Kd is a multiple of
+ *           512, the scales are 16-byte aligned and
+ *           (M + 1)(2 Kd + 16) + Kd/2 <= 75776 bytes (M <= 6 at Kd = 5120),
+ *           else with direct register loads; both forms give the same bits.
  *   N       output columns (vocabulary rows of the head), N >= 1.
  *   w       device weights, layout per fmt:
  *             MTPV_W_BF16:     bf16 [N, Kd] (nn.Linear out x in layout);
@@ -122,6 +123,31 @@ MTPV_API size_t mtpv_lm_head_workspace_bytes(int M, int Kd, int N, mtpv_wfmt fmt
 MTPV_API mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, const void *w,
                                 const void *scales, mtpv_wfmt fmt, float *y, void *ws,
                                 size_t ws_bytes, mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
+ * mtpv_lm_head_pair -- the two projections of a verify step in one call:
+ *
+ *   yt[Mt, N] = xt[Mt, Kd] . W^T            (bf16 head, as MTPV_W_BF16)
+ *   yd[Md, N] = xd[Md, Kd] . deq(wq, s)^T   (int4 group-64 head, as
+ *                                            MTPV_W_INT4_G64)
+ *
+ * Passage: hazakura.dev MTPLX notes, Layer 0 (the target head at full
+ * precision, the draft through a 4-bit copy) and its cached-graph item (one
+ * fixed launch sequence per step).  Arguments as in mtpv_lm_head_smallm, the
+ * same Kd and N for both heads.  When 1 <= Mt <= 4, 1 <= Md <= 8 and the
+ * staged activations fit in shared memory (4 Mt Kd + Md (2 Kd + 16) + Kd/2
+ * <= 232192 bytes; Mt = 4, Md = 3 at Kd = 5120 does), both heads run in ONE
+ * persistent kernel whose warps take items from a single list in which the
+ * int4 tiles are spread evenly among the bf16 row groups, so the int4 head's
+ * dequantisation hides behind the bf16 stream.  Otherwise the call makes the
+ * two mtpv_lm_head_smallm launches.  Either way the values are those
+ * mtpv_lm_head_smallm gives (same arithmetic, bit for bit).
+ * Errors: as mtpv_lm_head_smallm.  ws: mtpv_lm_head_workspace_bytes (0).
+ * ---------------------------------------------------------------------- */
+MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt,
+                                       const void *xd, int Md, const void *wq,
+                                       const void *scales, float *yd, int Kd, int N, void *ws,
+                                       size_t ws_bytes, mtpv_stream stream);
 
 /* ------------------------------------------------------------------------
  * mtpv_verify -- Leviathan-Chen verification of B independent sequences.

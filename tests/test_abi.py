@@ -78,6 +78,25 @@ def _p(v):
     return ctypes.c_void_p(v)
 
 
+def test_lm_head_pair_argument_checks(lib):
+    f = lib.mtpv_lm_head_pair
+    a = 1 << 20  # a fake, aligned device address: never dereferenced on these paths
+    P = _p(a)
+    ok = (P, 4, P, P, P, 3, P, P, P, 5120, 1000, None, 0, None)
+    bad = [
+        (None,) + ok[1:],                              # xt missing
+        ok[:8] + (None,) + ok[9:],                     # yd missing
+        ok[:1] + (0,) + ok[2:],                        # Mt = 0
+        ok[:5] + (65,) + ok[6:],                       # Md > 64
+        ok[:9] + (5000,) + ok[10:],                    # Kd % 64
+        ok[:10] + (0,) + ok[11:],                      # N = 0
+        ok[:2] + (_p(a + 8),) + ok[3:],                # w misaligned
+        ok[:7] + (_p(a + 1),) + ok[8:],                # scales misaligned
+    ]
+    for args in bad:
+        assert f(*args) == INVALID
+
+
 def test_lm_head_argument_checks(lib):
     f = lib.mtpv_lm_head_smallm
     ok = 1 << 20  # a fake, aligned device address: never dereferenced on these paths

@@ -87,6 +87,17 @@ bool lm_head_shape_ok(int M, int Kd, int N) {
 
 char *at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
 
+// Both heads: one fused launch when the kernel takes the shapes, else two.
+cudaError_t launch_heads(const void *xt, int Mt, const void *w, float *yt, const void *xd, int Md,
+                         const void *wq, const void *scales, float *yd, int Kd, int N,
+                         cudaStream_t s) {
+    if (mtpv::lm_heads_pair_ok(Mt, Md, Kd, scales))
+        return mtpv::launch_lm_heads_pair(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, s);
+    cudaError_t e = mtpv::launch_lm_head(xt, Mt, Kd, N, w, nullptr, MTPV_W_BF16, yt, s);
+    if (e != cudaSuccess) return e;
+    return mtpv::launch_lm_head(xd, Md, Kd, N, wq, scales, MTPV_W_INT4_G64, yd, s);
+}
+
 mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *drafts, const float *ua,
                           const float *us, int B, int K, int V, float T, float top_p,
                           int32_t *out_tokens, int32_t *out_acc, int32_t *row_status, void *ws,
@@ -146,6 +157,19 @@ mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, const void 
     if (fmt == MTPV_W_INT4_G64 && (!scales || !aligned(scales, 2))) return MTPV_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 4)) return MTPV_ERR_INVALID_ARG;
     return cuda_status(mtpv::launch_lm_head(x, M, Kd, N, w, scales, (int)fmt, y, (cudaStream_t)stream));
+}
+
+mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
+                              int Md, const void *wq, const void *scales, float *yd, int Kd, int N,
+                              void *ws, size_t ws_bytes, mtpv_stream stream) {
+    (void)ws;
+    (void)ws_bytes;
+    if (!xt || !w || !yt || !xd || !wq || !scales || !yd) return MTPV_ERR_INVALID_ARG;
+    if (!lm_head_shape_ok(Mt, Kd, N) || !lm_head_shape_ok(Md, Kd, N)) return MTPV_ERR_INVALID_ARG;
+    if (!aligned(xt, 16) || !aligned(w, 16) || !aligned(yt, 4) || !aligned(xd, 16) ||
+        !aligned(wq, 16) || !aligned(scales, 2) || !aligned(yd, 4))
+        return MTPV_ERR_INVALID_ARG;
+    return cuda_status(launch_heads(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, (cudaStream_t)stream));
 }
 
 size_t mtpv_verify_workspace_bytes(int B, int K, int V) {
@@ -230,9 +254,8 @@ mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const vo
     cudaStream_t s = (cudaStream_t)stream;
     float *tl = target_logits ? target_logits : reinterpret_cast<float *>(at(ws, l.tl));
     float *dl = draft_logits ? draft_logits : reinterpret_cast<float *>(at(ws, l.dl));
-    cudaError_t e = mtpv::launch_lm_head(h_target, B * (K + 1), h, V, w_target, nullptr, MTPV_W_BF16, tl, s);
-    if (e != cudaSuccess) return cuda_status(e);
-    e = mtpv::launch_lm_head(h_draft, B * K, h, V, w_draft, s_draft, MTPV_W_INT4_G64, dl, s);
+    const cudaError_t e =
+        launch_heads(h_target, B * (K + 1), w_target, tl, h_draft, B * K, w_draft, s_draft, dl, h, V, s);
     if (e != cudaSuccess) return cuda_status(e);
     return launch_verify(tl, dl, draft_tokens, u_accept, u_sample, B, K, V, temperature, top_p,
                          out_tokens, out_accepted, row_status, at(ws, l.verify), s);

@@ -42,104 +42,98 @@ __device__ __forceinline__ int swz8(int k) {
 }
 
 // bf16 weights with the activations staged as fp32 (no per-use widening).
+// Staging: every thread of the block takes part.
+template <int M>
+__device__ __forceinline__ void bf16_stage_x(float *xsf, const uint16_t *__restrict__ x, int Kd) {
+    for (int i = threadIdx.x; i < M * Kd; i += blockDim.x) {
+        const int m = i / Kd, k = i - m * Kd;
+        xsf[m * Kd + swz8(k)] = __uint_as_float((uint32_t)x[i] << 16);
+    }
+}
+
+// One group of RW consecutive weight rows (r0 = g * RW) for the calling warp.
+template <int M, int RW, int U>
+__device__ __forceinline__ void bf16_group(const float *xsf, int Kd, int N,
+                                           const uint16_t *__restrict__ W, float *__restrict__ y,
+                                           int ldy, int g) {
+    const int nch = Kd >> 3;
+    const int lane = threadIdx.x & 31;
+    const int r0 = g * RW;
+    const uint4 *wr[RW];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+        wr[r] = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + r, N - 1) * Kd);
+    float acc[RW][M];
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
+    for (int c0 = lane; c0 < nch; c0 += 32 * U) {
+        uint4 wv[U][RW];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + 32 * u;
+#pragma unroll
+            for (int r = 0; r < RW; ++r)
+                wv[u][r] = (c < nch) ? ld_stream16(wr[r] + c) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int c = c0 + 32 * u;
+            if (c < nch) {
+#pragma unroll
+                for (int m = 0; m < M; ++m) {
+                    const int sw = (c >> 2) & 1;
+                    const float4 a = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 8 + (sw << 2));
+                    const float4 b = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 8 + ((sw ^ 1) << 2));
+#pragma unroll
+                    for (int r = 0; r < RW; ++r) {
+                        const uint4 w = wv[u][r];
+                        float t = acc[r][m];
+                        t = fmaf(a.x, bf16_lo(w.x), t); t = fmaf(a.y, bf16_hi(w.x), t);
+                        t = fmaf(a.z, bf16_lo(w.y), t); t = fmaf(a.w, bf16_hi(w.y), t);
+                        t = fmaf(b.x, bf16_lo(w.z), t); t = fmaf(b.y, bf16_hi(w.z), t);
+                        t = fmaf(b.z, bf16_lo(w.w), t); t = fmaf(b.w, bf16_hi(w.w), t);
+                        acc[r][m] = t;
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < RW; ++r)
+#pragma unroll
+        for (int m = 0; m < M; ++m) {
+            const float v = warp_sum(acc[r][m]);
+            if (lane == 0 && r0 + r < N) y[(size_t)m * ldy + r0 + r] = v;
+        }
+}
+
 template <int M, int RW, int U>
 __global__ void __launch_bounds__(kGemvThreads) lm_head_bf16_xf32_kernel(
     const uint16_t *__restrict__ x, int Kd, int N, const uint16_t *__restrict__ W,
     float *__restrict__ y, int ldy) {
     extern __shared__ float xsf[];  // [M][Kd]
-    for (int i = threadIdx.x; i < M * Kd; i += kGemvThreads) {
-        const int m = i / Kd, k = i - m * Kd;
-        xsf[m * Kd + swz8(k)] = __uint_as_float((uint32_t)x[i] << 16);
-    }
+    bf16_stage_x<M>(xsf, x, Kd);
     __syncthreads();
-    const int nch = Kd >> 3;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int groups = (N + RW - 1) / RW;
-    for (int g = blockIdx.x * kGemvWarps + warp; g < groups; g += gridDim.x * kGemvWarps) {
-        const int r0 = g * RW;
-        const uint4 *wr[RW];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-            wr[r] = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + r, N - 1) * Kd);
-        float acc[RW][M];
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
-        for (int c0 = lane; c0 < nch; c0 += 32 * U) {
-            uint4 wv[U][RW];
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-#pragma unroll
-                for (int r = 0; r < RW; ++r)
-                    wv[u][r] = (c < nch) ? ld_stream16(wr[r] + c) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int c = c0 + 32 * u;
-                if (c < nch) {
-#pragma unroll
-                    for (int m = 0; m < M; ++m) {
-                        const int sw = (c >> 2) & 1;
-                        const float4 a = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 8 + (sw << 2));
-                        const float4 b = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 8 + ((sw ^ 1) << 2));
-#pragma unroll
-                        for (int r = 0; r < RW; ++r) {
-                            const uint4 w = wv[u][r];
-                            float t = acc[r][m];
-                            t = fmaf(a.x, bf16_lo(w.x), t); t = fmaf(a.y, bf16_hi(w.x), t);
-                            t = fmaf(a.z, bf16_lo(w.y), t); t = fmaf(a.w, bf16_hi(w.y), t);
-                            t = fmaf(b.x, bf16_lo(w.z), t); t = fmaf(b.y, bf16_hi(w.z), t);
-                            t = fmaf(b.z, bf16_lo(w.w), t); t = fmaf(b.w, bf16_hi(w.w), t);
-                            acc[r][m] = t;
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int r = 0; r < RW; ++r)
-#pragma unroll
-            for (int m = 0; m < M; ++m) {
-                const float v = warp_sum(acc[r][m]);
-                if (lane == 0 && r0 + r < N) y[(size_t)m * ldy + r0 + r] = v;
-            }
-    }
+    for (int g = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); g < groups; g += gridDim.x * kGemvWarps)
+        bf16_group<M, RW, U>(xsf, Kd, N, W, y, ldy, g);
 }
 
 // ---------------------------------------------------------------------------
-// int4 group-64 weights on the tensor cores (mma.sync m16n8k16, bf16 in,
-// fp32 accumulate), direct-load form: the fallback for shapes the fp16 ring
-// kernel below does not take.  The weights are the A
-// operand (16 vocabulary rows x 16 k), the activations the B operand (k x 8
-// activation rows).  Dequantisation writes the A registers directly: one
-// LOP3 per two weights, ((w >> 4j) & 0x000F000F) | 0x43004300 is the bf16
-// pair (128 + n_j, 128 + n_{j+4}), exact.  Each 64-weight group gets a fresh
-// accumulator so its scale applies exactly; the +128 offset is removed with
-// the group's activation sum: sum (n - 8) x = sum (128 + n) x - 136 sum x.
-//
-// Lane (g = lane/4, t = lane%4) loads 8 bytes (16 nibbles, physical k
-// 16t..16t+15 of the group) of rows g and g+8 of the 16-row block.  MMA j
-// (j = 0..3) of a group takes, for logical k (2t, 2t+1, 2t+8, 2t+9), the
-// physical k (16t + j, +4, +8, +12); the activations are stored in shared
-// memory already in that order, so each lane's B fragments for the 4 MMAs of
-// a group are 32 contiguous bytes.  Rows of that layout are padded to an odd
-// number of 16-byte chunks, which keeps the 128-bit loads conflict-free.
+// int4 group-64 weights on the tensor cores (mma.sync m16n8k16, fp32
+// accumulate).  The weights are the A operand (16 vocabulary rows x 16 k), the
+// activations the B operand (k x 8 activation rows).  Lane (g = lane/4,
+// t = lane%4) holds 8 bytes (16 nibbles, physical k 16t..16t+15 of a 64-weight
+// group) of rows g and g+8 of a 16-row tile.  MMA j (j = 0..3) of a group
+// takes, for logical k (2t, 2t+1, 2t+8, 2t+9), the physical k (16t + j, +4,
+// +8, +12); the activations are staged in shared memory already in that
+// order, so each lane's B fragments for the 4 MMAs of a group are 32
+// contiguous bytes.  Staged rows are padded to an odd number of 16-byte
+// chunks, which keeps the 128-bit loads conflict-free.  Each group gets a
+// fresh accumulator so its bf16 scale applies exactly.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
-                                               uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
-        "{%8,%9}, {%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t nib_pair_bf16(uint32_t w, int j) {
-    return ((w >> (4 * j)) & 0x000F000Fu) | 0x43004300u;
-}
-
 __device__ __forceinline__ uint2 ld_stream8(const void *p) {
     uint2 r;
     asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v2.u32 {%0,%1}, [%2];"
@@ -148,116 +142,13 @@ __device__ __forceinline__ uint2 ld_stream8(const void *p) {
     return r;
 }
 
-// Position (in bf16 units, within one activation row of the staged layout) of
-// activation k: group G, quad t, MMA j, slot s with k % 64 = 16t + j + 4s.
+// Position (in 16-bit units, within one activation row of the staged layout)
+// of activation k: group G, quad t, MMA j, slot s with k % 64 = 16t + j + 4s.
 __device__ __forceinline__ int mma_x_pos(int k) {
     const int G = k >> 6, kk = k & 63;
     const int t = kk >> 4, w = kk & 15;
     const int j = w & 3, sl = w >> 2;
     return G * 64 + t * 16 + j * 4 + sl;
-}
-
-template <int RB, int U>
-__global__ void __launch_bounds__(kGemvThreads) lm_head_int4_mma_kernel(
-    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint8_t *__restrict__ Wq,
-    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
-    extern __shared__ uint4 smem_mma[];
-    const int Gt = Kd >> 6;
-    const int rowc = Gt * 8 + 1;  // 16-byte chunks per staged activation row (odd)
-    uint16_t *xb = reinterpret_cast<uint16_t *>(smem_mma);                   // [M][rowc * 8]
-    float *xs = reinterpret_cast<float *>(smem_mma + M * rowc);              // [Gt][8]
-    // stage: permuted bf16 activations of the M real rows, and group sums
-    for (int i = threadIdx.x; i < M * Kd; i += kGemvThreads) {
-        const int m = i / Kd, k = i - m * Kd;
-        xb[m * rowc * 8 + mma_x_pos(k)] = x[i];
-    }
-    for (int i = threadIdx.x; i < Gt * 8; i += kGemvThreads) {
-        const int G = i >> 3, m = i & 7;
-        float sum = 0.0f;
-        if (m < M)
-            for (int k = 0; k < 64; ++k) sum += __uint_as_float((uint32_t)x[m * Kd + G * 64 + k] << 16);
-        xs[i] = sum;
-    }
-    __syncthreads();
-
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int g = lane >> 2, t = lane & 3;
-    const int rowbytes = Kd >> 1;
-    const bool has_row = g < M;                // lanes g >= M feed zero activations
-    const uint4 *xrow = smem_mma + (has_row ? g : 0) * rowc;
-    const int nblk = (N + 15) / 16;
-    const int ntask = (nblk + RB - 1) / RB;
-    for (int task = blockIdx.x * kGemvWarps + warp; task < ntask; task += gridDim.x * kGemvWarps) {
-        const uint8_t *wr[RB][2];
-        const uint16_t *sr[RB][2];
-#pragma unroll
-        for (int rb = 0; rb < RB; ++rb)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-                const int row = min((task * RB + rb) * 16 + g + 8 * h, N - 1);
-                wr[rb][h] = Wq + (size_t)row * rowbytes + 8 * t;
-                sr[rb][h] = S + (size_t)row * Gt;
-            }
-        float acc[RB][4];
-#pragma unroll
-        for (int rb = 0; rb < RB; ++rb)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) acc[rb][e] = 0.0f;
-
-        for (int G0 = 0; G0 < Gt; G0 += U) {
-            uint2 wv[U][RB][2];
-            float sc[U][RB][2];
-#pragma unroll
-            for (int u = 0; u < U; ++u)
-#pragma unroll
-                for (int rb = 0; rb < RB; ++rb)
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const int G = G0 + u;
-                        wv[u][rb][h] = G < Gt ? ld_stream8(wr[rb][h] + G * 32) : make_uint2(0, 0);
-                        sc[u][rb][h] = G < Gt ? __uint_as_float((uint32_t)__ldg(sr[rb][h] + G) << 16) : 0.0f;
-                    }
-#pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int G = G0 + u;
-                if (G < Gt) {
-                    const uint4 z4 = make_uint4(0, 0, 0, 0);
-                    const uint4 bA = has_row ? xrow[G * 8 + 2 * t] : z4;
-                    const uint4 bB = has_row ? xrow[G * 8 + 2 * t + 1] : z4;
-                    const uint32_t bl[4] = {bA.x, bA.z, bB.x, bB.z};  // b0b1 of MMA j
-                    const uint32_t bh[4] = {bA.y, bA.w, bB.y, bB.w};  // b2b3 of MMA j
-                    const float2 xsum = *reinterpret_cast<const float2 *>(xs + G * 8 + 2 * t);
-#pragma unroll
-                    for (int rb = 0; rb < RB; ++rb) {
-                        float c[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const uint32_t a[4] = {nib_pair_bf16(wv[u][rb][0].x, j),
-                                                   nib_pair_bf16(wv[u][rb][1].x, j),
-                                                   nib_pair_bf16(wv[u][rb][0].y, j),
-                                                   nib_pair_bf16(wv[u][rb][1].y, j)};
-                            mma_bf16_16816(c, a, bl[j], bh[j]);
-                        }
-                        const float s0 = sc[u][rb][0], s1 = sc[u][rb][1];
-                        acc[rb][0] = fmaf(s0, fmaf(-136.0f, xsum.x, c[0]), acc[rb][0]);
-                        acc[rb][1] = fmaf(s0, fmaf(-136.0f, xsum.y, c[1]), acc[rb][1]);
-                        acc[rb][2] = fmaf(s1, fmaf(-136.0f, xsum.x, c[2]), acc[rb][2]);
-                        acc[rb][3] = fmaf(s1, fmaf(-136.0f, xsum.y, c[3]), acc[rb][3]);
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int rb = 0; rb < RB; ++rb) {
-            const int r0 = (task * RB + rb) * 16;
-            const int m0 = 2 * t, m1 = 2 * t + 1;
-            const int ra = r0 + g, rbw = r0 + g + 8;
-            if (m0 < M && ra < N) y[(size_t)m0 * ldy + ra] = acc[rb][0];
-            if (m1 < M && ra < N) y[(size_t)m1 * ldy + ra] = acc[rb][1];
-            if (m0 < M && rbw < N) y[(size_t)m0 * ldy + rbw] = acc[rb][2];
-            if (m1 < M && rbw < N) y[(size_t)m1 * ldy + rbw] = acc[rb][3];
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -284,17 +175,19 @@ struct Int4Ring {
     static constexpr int kWarpBytes = NST * kStageBytes;
 };
 
-// fp16 form of the ring kernel.  A word's nibbles become fp16 pairs with one
-// shift and four LOP3 (Kim et al., "Who Says Elephants Can't Run", 2022; the
-// Marlin kernel, Frantar et al., 2024): the fp16 mantissa holds a nibble at
-// bit 0 or bit 4 of each half, so
-//   (w & 0x000F000F) | 0x64006400 = (1024 + n_j, 1024 + n_{j+4})      j = 0
-//   (w & 0x00F000F0) | 0x64006400 = (1024 + 16 n_j, 1024 + 16 n_{j+4}) j = 1
-// and j = 2, 3 the same on w >> 8.  The activations paired with the j = 1, 3
-// halves are stored divided by 16, and every group's offset term
-// (1032 x or 1152 x/16 per weight) is removed with a precomputed sum.  The
-// activations are fp16, exact after a per-row power-of-two prescale that
-// keeps |x| <= 2^14 (undone on the output).  Layouts as in the bf16 kernels.
+// fp16 dequantisation on the tensor cores.  A word's nibbles become fp16
+// pairs with three shifts and four LOP3 (the magic-number conversion of Kim
+// et al., "Who Says Elephants Can't Run", 2022, and the Marlin kernel,
+// Frantar et al., 2024): with nibble n_j moved to bits 4..7 of the low half
+// and n_{j+4} to bits 4..7 of the high half,
+//   (v & 0x00F000F0) | 0x64006400 = (1024 + 16 n_j, 1024 + 16 n_{j+4})
+// exactly.  Every activation is staged divided by 16, so a weight contributes
+// (64 + n) x, and each group's offset term 72 x (1152 x / 16 per weight) is
+// removed with a precomputed sum: the offset is 72 weight steps, which keeps
+// the fp32 cancellation small (putting the nibble at bit 0 instead would make
+// it 1032 steps).  The activations are fp16, exact after a per-row
+// power-of-two scale that puts the row's largest |x| in [2^9, 2^10) before
+// the division by 16 (undone on the output).  Layouts as in the bf16 kernels.
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
@@ -310,75 +203,81 @@ __device__ __forceinline__ void mma_f16_16816_zc(float (&c)[4], const uint32_t (
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
 
-// the four fp16 pairs of one word (pair j = weights (j, j + 4) of the word)
+// the four fp16 pairs of one word (pair j = weights (j, j + 4) of the word),
+// each (1024 + 16 n_j, 1024 + 16 n_{j+4})
 __device__ __forceinline__ void nib_pairs_f16(uint32_t w, uint32_t (&p)[4]) {
-    const uint32_t w8 = w >> 8;
-    p[0] = (w & 0x000F000Fu) | 0x64006400u;
+    p[0] = ((w << 4) & 0x00F000F0u) | 0x64006400u;
     p[1] = (w & 0x00F000F0u) | 0x64006400u;
-    p[2] = (w8 & 0x000F000Fu) | 0x64006400u;
-    p[3] = (w8 & 0x00F000F0u) | 0x64006400u;
+    p[2] = ((w >> 4) & 0x00F000F0u) | 0x64006400u;
+    p[3] = ((w >> 8) & 0x00F000F0u) | 0x64006400u;
 }
 
-template <int GPS, int NST, int NT>
-__global__ void __launch_bounds__(NT) lm_head_int4_f16_kernel(
-    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint8_t *__restrict__ Wq,
-    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
-    using R = Int4Ring<GPS, NST>;
-    static_assert(GPS % 8 == 0, "scale rows are copied in 16-byte chunks");
-    constexpr int NW = NT / 32;
-    extern __shared__ uint4 smem_mma[];
-    __shared__ unsigned int row_amax[8];
-    __shared__ float row_unscale[8];
+// Activation staging of the fp16 int4 kernels: per-row power-of-two
+// prescale, fp16, permuted (plus, with zero_row, a row of zeros at index M),
+// and the per-group offset sums.  Every thread of the block takes part; the block synchronises inside.
+__device__ __forceinline__ void int4_f16_stage_x(uint16_t *xb, float *xs, unsigned int *row_amax,
+                                                 float *row_unscale, const uint16_t *__restrict__ x,
+                                                 int M, int Kd, bool zero_row) {
     const int Gt = Kd >> 6;
     const int rowc = Gt * 8 + 1;
-    uint16_t *xb = reinterpret_cast<uint16_t *>(smem_mma);                   // [M + 1][rowc * 8] fp16
-    float *xs = reinterpret_cast<float *>(smem_mma + (M + 1) * rowc);        // [Gt][8] offset sums
-    unsigned char *rings = reinterpret_cast<unsigned char *>(xs + Gt * 8);   // [warps][NST][stage]
-
-    // --- stage the activations: per-row power-of-two prescale, fp16, permuted
     if (threadIdx.x < 8) row_amax[threadIdx.x] = 0u;
     __syncthreads();
-    for (int i = threadIdx.x; i < M * Kd; i += NT)
+    for (int i = threadIdx.x; i < M * Kd; i += blockDim.x)
         atomicMax(&row_amax[i / Kd], ((uint32_t)x[i] << 16) & 0x7fffffffu);
-    for (int i = threadIdx.x; i < rowc * 8; i += NT) xb[M * rowc * 8 + i] = 0;
+    if (zero_row)
+        for (int i = threadIdx.x; i < rowc * 8; i += blockDim.x) xb[M * rowc * 8 + i] = 0;
     __syncthreads();
     if (threadIdx.x < 8) {
-        // largest exponent e with 2^e <= max|x|; shift rows above 2^14 down
-        const int e = (int)(row_amax[threadIdx.x] >> 23) - 127;
-        const int sh = e > 13 ? e - 13 : 0;
+        // sh: the row's largest |x| times 2^-sh lies in [2^9, 2^10) (e: the
+        // largest exponent with 2^e <= max|x|); an all-zero row keeps sh = 0
+        const uint32_t amax = row_amax[threadIdx.x];
+        int sh = amax ? (int)(amax >> 23) - 127 - 9 : 0;
+        sh = max(-100, min(100, sh));
         row_unscale[threadIdx.x] = __uint_as_float((uint32_t)(127 + sh) << 23);
-        row_amax[threadIdx.x] = (uint32_t)sh;
+        row_amax[threadIdx.x] = (uint32_t)sh;  // read back as int
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < M * Kd; i += NT) {
+    for (int i = threadIdx.x; i < M * Kd; i += blockDim.x) {
         const int m = i / Kd, k = i - m * Kd;
-        const int j = (k & 15) & 3;
-        const int sh = (int)row_amax[m] + ((j & 1) ? 4 : 0);
+        const int sh = (int)row_amax[m] + 4;  // the row's scale, then / 16
         const float v = __uint_as_float((uint32_t)x[i] << 16) * __uint_as_float((uint32_t)(127 - sh) << 23);
         xb[m * rowc * 8 + mma_x_pos(k)] = __half_as_ushort(__float2half_rn(v));
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < Gt * 8; i += NT) {
+    for (int i = threadIdx.x; i < Gt * 8; i += blockDim.x) {
         const int G = i >> 3, m = i & 7;
         float sum = 0.0f;
         if (m < M)
             for (int k = G * 64; k < G * 64 + 64; ++k) {
                 const float b = __half2float(__ushort_as_half(xb[m * rowc * 8 + mma_x_pos(k)]));
-                sum = fmaf((((k & 15) & 3) & 1) ? 1152.0f : 1032.0f, b, sum);
+                sum = fmaf(1152.0f, b, sum);
             }
         xs[i] = sum;
     }
     __syncthreads();
+}
 
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+// The 16-row tiles of warp gw of nw warps (grid-wide numbering), streamed
+// through the warp's own ring at `ring`.
+template <int GPS, int NST>
+__device__ __forceinline__ void int4_f16_tiles(const uint4 *xstage, const float *xs,
+                                               const float *row_unscale, unsigned char *ring,
+                                               int M, int Kd, int N,
+                                               const uint8_t *__restrict__ Wq,
+                                               const uint16_t *__restrict__ S, float *__restrict__ y,
+                                               int ldy, int gw, int nw) {
+    using R = Int4Ring<GPS, NST>;
+    static_assert(GPS % 8 == 0, "scale rows are copied in 16-byte chunks");
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
     const size_t rowbytes = (size_t)(Kd >> 1);
-    const uint4 *xrow = smem_mma + (g < M ? g : M) * rowc + 2 * t;
+    const uint4 *xrow = xstage + (g < M ? g : M) * rowc + 2 * t;
     const float *xsl = xs + 2 * t;
-    unsigned char *ring = rings + (size_t)warp * R::kWarpBytes;
     const int nblk = (N + 15) / 16;
     const int nst = Gt / GPS;
-    const int first = blockIdx.x * NW + warp, stride = gridDim.x * NW;
+    const int first = gw, stride = nw;
 
     // per-lane copy pattern of a stage: chunk q = lane + 32 i of the 16 x (2 GPS) tile
     constexpr int kCp = GPS;  // 16-byte weight chunks per lane per stage
@@ -486,6 +385,193 @@ __global__ void __launch_bounds__(NT) lm_head_int4_f16_kernel(
     cp_async_wait<0>();
 }
 
+template <int GPS, int NST, int NT>
+__global__ void __launch_bounds__(NT) lm_head_int4_f16_kernel(
+    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint8_t *__restrict__ Wq,
+    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
+    using R = Int4Ring<GPS, NST>;
+    constexpr int NW = NT / 32;
+    extern __shared__ uint4 smem_mma[];
+    __shared__ unsigned int row_amax[8];
+    __shared__ float row_unscale[8];
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    uint16_t *xb = reinterpret_cast<uint16_t *>(smem_mma);                   // [M + 1][rowc * 8] fp16
+    float *xs = reinterpret_cast<float *>(smem_mma + (M + 1) * rowc);        // [Gt][8] offset sums
+    unsigned char *rings = reinterpret_cast<unsigned char *>(xs + Gt * 8);   // [warps][NST][stage]
+    int4_f16_stage_x(xb, xs, row_amax, row_unscale, x, M, Kd, true);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5;
+    int4_f16_tiles<GPS, NST>(smem_mma, xs, row_unscale, rings + (size_t)warp * R::kWarpBytes, M, Kd,
+                             N, Wq, S, y, ldy, blockIdx.x * NW + warp, gridDim.x * NW);
+}
+
+// ---------------------------------------------------------------------------
+// Both heads of a verify step in one persistent launch.  Every warp takes
+// work items from one list in which the int4 tasks (RB 16-row tiles each) are
+// spread evenly among the bf16 row groups, so at any moment most warps stream
+// the bf16 head while a few dequantise the int4 head: the int4 head's
+// dequantisation and latency hide behind the bf16 stream instead of running
+// as a launch of its own.  The int4 task loads its nibbles straight into
+// registers (8 bytes per lane and row per group) and computes exactly as the
+// fp16 ring kernel does (same MMA operands, order and epilogue), and the bf16
+// group is the bf16 kernel's, so each head's logits are bit-identical to its
+// own kernel's.
+// ---------------------------------------------------------------------------
+template <int RB, int UI>
+__device__ __forceinline__ void int4_f16_direct_task(const uint4 *xstage, const float *xs,
+                                                     const float *row_unscale, int M, int Kd, int N,
+                                                     const uint8_t *__restrict__ Wq,
+                                                     const uint16_t *__restrict__ S,
+                                                     float *__restrict__ y, int ldy, int task) {
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    const int lane = threadIdx.x & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const size_t rowbytes = (size_t)(Kd >> 1);
+    const bool has_row = g < M;  // lanes of MMA columns past the last row feed zeros
+    const uint4 *xrow = xstage + (has_row ? g : 0) * rowc + 2 * t;
+    const float *xsl = xs + 2 * t;
+    const uint8_t *wr[RB][2];
+    const uint16_t *sr[RB][2];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int row = min((task * RB + rb) * 16 + g + 8 * h, N - 1);
+            wr[rb][h] = Wq + (size_t)row * rowbytes + 8 * t;
+            sr[rb][h] = S + (size_t)row * Gt;
+        }
+    float acc[RB][4];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[rb][e] = 0.0f;
+    for (int G0 = 0; G0 < Gt; G0 += UI) {
+        uint2 wv[UI][RB][2];
+        float sc[UI][RB][2];
+#pragma unroll
+        for (int u = 0; u < UI; ++u)
+#pragma unroll
+            for (int rb = 0; rb < RB; ++rb)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int G = G0 + u;
+                    wv[u][rb][h] = G < Gt ? ld_stream8(wr[rb][h] + G * 32) : make_uint2(0, 0);
+                    sc[u][rb][h] = G < Gt ? __uint_as_float((uint32_t)__ldg(sr[rb][h] + G) << 16) : 0.0f;
+                }
+#pragma unroll
+        for (int u = 0; u < UI; ++u) {
+            const int G = G0 + u;
+            if (G < Gt) {
+                const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+                const uint4 bA = has_row ? xrow[G * 8] : z4;
+                const uint4 bB = has_row ? xrow[G * 8 + 1] : z4;
+                const float2 corr = *reinterpret_cast<const float2 *>(xsl + G * 8);
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    uint32_t p0x[4], p1x[4], p0y[4], p1y[4];
+                    nib_pairs_f16(wv[u][rb][0].x, p0x);
+                    nib_pairs_f16(wv[u][rb][1].x, p1x);
+                    nib_pairs_f16(wv[u][rb][0].y, p0y);
+                    nib_pairs_f16(wv[u][rb][1].y, p1y);
+                    float c[4];
+                    {
+                        const uint32_t a[4] = {p0x[0], p1x[0], p0y[0], p1y[0]};
+                        mma_f16_16816_zc(c, a, bA.x, bA.y);
+                    }
+                    {
+                        const uint32_t a[4] = {p0x[1], p1x[1], p0y[1], p1y[1]};
+                        mma_f16_16816(c, a, bA.z, bA.w);
+                    }
+                    {
+                        const uint32_t a[4] = {p0x[2], p1x[2], p0y[2], p1y[2]};
+                        mma_f16_16816(c, a, bB.x, bB.y);
+                    }
+                    {
+                        const uint32_t a[4] = {p0x[3], p1x[3], p0y[3], p1y[3]};
+                        mma_f16_16816(c, a, bB.z, bB.w);
+                    }
+                    const float s0 = sc[u][rb][0], s1 = sc[u][rb][1];
+                    acc[rb][0] = fmaf(s0, c[0] - corr.x, acc[rb][0]);
+                    acc[rb][1] = fmaf(s0, c[1] - corr.y, acc[rb][1]);
+                    acc[rb][2] = fmaf(s1, c[2] - corr.x, acc[rb][2]);
+                    acc[rb][3] = fmaf(s1, c[3] - corr.y, acc[rb][3]);
+                }
+            }
+        }
+    }
+    const int m0 = 2 * t, m1 = 2 * t + 1;
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+        const int ra = (task * RB + rb) * 16 + g, rbw = ra + 8;
+        if (m0 < M) {
+            const float us = row_unscale[m0];
+            if (ra < N) y[(size_t)m0 * ldy + ra] = acc[rb][0] * us;
+            if (rbw < N) y[(size_t)m0 * ldy + rbw] = acc[rb][2] * us;
+        }
+        if (m1 < M) {
+            const float us = row_unscale[m1];
+            if (ra < N) y[(size_t)m1 * ldy + ra] = acc[rb][1] * us;
+            if (rbw < N) y[(size_t)m1 * ldy + rbw] = acc[rb][3] * us;
+        }
+    }
+}
+
+// Standalone direct-load fp16 kernel: the int4 shapes the ring kernel does not
+// take (its staging or ring would not fit in shared memory, Kd not a
+// multiple of 512, unaligned scales).  Same arithmetic as the ring kernel.
+template <int RB, int UI>
+__global__ void __launch_bounds__(kGemvThreads) lm_head_int4_f16_direct_kernel(
+    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint8_t *__restrict__ Wq,
+    const uint16_t *__restrict__ S, float *__restrict__ y, int ldy) {
+    extern __shared__ uint4 smem_dir[];
+    __shared__ unsigned int row_amax[8];
+    __shared__ float row_unscale[8];
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    uint16_t *xb = reinterpret_cast<uint16_t *>(smem_dir);               // [M][rowc * 8]
+    float *xs = reinterpret_cast<float *>(smem_dir + (size_t)M * rowc);  // [Gt][8]
+    int4_f16_stage_x(xb, xs, row_amax, row_unscale, x, M, Kd, false);
+    const int tasks = ((N + 15) / 16 + RB - 1) / RB;
+    for (int task = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); task < tasks; task += gridDim.x * kGemvWarps)
+        int4_f16_direct_task<RB, UI>(smem_dir, xs, row_unscale, M, Kd, N, Wq, S, y, ldy, task);
+}
+
+constexpr int kMixWarps = 16;
+constexpr int kMixThreads = 32 * kMixWarps;
+
+template <int MT, int RW, int U, int RB, int UI>
+__global__ void __launch_bounds__(kMixThreads, 1) lm_heads_mixed_kernel(
+    const uint16_t *__restrict__ xt, const uint16_t *__restrict__ W, float *__restrict__ yt,
+    const uint16_t *__restrict__ xd, int Md, const uint8_t *__restrict__ Wq,
+    const uint16_t *__restrict__ S, float *__restrict__ yd, int Kd, int N) {
+    extern __shared__ uint4 smem_mix[];
+    __shared__ unsigned int row_amax[8];
+    __shared__ float row_unscale[8];
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    float *xsf = reinterpret_cast<float *>(smem_mix);                         // [MT][Kd] fp32
+    uint4 *x4 = smem_mix + (size_t)MT * Kd / 4;                               // int4 staging
+    uint16_t *xb = reinterpret_cast<uint16_t *>(x4);                          // [Md][rowc * 8]
+    float *xs = reinterpret_cast<float *>(x4 + (size_t)Md * rowc);            // [Gt][8]
+    bf16_stage_x<MT>(xsf, xt, Kd);
+    int4_f16_stage_x(xb, xs, row_amax, row_unscale, xd, Md, Kd, false);  // ends with a block barrier
+    const long long groups = (N + RW - 1) / RW;
+    const long long tasks = ((N + 15) / 16 + RB - 1) / RB;
+    const long long items = groups + tasks;
+    const int nw = gridDim.x * kMixWarps;
+    for (long long k = blockIdx.x * kMixWarps + (threadIdx.x >> 5); k < items; k += nw) {
+        // item k is an int4 task iff floor((k+1) T / I) > floor(k T / I): the
+        // tasks are spread evenly; floor(k T / I) items before k are tasks
+        const long long before = k * tasks / items;
+        if ((k + 1) * tasks / items > before)
+            int4_f16_direct_task<RB, UI>(x4, xs, row_unscale, Md, Kd, N, Wq, S, yd, N, (int)before);
+        else
+            bf16_group<MT, RW, U>(xsf, Kd, N, W, yt, N, (int)(k - before));
+    }
+}
+
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -506,8 +592,8 @@ static cudaError_t launch_bf16(const uint16_t *x, int Kd, int N, const uint16_t 
     return cudaGetLastError();
 }
 
-// Shared memory of the direct-load tensor-core int4 kernel for M (<= 8) rows.
-static size_t int4_mma_smem(int M, int Kd) {
+// Shared memory of the direct-load fp16 int4 kernel for M (<= 8) rows.
+static size_t int4_direct_smem(int M, int Kd) {
     const size_t Gt = (size_t)Kd / 64;
     return (size_t)M * (Gt * 8 + 1) * 16 + Gt * 8 * sizeof(float);
 }
@@ -538,11 +624,11 @@ static cudaError_t launch_int4_f16(const uint16_t *x, int M, int Kd, int N, cons
     return cudaGetLastError();
 }
 
-static cudaError_t launch_int4_mma(const uint16_t *x, int M, int Kd, int N, const uint8_t *Wq,
-                                   const uint16_t *S, float *y, int ldy, cudaStream_t s) {
-    constexpr int RB = 2, U = 4;
-    auto k = lm_head_int4_mma_kernel<RB, U>;
-    const size_t smem = int4_mma_smem(M, Kd);
+static cudaError_t launch_int4_direct(const uint16_t *x, int M, int Kd, int N, const uint8_t *Wq,
+                                      const uint16_t *S, float *y, int ldy, cudaStream_t s) {
+    constexpr int RB = 2, UI = 4;
+    auto k = lm_head_int4_f16_direct_kernel<RB, UI>;
+    const size_t smem = int4_direct_smem(M, Kd);
     int occ = 0;
     cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ);
     if (e != cudaSuccess) return e;
@@ -551,6 +637,44 @@ static cudaError_t launch_int4_mma(const uint16_t *x, int M, int Kd, int N, cons
     const int grid = std::min(need, kSMs * occ);
     k<<<grid, kGemvThreads, smem, s>>>(x, M, Kd, N, Wq, S, y, ldy);
     return cudaGetLastError();
+}
+
+static size_t heads_pair_smem(int Mt, int Md, int Kd) {
+    const size_t Gt = (size_t)Kd / 64;
+    return (size_t)Mt * Kd * sizeof(float) + (size_t)Md * (Gt * 8 + 1) * 16 + Gt * 8 * sizeof(float);
+}
+
+bool lm_heads_pair_ok(int Mt, int Md, int Kd, const void *scales) {
+    (void)scales;
+    return Mt >= 1 && Mt <= 4 && Md >= 1 && Md <= 8 && heads_pair_smem(Mt, Md, Kd) <= (size_t)227 * 1024 - 256;
+}
+
+template <int MT>
+static cudaError_t launch_pair(const uint16_t *xt, const uint16_t *W, float *yt, const uint16_t *xd,
+                               int Md, const uint8_t *Wq, const uint16_t *S, float *yd, int Kd,
+                               int N, cudaStream_t s) {
+    auto k = lm_heads_mixed_kernel<MT, 4, 4, 2, 4>;
+    const size_t smem = heads_pair_smem(MT, Md, Kd);
+    int occ = 0;
+    cudaError_t e = kernel_setup((const void *)k, kMixThreads, smem, &occ);
+    if (e != cudaSuccess) return e;
+    k<<<kSMs * occ, kMixThreads, smem, s>>>(xt, W, yt, xd, Md, Wq, S, yd, Kd, N);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
+                                 int Md, const void *wq, const void *scales, float *yd, int Kd,
+                                 int N, cudaStream_t s) {
+    if (!lm_heads_pair_ok(Mt, Md, Kd, scales)) return cudaErrorInvalidValue;
+    const uint16_t *xt16 = static_cast<const uint16_t *>(xt), *xd16 = static_cast<const uint16_t *>(xd);
+    const uint16_t *W = static_cast<const uint16_t *>(w), *S = static_cast<const uint16_t *>(scales);
+    const uint8_t *Wq = static_cast<const uint8_t *>(wq);
+    switch (Mt) {
+        case 1: return launch_pair<1>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
+        case 2: return launch_pair<2>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
+        case 3: return launch_pair<3>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
+        default: return launch_pair<4>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
+    }
 }
 
 size_t lm_head_max_smem_rows(int Kd) {
@@ -588,8 +712,8 @@ cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, c
                 if (e != cudaSuccess) return e;
                 continue;
             }
-            if (int4_mma_smem(mm, Kd) <= (size_t)227 * 1024) {
-                e = launch_int4_mma(xm, mm, Kd, N, Wq, S, ym, N, s);
+            if (int4_direct_smem(mm, Kd) <= (size_t)227 * 1024) {
+                e = launch_int4_direct(xm, mm, Kd, N, Wq, S, ym, N, s);
                 if (e != cudaSuccess) return e;
                 continue;
             }

@@ -14,4 +14,13 @@ size_t lm_head_max_smem_rows(int Kd);
 cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, const void *scales,
                            int fmt, float *y, cudaStream_t s);
 
+// Both heads of a verify step in one launch: yt[Mt, N] = xt . W^T (bf16 head)
+// and yd[Md, N] = xd . deq(Wq, S)^T (int4 group-64 head), same Kd and N.
+// lm_heads_pair_ok tells whether the fused kernel takes these shapes and
+// pointers; otherwise the heads run as two launch_lm_head calls.
+bool lm_heads_pair_ok(int Mt, int Md, int Kd, const void *scales);
+cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
+                                 int Md, const void *wq, const void *scales, float *yd, int Kd,
+                                 int N, cudaStream_t s);
+
 }  // namespace mtpv
