@@ -245,7 +245,8 @@ def run_gpu(args, c, rank, world, local_rank):
     ws = mtpv.workspace(mtpv.verify_step_workspace_bytes(B, K, V, h), dev)
     # the step runs both heads in one launch when the fused kernel takes the shapes
     fused = B * (K + 1) <= 4 and B * K <= 8 and h % 512 == 0 and \
-        (B * (K + 1) * h * 4 + (B * K + 1) * (h // 8 + 1) * 16 + h // 2 + 8 * 13056) <= 227 * 1024 - 256
+        (B * (K + 1) * h * 4 + (B * K + 1) * (h // 8 + 1) * 16 + h // 2 + 4 * 13056) <= 227 * 1024 - 256
+    pws = mtpv.workspace(mtpv.load().mtpv_lm_head_pair_workspace_bytes(B * (K + 1), B * K, h, V), dev)
     vws = mtpv.workspace(mtpv.verify_workspace_bytes(B, K, V), dev)
     stream = torch.cuda.current_stream(dev)
 
@@ -293,7 +294,7 @@ def run_gpu(args, c, rank, world, local_rank):
             j = i % POOL
             ev = evs[i]
             ev[0].record(stream)
-            mtpv.lm_head_pair(ht[j], W, tl.view(B * (K + 1), V), hd[j], Wq, S, dl.view(B * K, V))
+            mtpv.lm_head_pair(ht[j], W, tl.view(B * (K + 1), V), hd[j], Wq, S, dl.view(B * K, V), ws=pws)
             ev[1].record(stream)
             mtpv.verify(tl, dl, dr[j], ua[j], us[j], T, top_p, ot, oa, rs, ws=vws)
             ev[2].record(stream)
@@ -405,7 +406,7 @@ def run_gpu(args, c, rank, world, local_rank):
                    "config_name": args.config},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak, "traffic": None,
-                     "kernel": "lm_heads_pair_kernel (both heads, one launch)" if fused
+                     "kernel": "lm_heads_mixed_kernel (both heads, one launch)" if fused
                                else "lm_head_bf16_xf32_kernel + lm_head_int4_f16_kernel",
                      "algorithmic_bytes_per_launch": heads_bytes, "peak_source": peak_kind},
         "step_roofline": {"achieved": sb["total"] / (step_ms * 1e-3) / 1e9, "peak": peak,

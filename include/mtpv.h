@@ -134,16 +134,22 @@ MTPV_API mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, co
  * Passage: hazakura.dev MTPLX notes, Layer 0 (the target head at full
  * precision, the draft through a 4-bit copy) and its cached-graph item (one
  * fixed launch sequence per step).  Arguments as in mtpv_lm_head_smallm, the
- * same Kd and N for both heads.  When 1 <= Mt <= 4, 1 <= Md <= 8 and the
- * staged activations fit in shared memory (4 Mt Kd + Md (2 Kd + 16) + Kd/2
- * <= 232192 bytes; Mt = 4, Md = 3 at Kd = 5120 does), both heads run in ONE
- * persistent kernel whose warps take items from a single list in which the
- * int4 tiles are spread evenly among the bf16 row groups, so the int4 head's
- * dequantisation hides behind the bf16 stream.  Otherwise the call makes the
- * two mtpv_lm_head_smallm launches.  Either way the values are those
- * mtpv_lm_head_smallm gives (same arithmetic, bit for bit).
- * Errors: as mtpv_lm_head_smallm.  ws: mtpv_lm_head_workspace_bytes (0).
+ * same Kd and N for both heads.  When 1 <= Mt <= 4, 1 <= Md <= 8, Kd is a
+ * multiple of 512, the scales are 16-byte aligned and the staging fits in
+ * shared memory (4 Mt Kd + (Md + 1)(2 Kd + 16) + Kd/2 + 52224 <= 232192
+ * bytes; Mt = 4, Md = 3 at Kd = 5120 does), both heads run in ONE persistent
+ * kernel: 4 of every CTA's 16 warps first stream the int4 head through their
+ * shared-memory rings (bound by dequantisation, not by HBM) and then join
+ * the other 12 on the bf16 head, whose row groups every warp takes one at a
+ * time from a counter in `ws`, so the bf16 stream keeps HBM busy to the
+ * end.  Otherwise the call makes the two mtpv_lm_head_smallm launches.
+ * Either way the values are those mtpv_lm_head_smallm gives (same
+ * arithmetic, bit for bit).
+ * ws, ws_bytes: at least mtpv_lm_head_pair_workspace_bytes() bytes (256),
+ * 4-byte aligned; need not be initialised (the call clears its counter on
+ * `stream`).  Errors: as mtpv_lm_head_smallm, and MTPV_ERR_WORKSPACE.
  * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_lm_head_pair_workspace_bytes(int Mt, int Md, int Kd, int N);
 MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt,
                                        const void *xd, int Md, const void *wq,
                                        const void *scales, float *yd, int Kd, int N, void *ws,

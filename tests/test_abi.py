@@ -95,6 +95,10 @@ def test_lm_head_pair_argument_checks(lib):
     ]
     for args in bad:
         assert f(*args) == INVALID
+    assert f(*ok) == 3                                           # no workspace: MTPV_ERR_WORKSPACE
+    assert f(*(ok[:11] + (P, 255, None))) == 3                   # workspace too small
+    assert lib.mtpv_lm_head_pair_workspace_bytes(4, 3, 5120, 151936) == 256
+    assert lib.mtpv_lm_head_pair_workspace_bytes(4, 3, 5000, 151936) == 0
 
 
 def test_lm_head_argument_checks(lib):

@@ -50,6 +50,7 @@ def load() -> ctypes.CDLL:
         "mtpv_status_string": ([I], ctypes.c_char_p),
         "mtpv_lm_head_workspace_bytes": ([I, I, I, I], Z),
         "mtpv_lm_head_smallm": ([P, I, I, I, P, P, I, P, P, Z, P], I),
+        "mtpv_lm_head_pair_workspace_bytes": ([I, I, I, I], Z),
         "mtpv_lm_head_pair": ([P, I, P, P, P, I, P, P, P, I, I, P, Z, P], I),
         "mtpv_verify_workspace_bytes": ([I, I, I], Z),
         "mtpv_verify": ([P, P, P, P, P, I, I, I, F, F, P, P, P, P, Z, P], I),
@@ -141,7 +142,9 @@ def lm_head_pair(xt, w, yt, xd, wq, scales, yd, ws=None, stream=None):
     Mt, Kd = xt.shape
     Md = xd.shape[0]
     N = w.shape[0]
-    wsb = 0 if ws is None else ws.numel() * ws.element_size()
+    if ws is None:
+        ws = workspace(load().mtpv_lm_head_pair_workspace_bytes(Mt, Md, Kd, N), xt.device)
+    wsb = ws.numel() * ws.element_size()
     _check("mtpv_lm_head_pair", load().mtpv_lm_head_pair(
         _ptr(xt), Mt, _ptr(w), _ptr(yt), _ptr(xd), Md, _ptr(wq), _ptr(scales), _ptr(yd), Kd, N,
         _ptr(ws), wsb, _stream(stream)))

@@ -42,11 +42,12 @@ VerifyWs verify_layout(int B, int K, int V) {
 }
 
 struct StepWs {
-    size_t tl, dl, verify, total;
+    size_t heads, tl, dl, verify, total;
 };
 StepWs step_layout(int B, int K, int V) {
     StepWs l;
-    l.tl = 0;
+    l.heads = 0;  // the fused heads kernel's work counter
+    l.tl = l.heads + up(mtpv::kHeadsPairWorkBytes);
     l.dl = l.tl + up(sizeof(float) * (size_t)B * (K + 1) * V);
     l.verify = l.dl + up(sizeof(float) * (size_t)B * K * V);
     l.total = l.verify + verify_layout(B, K, V).total;
@@ -89,10 +90,10 @@ char *at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
 
 // Both heads: one fused launch when the kernel takes the shapes, else two.
 cudaError_t launch_heads(const void *xt, int Mt, const void *w, float *yt, const void *xd, int Md,
-                         const void *wq, const void *scales, float *yd, int Kd, int N,
+                         const void *wq, const void *scales, float *yd, int Kd, int N, void *work,
                          cudaStream_t s) {
     if (mtpv::lm_heads_pair_ok(Mt, Md, Kd, scales))
-        return mtpv::launch_lm_heads_pair(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, s);
+        return mtpv::launch_lm_heads_pair(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, work, s);
     cudaError_t e = mtpv::launch_lm_head(xt, Mt, Kd, N, w, nullptr, MTPV_W_BF16, yt, s);
     if (e != cudaSuccess) return e;
     return mtpv::launch_lm_head(xd, Md, Kd, N, wq, scales, MTPV_W_INT4_G64, yd, s);
@@ -159,17 +160,21 @@ mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, const void 
     return cuda_status(mtpv::launch_lm_head(x, M, Kd, N, w, scales, (int)fmt, y, (cudaStream_t)stream));
 }
 
+size_t mtpv_lm_head_pair_workspace_bytes(int Mt, int Md, int Kd, int N) {
+    if (!lm_head_shape_ok(Mt, Kd, N) || !lm_head_shape_ok(Md, Kd, N)) return 0;
+    return mtpv::kHeadsPairWorkBytes;
+}
+
 mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
                               int Md, const void *wq, const void *scales, float *yd, int Kd, int N,
                               void *ws, size_t ws_bytes, mtpv_stream stream) {
-    (void)ws;
-    (void)ws_bytes;
     if (!xt || !w || !yt || !xd || !wq || !scales || !yd) return MTPV_ERR_INVALID_ARG;
     if (!lm_head_shape_ok(Mt, Kd, N) || !lm_head_shape_ok(Md, Kd, N)) return MTPV_ERR_INVALID_ARG;
     if (!aligned(xt, 16) || !aligned(w, 16) || !aligned(yt, 4) || !aligned(xd, 16) ||
         !aligned(wq, 16) || !aligned(scales, 2) || !aligned(yd, 4))
         return MTPV_ERR_INVALID_ARG;
-    return cuda_status(launch_heads(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, (cudaStream_t)stream));
+    if (!ws || !aligned(ws, 4) || ws_bytes < mtpv::kHeadsPairWorkBytes) return MTPV_ERR_WORKSPACE;
+    return cuda_status(launch_heads(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, ws, (cudaStream_t)stream));
 }
 
 size_t mtpv_verify_workspace_bytes(int B, int K, int V) {
@@ -254,8 +259,8 @@ mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const vo
     cudaStream_t s = (cudaStream_t)stream;
     float *tl = target_logits ? target_logits : reinterpret_cast<float *>(at(ws, l.tl));
     float *dl = draft_logits ? draft_logits : reinterpret_cast<float *>(at(ws, l.dl));
-    const cudaError_t e =
-        launch_heads(h_target, B * (K + 1), w_target, tl, h_draft, B * K, w_draft, s_draft, dl, h, V, s);
+    const cudaError_t e = launch_heads(h_target, B * (K + 1), w_target, tl, h_draft, B * K, w_draft,
+                                       s_draft, dl, h, V, at(ws, l.heads), s);
     if (e != cudaSuccess) return cuda_status(e);
     return launch_verify(tl, dl, draft_tokens, u_accept, u_sample, B, K, V, temperature, top_p,
                          out_tokens, out_accepted, row_status, at(ws, l.verify), s);

@@ -538,14 +538,24 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_int4_f16_direct_kernel(
         int4_f16_direct_task<RB, UI>(smem_dir, xs, row_unscale, M, Kd, N, Wq, S, y, ldy, task);
 }
 
-constexpr int kMixWarps = 16;
+constexpr int kMixWarps = 16;      // per CTA, one CTA per SM
+constexpr int kMixInt4Warps = 4;   // the last 4 warps of a CTA own int4 rings
 constexpr int kMixThreads = 32 * kMixWarps;
 
-template <int MT, int RW, int U, int RB, int UI>
+// Both heads of a verify step in one persistent launch.  The last
+// kMixInt4Warps warps of every CTA first stream their share of the int4 head
+// through their cp.async rings (bound by dequantisation and copy latency, not
+// by HBM), then join the other warps on the bf16 head, whose 4-row groups all
+// warps take one at a time from a global counter (`work`, zero on entry), so
+// the bf16 stream keeps every SM busy to the end whatever the int4 warps'
+// speed.  Each head's values are bit-identical to its own kernel's (same
+// device functions).
+template <int MT, int RW, int U, int GPS, int NST>
 __global__ void __launch_bounds__(kMixThreads, 1) lm_heads_mixed_kernel(
     const uint16_t *__restrict__ xt, const uint16_t *__restrict__ W, float *__restrict__ yt,
     const uint16_t *__restrict__ xd, int Md, const uint8_t *__restrict__ Wq,
-    const uint16_t *__restrict__ S, float *__restrict__ yd, int Kd, int N) {
+    const uint16_t *__restrict__ S, float *__restrict__ yd, int Kd, int N, unsigned int *work) {
+    using R = Int4Ring<GPS, NST>;
     extern __shared__ uint4 smem_mix[];
     __shared__ unsigned int row_amax[8];
     __shared__ float row_unscale[8];
@@ -553,22 +563,24 @@ __global__ void __launch_bounds__(kMixThreads, 1) lm_heads_mixed_kernel(
     const int rowc = Gt * 8 + 1;
     float *xsf = reinterpret_cast<float *>(smem_mix);                         // [MT][Kd] fp32
     uint4 *x4 = smem_mix + (size_t)MT * Kd / 4;                               // int4 staging
-    uint16_t *xb = reinterpret_cast<uint16_t *>(x4);                          // [Md][rowc * 8]
-    float *xs = reinterpret_cast<float *>(x4 + (size_t)Md * rowc);            // [Gt][8]
+    uint16_t *xb = reinterpret_cast<uint16_t *>(x4);                          // [Md + 1][rowc * 8]
+    float *xs = reinterpret_cast<float *>(x4 + (size_t)(Md + 1) * rowc);      // [Gt][8]
+    unsigned char *rings = reinterpret_cast<unsigned char *>(xs + Gt * 8);    // [int4 warps][NST][stage]
     bf16_stage_x<MT>(xsf, xt, Kd);
-    int4_f16_stage_x(xb, xs, row_amax, row_unscale, xd, Md, Kd, false);  // ends with a block barrier
-    const long long groups = (N + RW - 1) / RW;
-    const long long tasks = ((N + 15) / 16 + RB - 1) / RB;
-    const long long items = groups + tasks;
-    const int nw = gridDim.x * kMixWarps;
-    for (long long k = blockIdx.x * kMixWarps + (threadIdx.x >> 5); k < items; k += nw) {
-        // item k is an int4 task iff floor((k+1) T / I) > floor(k T / I): the
-        // tasks are spread evenly; floor(k T / I) items before k are tasks
-        const long long before = k * tasks / items;
-        if ((k + 1) * tasks / items > before)
-            int4_f16_direct_task<RB, UI>(x4, xs, row_unscale, Md, Kd, N, Wq, S, yd, N, (int)before);
-        else
-            bf16_group<MT, RW, U>(xsf, Kd, N, W, yt, N, (int)(k - before));
+    int4_f16_stage_x(xb, xs, row_amax, row_unscale, xd, Md, Kd, true);  // ends with a block barrier
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int w4 = warp - (kMixWarps - kMixInt4Warps);
+    if (w4 >= 0)
+        int4_f16_tiles<GPS, NST>(x4, xs, row_unscale, rings + (size_t)w4 * R::kWarpBytes, Md, Kd, N,
+                                 Wq, S, yd, N, blockIdx.x * kMixInt4Warps + w4,
+                                 gridDim.x * kMixInt4Warps);
+    const unsigned groups = (unsigned)((N + RW - 1) / RW);
+    for (;;) {
+        unsigned g = 0;
+        if (lane == 0) g = atomicAdd(work, 1u);
+        g = __shfl_sync(0xffffffffu, g, 0);
+        if (g >= groups) break;
+        bf16_group<MT, RW, U>(xsf, Kd, N, W, yt, N, (int)g);
     }
 }
 
@@ -641,39 +653,43 @@ static cudaError_t launch_int4_direct(const uint16_t *x, int M, int Kd, int N, c
 
 static size_t heads_pair_smem(int Mt, int Md, int Kd) {
     const size_t Gt = (size_t)Kd / 64;
-    return (size_t)Mt * Kd * sizeof(float) + (size_t)Md * (Gt * 8 + 1) * 16 + Gt * 8 * sizeof(float);
+    return (size_t)Mt * Kd * sizeof(float) + (size_t)(Md + 1) * (Gt * 8 + 1) * 16 +
+           Gt * 8 * sizeof(float) + (size_t)kMixInt4Warps * Int4Ring<kF16Gps, kF16Nst>::kWarpBytes;
 }
 
 bool lm_heads_pair_ok(int Mt, int Md, int Kd, const void *scales) {
-    (void)scales;
-    return Mt >= 1 && Mt <= 4 && Md >= 1 && Md <= 8 && heads_pair_smem(Mt, Md, Kd) <= (size_t)227 * 1024 - 256;
+    return Mt >= 1 && Mt <= 4 && Md >= 1 && Md <= 8 && Kd % (64 * kF16Gps) == 0 &&
+           ((uintptr_t)scales & 15) == 0 && heads_pair_smem(Mt, Md, Kd) <= (size_t)227 * 1024 - 256;
 }
 
 template <int MT>
 static cudaError_t launch_pair(const uint16_t *xt, const uint16_t *W, float *yt, const uint16_t *xd,
                                int Md, const uint8_t *Wq, const uint16_t *S, float *yd, int Kd,
-                               int N, cudaStream_t s) {
-    auto k = lm_heads_mixed_kernel<MT, 4, 4, 2, 4>;
+                               int N, unsigned int *work, cudaStream_t s) {
+    auto k = lm_heads_mixed_kernel<MT, 4, 4, kF16Gps, kF16Nst>;
     const size_t smem = heads_pair_smem(MT, Md, Kd);
     int occ = 0;
     cudaError_t e = kernel_setup((const void *)k, kMixThreads, smem, &occ);
     if (e != cudaSuccess) return e;
-    k<<<kSMs * occ, kMixThreads, smem, s>>>(xt, W, yt, xd, Md, Wq, S, yd, Kd, N);
+    e = cudaMemsetAsync(work, 0, sizeof(unsigned int), s);
+    if (e != cudaSuccess) return e;
+    k<<<kSMs * occ, kMixThreads, smem, s>>>(xt, W, yt, xd, Md, Wq, S, yd, Kd, N, work);
     return cudaGetLastError();
 }
 
 cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
                                  int Md, const void *wq, const void *scales, float *yd, int Kd,
-                                 int N, cudaStream_t s) {
-    if (!lm_heads_pair_ok(Mt, Md, Kd, scales)) return cudaErrorInvalidValue;
+                                 int N, void *work, cudaStream_t s) {
+    if (!lm_heads_pair_ok(Mt, Md, Kd, scales) || !work) return cudaErrorInvalidValue;
     const uint16_t *xt16 = static_cast<const uint16_t *>(xt), *xd16 = static_cast<const uint16_t *>(xd);
     const uint16_t *W = static_cast<const uint16_t *>(w), *S = static_cast<const uint16_t *>(scales);
     const uint8_t *Wq = static_cast<const uint8_t *>(wq);
+    unsigned int *wk = static_cast<unsigned int *>(work);
     switch (Mt) {
-        case 1: return launch_pair<1>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
-        case 2: return launch_pair<2>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
-        case 3: return launch_pair<3>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
-        default: return launch_pair<4>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, s);
+        case 1: return launch_pair<1>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
+        case 2: return launch_pair<2>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
+        case 3: return launch_pair<3>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
+        default: return launch_pair<4>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
     }
 }
 

@@ -17,10 +17,13 @@ cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, c
 // Both heads of a verify step in one launch: yt[Mt, N] = xt . W^T (bf16 head)
 // and yd[Md, N] = xd . deq(Wq, S)^T (int4 group-64 head), same Kd and N.
 // lm_heads_pair_ok tells whether the fused kernel takes these shapes and
-// pointers; otherwise the heads run as two launch_lm_head calls.
+// pointers; otherwise the heads run as two launch_lm_head calls.  `work` is
+// kHeadsPairWorkBytes of device scratch (the fused kernel's work counter,
+// cleared on the stream before the kernel).
+constexpr size_t kHeadsPairWorkBytes = 256;
 bool lm_heads_pair_ok(int Mt, int Md, int Kd, const void *scales);
 cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
                                  int Md, const void *wq, const void *scales, float *yd, int Kd,
-                                 int N, cudaStream_t s);
+                                 int N, void *work, cudaStream_t s);
 
 }  // namespace mtpv
