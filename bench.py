@@ -49,6 +49,22 @@ POOL = 64
 METRIC = "verify steps/s (K=3, V=151936, h=5120) and achieved HBM GB/s vs roofline"
 
 
+def recorded_traffic(kernel_source: str, profile: str):
+    """DRAM bytes per launch from a committed ncu summary, or None when the
+    kernel's source changed since the counters were taken."""
+    import hashlib
+    try:
+        text = open(os.path.join(ROOT, "profiles", profile)).read()
+        line = next(l for l in text.splitlines() if "traffic_bytes_per_launch=" in l)
+        f = dict(kv.split("=", 1) for kv in line.split())
+        src = open(os.path.join(ROOT, kernel_source), "rb").read()
+        if f.get("sha256") != hashlib.sha256(src).hexdigest():
+            return None
+        return int(f["traffic_bytes_per_launch"])
+    except Exception:
+        return None
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -405,7 +421,10 @@ def run_gpu(args, c, rank, world, local_rank):
                    "l2": "inputs larger than L2: 1.98 GB of head weights streamed per step",
                    "config_name": args.config},
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                     "frac": achieved / peak, "traffic": None,
+                     "frac": achieved / peak,
+                     "traffic": recorded_traffic("verify_step_lm_b200/csrc/lm_head.cu",
+                                                 "lm_heads_mixed_qwen27b.md") if fused and
+                                args.config == "qwen27b" else None,
                      "kernel": "lm_heads_mixed_kernel (both heads, one launch)" if fused
                                else "lm_head_bf16_xf32_kernel + lm_head_int4_f16_kernel",
                      "algorithmic_bytes_per_launch": heads_bytes, "peak_source": peak_kind},
