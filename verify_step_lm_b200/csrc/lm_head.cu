@@ -155,9 +155,11 @@ __device__ __forceinline__ int mma_x_pos(int k) {
 // cp.async ring used by the fp16 int4 kernel: every warp owns NST
 // shared-memory stages, each a 16-row x GPS-group tile of the head (and its
 // scales), filled with 16-byte cp.async copies while the warp computes on an
-// earlier stage.  Tile rows are XOR-swizzled in 16-byte chunks (chunk c of row
-// r at c ^ (r & 7)), so the per-lane 8-byte fragment reads hit every bank pair
-// once.
+// earlier stage.  Tile rows are XOR-swizzled in 16-byte chunks (chunk c of
+// row r at c ^ (r & 7)) and tile row 2i feeds MMA row i, row 2i + 1 MMA row
+// i + 8: the four rows a half-warp reads in one instruction then have four
+// different swizzles, so the per-lane 8-byte fragment reads cover all 32
+// banks once.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
     const unsigned sa = (unsigned)__cvta_generic_to_shared(smem);
@@ -325,17 +327,18 @@ __device__ __forceinline__ void int4_f16_tiles(const uint4 *xstage, const float 
             const unsigned char *slot = ring + slot_i * R::kStageBytes;
             if (++slot_i == NST) slot_i = 0;
             const uint16_t *ssl = reinterpret_cast<const uint16_t *>(slot + R::kTileBytes);
-            const unsigned char *rowg = slot + g * (GPS * 32) + 8 * (t & 1);
-            const unsigned char *rowg8 = rowg + 8 * (GPS * 32);
+            // MMA row g is tile row 2g, MMA row g + 8 is tile row 2g + 1
+            const unsigned char *rowg = slot + (2 * g) * (GPS * 32) + 8 * (t & 1);
+            const unsigned char *rowg8 = rowg + GPS * 32;
             const uint4 *xr = xrow + st * GPS * 8;
             const float *xc = xsl + st * GPS * 8;
 #pragma unroll
             for (int gq = 0; gq < GPS; ++gq) {
-                const int sw = ((2 * gq + (t >> 1)) ^ g) << 4;
+                const int sw = ((2 * gq + (t >> 1)) ^ ((2 * g) & 7)) << 4;
                 const uint2 w0 = *reinterpret_cast<const uint2 *>(rowg + sw);
-                const uint2 w1 = *reinterpret_cast<const uint2 *>(rowg8 + sw);
-                const float s0 = __uint_as_float((uint32_t)ssl[g * GPS + gq] << 16);
-                const float s1 = __uint_as_float((uint32_t)ssl[(g + 8) * GPS + gq] << 16);
+                const uint2 w1 = *reinterpret_cast<const uint2 *>(rowg8 + (sw ^ 16));
+                const float s0 = __uint_as_float((uint32_t)ssl[(2 * g) * GPS + gq] << 16);
+                const float s1 = __uint_as_float((uint32_t)ssl[(2 * g + 1) * GPS + gq] << 16);
                 const uint4 bA = xr[gq * 8];
                 const uint4 bB = xr[gq * 8 + 1];
                 const float2 corr = *reinterpret_cast<const float2 *>(xc + gq * 8);
@@ -370,7 +373,7 @@ __device__ __forceinline__ void int4_f16_tiles(const uint4 *xstage, const float 
         }
         const int r0 = task * 16;
         const int m0 = 2 * t, m1 = 2 * t + 1;
-        const int ra = r0 + g, rbw = r0 + g + 8;
+        const int ra = r0 + 2 * g, rbw = ra + 1;  // MMA rows g, g + 8
         if (m0 < M) {
             const float us = row_unscale[m0];
             if (ra < N) y[(size_t)m0 * ldy + ra] = acc[0] * us;
