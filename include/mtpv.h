@@ -91,9 +91,11 @@ MTPV_API const char *mtpv_status_string(mtpv_status st);
  *   y[m][n] = sum_k x[m][k] * Wd[n][k],  0 <= m < M, 0 <= n < N   (fp32 out)
  *
  *   x       device, bf16 [M, Kd] row-major (activations / hidden states).
- *   M       rows, 1 <= M <= 64.  The kernels are built for M <= 8; larger M is
- *           processed in groups of min(8, floor(232448 / (4 Kd))) rows (the
- *           weights are re-read per group).
+ *   M       rows, 1 <= M <= 64.  MTPV_W_BF16 with M <= 8 streams the head on
+ *           the CUDA cores; with M > 8 (and Kd <= 7232) it runs on the tensor
+ *           cores (mma.sync bf16, fp32 accumulation), 16 rows per pass.
+ *           Other shapes go in groups of min(8, floor(232448 / (4 Kd)))
+ *           rows.  The weights are re-read once per pass or group.
  *   Kd      reduction length, a positive multiple of 64, at most 58112 (the
  *           kernels stage each activation row in shared memory as fp32).
  *           MTPV_W_INT4_G64 runs on the tensor cores (fp16 MMA of exactly
@@ -256,6 +258,38 @@ MTPV_API size_t mtpv_sample_workspace_bytes(int R, int V);
 MTPV_API mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, float top_p,
                         const float *u, int32_t *out, int32_t *row_status, void *ws,
                         size_t ws_bytes, mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
+ * mtpv_draft_loop -- the draft phase that precedes a verify step: K draft
+ * tokens per sequence, one position after the other.
+ *
+ * Passage: hazakura.dev MTPLX notes, Layer 2 "Draft" (the MTP head proposes
+ * K tokens, each drawn from the draft distribution through the 4-bit LM
+ * head) and Layer 0 (the draft head's 4-bit copy of the LM head).  The MTP
+ * head's own transformer layers are outside this library: the caller passes
+ * the draft hidden state of every position.
+ *
+ * For position i = 0..K-1, in order:
+ *   draft_logits[b][i] = h_draft[b][i] . deq(w_draft, s_draft)^T
+ *   out_drafts[b][i]   = one draw from q'_i (temperature + top-p exactly as
+ *                        mtpv_verify; inverse CDF with u_draft[b][i])
+ *
+ *   w_draft, s_draft  int4 group-64 head, as MTPV_W_INT4_G64 [V, h]
+ *   h_draft           device bf16 [B, K, h] (16-byte aligned)
+ *   u_draft           device fp32 [B, K] in [0, 1)
+ *   out_drafts        device int32 [B, K] (-1 for a row with a non-finite logit)
+ *   draft_logits      device fp32 [B, K, V], or NULL (kept in the workspace)
+ *   1 <= B <= 64, 1 <= K <= 16, V and h as mtpv_verify_step.
+ *   ws of at least mtpv_draft_loop_workspace_bytes(B, K, V, h) bytes.
+ * One int4-head launch and the two sampler launches per position (with
+ * B > 1, small copies gather position i's rows); asynchronous on `stream`.
+ * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_draft_loop_workspace_bytes(int B, int K, int V, int h);
+MTPV_API mtpv_status mtpv_draft_loop(const void *w_draft, const void *s_draft, const void *h_draft,
+                                     const float *u_draft, int B, int K, int V, int h,
+                                     float temperature, float top_p, int32_t *out_drafts,
+                                     float *draft_logits, void *ws, size_t ws_bytes,
+                                     mtpv_stream stream);
 
 /* ------------------------------------------------------------------------
  * mtpv_verify_step -- the whole verify step for B sequences in one call:

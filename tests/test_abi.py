@@ -101,6 +101,30 @@ def test_lm_head_pair_argument_checks(lib):
     assert lib.mtpv_lm_head_pair_workspace_bytes(4, 3, 5000, 151936) == 0
 
 
+def test_draft_loop_argument_checks(lib):
+    f = lib.mtpv_draft_loop
+    a = 1 << 20  # a fake, aligned device address: never dereferenced on these paths
+    P = _p(a)
+    need = lib.mtpv_draft_loop_workspace_bytes(1, 3, 151936, 5120)
+    assert need > 0
+    assert lib.mtpv_draft_loop_workspace_bytes(65, 3, 1000, 512) == 0   # B > 64
+    assert lib.mtpv_draft_loop_workspace_bytes(1, 17, 1000, 512) == 0   # K > 16
+    assert lib.mtpv_draft_loop_workspace_bytes(1, 3, 1000, 500) == 0    # h % 64
+    ok = (P, P, P, P, 1, 3, 151936, 5120, 0.6, 0.95, P, None, P, need, None)
+    bad = [
+        (None,) + ok[1:],                          # no weights
+        ok[:4] + (0,) + ok[5:],                    # B = 0
+        ok[:8] + (-1.0,) + ok[9:],                 # T < 0
+        ok[:9] + (0.0,) + ok[10:],                 # top_p = 0
+        ok[:10] + (None,) + ok[11:],               # no output
+        ok[:2] + (_p(a + 8),) + ok[3:],            # h_draft misaligned
+    ]
+    for args in bad:
+        assert f(*args) == INVALID
+    assert f(*(ok[:12] + (None, need, None))) == WORKSPACE
+    assert f(*(ok[:13] + (need - 1, None))) == WORKSPACE
+
+
 def test_lm_head_argument_checks(lib):
     f = lib.mtpv_lm_head_smallm
     ok = 1 << 20  # a fake, aligned device address: never dereferenced on these paths

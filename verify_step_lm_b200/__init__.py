@@ -56,6 +56,8 @@ def load() -> ctypes.CDLL:
         "mtpv_verify": ([P, P, P, P, P, I, I, I, F, F, P, P, P, P, Z, P], I),
         "mtpv_sample_workspace_bytes": ([I, I], Z),
         "mtpv_sample": ([P, I, I, F, F, P, P, P, P, Z, P], I),
+        "mtpv_draft_loop_workspace_bytes": ([I, I, I, I], Z),
+        "mtpv_draft_loop": ([P, P, P, P, I, I, I, I, F, F, P, P, P, Z, P], I),
         "mtpv_verify_step_workspace_bytes": ([I, I, I, I], Z),
         "mtpv_verify_step": ([P, P, P, P, P, P, P, P, I, I, I, I, F, F, P, P, P, P, P, P, Z, P], I),
         "mtpv_verify_step_host_workspace_bytes": ([I, I, I, I], Z),
@@ -174,6 +176,19 @@ def sample(logits, temperature: float, top_p: float, u, out, row_status=None, ws
         _ptr(logits), R, V, float(temperature), float(top_p), _ptr(u), _ptr(out), _ptr(row_status),
         _ptr(ws), ws.numel(), _stream(stream)))
     return out
+
+
+def draft_loop(w_draft, s_draft, h_draft, u_draft, B: int, K: int, temperature: float, top_p: float,
+               out_drafts, draft_logits=None, ws=None, stream=None):
+    """The draft phase: K positions, each an int4-head projection and one draw from q'."""
+    V = w_draft.shape[0]
+    h = h_draft.shape[-1]
+    if ws is None:
+        ws = workspace(load().mtpv_draft_loop_workspace_bytes(B, K, V, h), w_draft.device)
+    _check("mtpv_draft_loop", load().mtpv_draft_loop(
+        _ptr(w_draft), _ptr(s_draft), _ptr(h_draft), _ptr(u_draft), B, K, V, h, float(temperature),
+        float(top_p), _ptr(out_drafts), _ptr(draft_logits), _ptr(ws), ws.numel(), _stream(stream)))
+    return out_drafts
 
 
 def verify_step(w_target, w_draft, s_draft, h_target, h_draft, draft_tokens, u_accept, u_sample,

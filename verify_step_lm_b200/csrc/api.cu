@@ -72,6 +72,26 @@ HostWs host_layout(int B, int K, int V, int h) {
     return l;
 }
 
+// draft loop: per position, the B hidden rows, their logits, uniforms and
+// tokens (B > 1 only: gathered from / scattered to the [B, K] layouts), then
+// the sampler's workspace.
+struct DraftWs {
+    size_t x, y, u, tok, samp, total;
+};
+size_t sample_ws_bytes(int R, int V) {
+    return up(sizeof(mtpv::RowSlot) * (size_t)R) + up(sizeof(double) * (size_t)R * V);
+}
+DraftWs draft_layout(int B, int V, int h) {
+    DraftWs l;
+    l.x = 0;
+    l.y = l.x + up((size_t)B * h * 2);
+    l.u = l.y + up(sizeof(float) * (size_t)B * V);
+    l.tok = l.u + up(sizeof(float) * (size_t)B);
+    l.samp = l.tok + up(sizeof(int32_t) * (size_t)B);
+    l.total = l.samp + sample_ws_bytes(B, V);
+    return l;
+}
+
 bool verify_shape_ok(int B, int K, int V) {
     return B >= 1 && K >= 1 && K <= kMaxK && V >= 1 && V <= kMaxV &&
            (long long)B * (2 * K + 1) <= kMaxRows;
@@ -229,6 +249,72 @@ mtpv_status mtpv_sample(const float *logits, int R, int V, float temperature, fl
     p.counters = nullptr;
     p.ecache = reinterpret_cast<double *>(at(ws, up(sizeof(mtpv::RowSlot) * (size_t)R)));
     return cuda_status(mtpv::launch_sampler(p, R, (cudaStream_t)stream));
+}
+
+size_t mtpv_draft_loop_workspace_bytes(int B, int K, int V, int h) {
+    if (!verify_shape_ok(B, K, V) || B > 64 || h < 64 || h % 64 || !lm_head_shape_ok(B, h, V)) return 0;
+    return draft_layout(B, V, h).total;
+}
+
+mtpv_status mtpv_draft_loop(const void *w_draft, const void *s_draft, const void *h_draft,
+                            const float *u_draft, int B, int K, int V, int h, float temperature,
+                            float top_p, int32_t *out_drafts, float *draft_logits, void *ws,
+                            size_t ws_bytes, mtpv_stream stream) {
+    if (!w_draft || !s_draft || !h_draft || !u_draft || !out_drafts) return MTPV_ERR_INVALID_ARG;
+    if (mtpv_draft_loop_workspace_bytes(B, K, V, h) == 0 || !sampling_params_ok(temperature, top_p))
+        return MTPV_ERR_INVALID_ARG;
+    if (!aligned(w_draft, 16) || !aligned(s_draft, 2) || !aligned(h_draft, 16) ||
+        (draft_logits && !aligned(draft_logits, 4)))
+        return MTPV_ERR_INVALID_ARG;
+    const DraftWs l = draft_layout(B, V, h);
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MTPV_ERR_WORKSPACE;
+    cudaStream_t s = (cudaStream_t)stream;
+    const char *hd = static_cast<const char *>(h_draft);
+    for (int i = 0; i < K; ++i) {
+        // position i: rows b*K + i of the [B, K, ...] inputs
+        const void *x = hd + (size_t)i * h * 2;
+        const float *u = u_draft + i;
+        float *y = draft_logits ? draft_logits + (size_t)i * V : reinterpret_cast<float *>(at(ws, l.y));
+        int32_t *tok = out_drafts + i;
+        cudaError_t e = cudaSuccess;
+        if (B > 1) {
+            x = at(ws, l.x);
+            u = reinterpret_cast<const float *>(at(ws, l.u));
+            y = reinterpret_cast<float *>(at(ws, l.y));
+            tok = reinterpret_cast<int32_t *>(at(ws, l.tok));
+            e = cudaMemcpy2DAsync(at(ws, l.x), (size_t)h * 2, hd + (size_t)i * h * 2, (size_t)K * h * 2,
+                                  (size_t)h * 2, B, cudaMemcpyDeviceToDevice, s);
+            if (e == cudaSuccess)
+                e = cudaMemcpy2DAsync(at(ws, l.u), sizeof(float), u_draft + i, (size_t)K * sizeof(float),
+                                      sizeof(float), B, cudaMemcpyDeviceToDevice, s);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+        e = mtpv::launch_lm_head(x, B, h, V, w_draft, s_draft, MTPV_W_INT4_G64, y, s);
+        if (e != cudaSuccess) return cuda_status(e);
+        mtpv::SamplerParams p = {};
+        p.tl = y;
+        p.u_samp = u;
+        p.B = B;
+        p.V = V;
+        p.T = temperature;
+        p.top_p = top_p;
+        p.verify = 0;
+        p.out_tokens = tok;
+        p.slots = reinterpret_cast<mtpv::RowSlot *>(at(ws, l.samp));
+        p.ecache = reinterpret_cast<double *>(at(ws, l.samp + up(sizeof(mtpv::RowSlot) * (size_t)B)));
+        e = mtpv::launch_sampler(p, B, s);
+        if (e != cudaSuccess) return cuda_status(e);
+        if (B > 1) {
+            e = cudaMemcpy2DAsync(out_drafts + i, (size_t)K * sizeof(int32_t), tok, sizeof(int32_t),
+                                  sizeof(int32_t), B, cudaMemcpyDeviceToDevice, s);
+            if (e == cudaSuccess && draft_logits)
+                e = cudaMemcpy2DAsync(draft_logits + (size_t)i * V, (size_t)K * V * sizeof(float), y,
+                                      (size_t)V * sizeof(float), (size_t)V * sizeof(float), B,
+                                      cudaMemcpyDeviceToDevice, s);
+            if (e != cudaSuccess) return cuda_status(e);
+        }
+    }
+    return MTPV_OK;
 }
 
 size_t mtpv_verify_step_workspace_bytes(int B, int K, int V, int h) {

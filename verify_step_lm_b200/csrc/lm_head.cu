@@ -122,6 +122,98 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_bf16_xf32_kernel(
 }
 
 // ---------------------------------------------------------------------------
+// bf16 head for 9..16 rows on the tensor cores (mma.sync m16n8k16 bf16, fp32
+// accumulate): the weights are the A operand (16 vocabulary rows x 16 k), the
+// activation rows the B operand (k x 8 rows, NT n-tiles).  The reduction
+// index is permuted inside every 32-k step so that each lane's fragments are
+// contiguous: lane (g, t) holds physical k 8t..8t+7 of the step, the first
+// four for the step's first MMA and the last four for its second (logical k
+// 2t, 2t+1, 2t+8, 2t+9 of an MMA are physical 8t + 0..3, or 8t + 4..7).
+// The A fragments are then one 16-byte global load per row, 64 contiguous
+// bytes per row per warp, and the B fragments one 16-byte shared-memory load
+// per n-tile; activation rows are padded by 64 bytes, which puts the two
+// rows of a quarter-warp on different halves of the banks.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                               uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+constexpr int kBmmaThreads = 512;
+
+template <int NT, int U>
+__global__ void __launch_bounds__(kBmmaThreads, 1) lm_head_bf16_mma_kernel(
+    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint16_t *__restrict__ W,
+    float *__restrict__ y, int ldy) {
+    extern __shared__ uint4 smem_bm[];
+    const int pitch = Kd + 32;  // bf16 elements per staged row (64 bytes of padding)
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_bm);
+    for (int i = threadIdx.x; i < M * (Kd / 8); i += blockDim.x) {
+        const int m = i / (Kd / 8), c = i - m * (Kd / 8);
+        *reinterpret_cast<uint4 *>(xs + (size_t)m * pitch + c * 8) =
+            *reinterpret_cast<const uint4 *>(x + (size_t)m * Kd + c * 8);
+    }
+    __syncthreads();
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int nwarps = blockDim.x >> 5;
+    const int ntiles = (N + 15) / 16;
+    const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+    for (int tile = blockIdx.x * nwarps + warp; tile < ntiles; tile += gridDim.x * nwarps) {
+        const int r0 = tile * 16;
+        const uint4 *wa = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + g, N - 1) * Kd) + t;
+        const uint4 *wb = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + g + 8, N - 1) * Kd) + t;
+        float acc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
+        for (int k0 = 0; k0 < Kd; k0 += 32 * U) {
+            uint4 va[U], vb[U];
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const bool in = k0 + 32 * u < Kd;
+                va[u] = in ? ld_stream16(wa + (k0 + 32 * u) / 8) : z4;
+                vb[u] = in ? ld_stream16(wb + (k0 + 32 * u) / 8) : z4;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int k = k0 + 32 * u;
+                if (k < Kd) {
+#pragma unroll
+                    for (int nt = 0; nt < NT; ++nt) {
+                        const int n = nt * 8 + g;
+                        const uint4 xv = n < M ? *reinterpret_cast<const uint4 *>(xs + (size_t)n * pitch + k + 8 * t)
+                                               : z4;
+                        const uint32_t a0[4] = {va[u].x, vb[u].x, va[u].y, vb[u].y};
+                        const uint32_t a1[4] = {va[u].z, vb[u].z, va[u].w, vb[u].w};
+                        mma_bf16_16816(acc[nt], a0, xv.x, xv.y);
+                        mma_bf16_16816(acc[nt], a1, xv.z, xv.w);
+                    }
+                }
+            }
+        }
+        const int ra = r0 + g, rb = ra + 8;
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const int m0 = nt * 8 + 2 * t, m1 = m0 + 1;
+            if (m0 < M) {
+                if (ra < N) y[(size_t)m0 * ldy + ra] = acc[nt][0];
+                if (rb < N) y[(size_t)m0 * ldy + rb] = acc[nt][2];
+            }
+            if (m1 < M) {
+                if (ra < N) y[(size_t)m1 * ldy + ra] = acc[nt][1];
+                if (rb < N) y[(size_t)m1 * ldy + rb] = acc[nt][3];
+            }
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
 // int4 group-64 weights on the tensor cores (mma.sync m16n8k16, fp32
 // accumulate).  The weights are the A operand (16 vocabulary rows x 16 k), the
 // activations the B operand (k x 8 activation rows).  Lane (g = lane/4,
@@ -607,6 +699,25 @@ static cudaError_t launch_bf16(const uint16_t *x, int Kd, int N, const uint16_t 
     return cudaGetLastError();
 }
 
+// Shared memory of the tensor-core bf16 kernel for M (<= 16) rows.
+static size_t bf16_mma_smem(int M, int Kd) { return (size_t)M * (Kd + 32) * 2; }
+
+template <int NT>
+static cudaError_t launch_bf16_mma(const uint16_t *x, int M, int Kd, int N, const uint16_t *W,
+                                   float *y, int ldy, cudaStream_t s) {
+    constexpr int U = 8;
+    auto k = lm_head_bf16_mma_kernel<NT, U>;
+    const size_t smem = bf16_mma_smem(M, Kd);
+    int occ = 0;
+    cudaError_t e = kernel_setup((const void *)k, kBmmaThreads, smem, &occ);
+    if (e != cudaSuccess) return e;
+    const int ntiles = (N + 15) / 16;
+    const int need = (ntiles + kBmmaThreads / 32 - 1) / (kBmmaThreads / 32);
+    const int grid = std::min(need, kSMs * occ);
+    k<<<grid, kBmmaThreads, smem, s>>>(x, M, Kd, N, W, y, ldy);
+    return cudaGetLastError();
+}
+
 // Shared memory of the direct-load fp16 int4 kernel for M (<= 8) rows.
 static size_t int4_direct_smem(int M, int Kd) {
     const size_t Gt = (size_t)Kd / 64;
@@ -704,6 +815,18 @@ size_t lm_head_max_smem_rows(int Kd) {
 cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, const void *scales,
                            int fmt, float *y, cudaStream_t s) {
     const uint16_t *xb = static_cast<const uint16_t *>(x);
+    if (fmt == MTPV_W_BF16 && M > 8 && bf16_mma_smem(16, Kd) <= (size_t)227 * 1024) {
+        // more than 8 rows: the tensor-core kernel, up to 16 rows per pass
+        const uint16_t *W = static_cast<const uint16_t *>(w);
+        for (int m0 = 0; m0 < M; m0 += 16) {
+            const int mm = std::min(16, M - m0);
+            const cudaError_t e =
+                mm > 8 ? launch_bf16_mma<2>(xb + (size_t)m0 * Kd, mm, Kd, N, W, y + (size_t)m0 * N, N, s)
+                       : launch_bf16_mma<1>(xb + (size_t)m0 * Kd, mm, Kd, N, W, y + (size_t)m0 * N, N, s);
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    }
     const int step = (int)std::min<size_t>(8, lm_head_max_smem_rows(Kd));
     if (step < 1) return cudaErrorInvalidValue;
     for (int m0 = 0; m0 < M; m0 += step) {
