@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
                     [--impl {mtpv,reference}] [--no-cpu-baseline] [--no-e2e] [--no-graph]
+    python bench.py --proj     (int4 decoder-layer projections at small M)
 
 One step = the whole verify step of one batch: the K+1 target rows through
 the bf16 LM head, the K draft rows through the int4 group-64 head, and the
@@ -452,6 +453,89 @@ def run_gpu(args, c, rank, world, local_rank):
     print(json.dumps(line), flush=True)
 
 
+# ---------------------------------------------------------------------------
+# decoder-layer projections (int4 g64, small M): a separate measurement mode
+# ---------------------------------------------------------------------------
+PROJ_SHAPES = [  # name, Kd, N (gate_up: N = 2F, output F)
+    ("qkv", 5120, 7168), ("o", 5120, 5120), ("gate_up", 5120, 2 * 17408), ("down", 17408, 5120)]
+
+
+def run_proj(args):
+    """Each projection of a 27B-class decoder layer at M in {1..6, 8}, weights
+    rotated over enough copies (>= 4x the L2) that every call streams them
+    from HBM; CUDA-event time per call, plain launches and CUDA-graph replay."""
+    import verify_step_lm_b200 as mtpv
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    mtpv.load()
+    peak, peak_kind = measured_peaks()
+    layer_bytes = sum(N * (Kd // 2) + N * (Kd // 64) * 2 for _, Kd, N in PROJ_SHAPES)
+    copies = max(2, -(-4 * 126 * 2 ** 20 // layer_bytes))
+    layers = []
+    for c in range(copies):
+        lay = {}
+        for name, Kd, N in PROJ_SHAPES:
+            W = synth.make_head(N, Kd, 0.02, seed=700 + 10 * c + len(lay), device=dev)
+            lay[name] = synth.quantize_int4_g64(W)
+            del W
+        layers.append(lay)
+    stream = torch.cuda.current_stream(dev)
+    out = {}
+    for M in (1, 2, 3, 4, 5, 6, 8):
+        row = {}
+        for name, Kd, N in PROJ_SHAPES:
+            x = synth.gaussian((M, Kd), 1.0, 900 + M, dev)
+            ncols = N // 2 if name == "gate_up" else N
+            y = torch.empty((M, ncols), dtype=torch.float32, device=dev)
+            if name == "gate_up":
+                ws = mtpv.workspace(mtpv.load().mtpv_int4_gate_up_workspace_bytes(M, Kd, N // 2), dev)
+                call = lambda lay: mtpv.int4_gate_up(x, lay[name][0], lay[name][1], y, ws=ws)
+            else:
+                ws = mtpv.workspace(mtpv.load().mtpv_int4_proj_workspace_bytes(M, Kd, N), dev)
+                call = lambda lay: mtpv.int4_proj(x, lay[name][0], lay[name][1], y, ws=ws)
+            for i in range(args.warmup):
+                call(layers[i % copies])
+            n = max(30, min(args.steps, 400))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for i in range(n):
+                call(layers[i % copies])
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us = 1e3 * e0.elapsed_time(e1) / n
+            graphs = []
+            for c in range(copies):
+                g = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(g):
+                    call(layers[c])
+                graphs.append(g)
+            for i in range(args.warmup):
+                graphs[i % copies].replay()
+            torch.cuda.synchronize()
+            e0.record(stream)
+            for i in range(n):
+                graphs[i % copies].replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            us_graph = 1e3 * e0.elapsed_time(e1) / n
+            del graphs
+            nbytes = N * (Kd // 2) + N * (Kd // 64) * 2 + M * Kd * 2 + M * ncols * 4
+            row[name] = {"us": us, "us_graph": us_graph, "gbs": nbytes / (us * 1e-6) / 1e9,
+                         "frac": nbytes / (us * 1e-6) / 1e9 / peak, "bytes": nbytes}
+        row["layer_us"] = sum(v["us"] for v in row.values() if isinstance(v, dict))
+        row["layer_us_graph"] = sum(v["us_graph"] for k, v in row.items() if isinstance(v, dict))
+        out[M] = row
+    line = {"metric": "int4 g64 decoder-layer projections (qkv, o, gate||up with SiLU, down) per layer",
+            "unit": "us", "higher_is_better": False, "n_gpus": 1, "data": "synthetic",
+            "config": {"workload": "27B-class layer: hidden 5120, intermediate 17408, qkv 7168; "
+                                   "W ~ N(0, 0.02^2) -> int4 g64, activations N(0,1) bf16",
+                       "weight_copies": copies, "l2": "weights rotated over >= 4x L2"},
+            "peak_gbs": peak, "peak_source": peak_kind, "by_m": out}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -462,6 +546,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--proj", action="store_true",
+                    help="time the int4 decoder-layer projections instead of the verify step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -471,6 +557,10 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
     if args.impl == "reference":
         run_reference(args, c, rank)
+        return
+    if args.proj:
+        if rank == 0:
+            run_proj(args)
         return
     if world > 1:
         import datetime

@@ -158,6 +158,45 @@ MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, fl
                                        size_t ws_bytes, mtpv_stream stream);
 
 /* ------------------------------------------------------------------------
+ * mtpv_int4_proj / mtpv_int4_gate_up -- small-M decoder-layer projections
+ * with int4 group-64 weights (the verify pass's other matmuls: attention
+ * qkv and o, MLP gate/up and down).
+ *
+ * Passage: hazakura.dev MTPLX notes, Layer 0 (matmuls specialised for
+ * M = 3..6 rows); gist.science BaseRT explainer, methodology (per-format
+ * decode GEMV with dequantisation in the inner loop; fused op chains).
+ *
+ *   mtpv_int4_proj:     y[M, N] = x[M, Kd] . deq(wq, scales)^T
+ *   mtpv_int4_gate_up:  h[M, F] = silu(x . G^T) * (x . U^T), where rows
+ *                       0..F-1 of the [2F, Kd] head are G (gate) and rows
+ *                       F..2F-1 are U (up); silu(g) = g / (1 + e^-g).
+ *
+ *   x       device bf16 [M, Kd] (16-byte aligned), 1 <= M <= 64.
+ *   wq      device uint8 [N, Kd/2] (N = 2F for gate_up), MTPV_W_INT4_G64
+ *           nibble order; scales device bf16 [N, Kd/64].
+ *   Kd      a positive multiple of 64, at most 92864.  A pass stages up to
+ *           8 activation rows in shared memory as fp16: 8 rows per pass up
+ *           to Kd = 14016, 6 at Kd = 17408, fewer beyond (the weights are
+ *           read once per pass).
+ *   y, h    device fp32 [M, N] / [M, F], fully overwritten.
+ * The reduction over Kd is split into slices when N alone gives too few
+ * 16-row tiles to fill the GPU; the slices' partial sums (workspace) are
+ * added in a fixed order, so results are deterministic.  Arithmetic: fp16
+ * MMA of exactly dequantised weights, fp32 accumulation per group, as
+ * mtpv_lm_head_smallm's int4 path.
+ * ws, ws_bytes: at least the matching *_workspace_bytes() bytes, 256-byte
+ * aligned.  Errors: MTPV_ERR_INVALID_ARG, MTPV_ERR_WORKSPACE, MTPV_ERR_CUDA.
+ * ---------------------------------------------------------------------- */
+MTPV_API size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N);
+MTPV_API mtpv_status mtpv_int4_proj(const void *x, int M, int Kd, int N, const void *wq,
+                                    const void *scales, float *y, void *ws, size_t ws_bytes,
+                                    mtpv_stream stream);
+MTPV_API size_t mtpv_int4_gate_up_workspace_bytes(int M, int Kd, int F);
+MTPV_API mtpv_status mtpv_int4_gate_up(const void *x, int M, int Kd, int F, const void *wq,
+                                       const void *scales, float *h, void *ws, size_t ws_bytes,
+                                       mtpv_stream stream);
+
+/* ------------------------------------------------------------------------
  * mtpv_verify -- Leviathan-Chen verification of B independent sequences.
  *
  * Passages: devtrends.cc MTPLX overview and devtrends.ru page (exact rejection

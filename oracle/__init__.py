@@ -18,6 +18,10 @@ passage of the pages it follows:
   Layer 2 cycle).
 * ``sample_rows`` -- one draw from each row's warped distribution (the draft
   phase's own sampling step, hazakura.dev notes, Layer 2 "Draft").
+* ``silu_mul`` / ``gate_up_int4g64`` -- the gated MLP of a decoder layer:
+  silu(x . G^T) * (x . U^T) with an int4 g64 gate||up head (the matmuls of
+  the small-M regime beyond the LM head, hazakura.dev notes, Layer 0;
+  gist.science BaseRT explainer, fused op chains).  Plain numpy in fp64.
 
 Every function here is pinned by tests in ``tests/test_oracle_*.py`` against
 closed forms, brute force on tiny inputs and independent library routines.
@@ -253,3 +257,21 @@ def sample_rows(logits, T: float, top_p: float, u, threads: int = 1):
     with ThreadPoolExecutor(len(jobs)) as ex:
         list(ex.map(run, jobs))
     return out, mr, st
+
+
+def silu_mul(g: np.ndarray, u: np.ndarray) -> np.ndarray:
+    """silu(g) * u elementwise in fp64, silu(g) = g / (1 + exp(-g))."""
+    g = np.asarray(g, dtype=np.float64)
+    u = np.asarray(u, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return g / (1.0 + np.exp(-g)) * u
+
+
+def gate_up_int4g64(x_bits: np.ndarray, Wq: np.ndarray, S_bits: np.ndarray, F: int,
+                    cols=None, threads: int = 1) -> np.ndarray:
+    """h[M, F] (or the columns ``cols`` of it) = silu(x . G^T) * (x . U^T) for
+    the int4 g64 head [2F, Kd] whose rows 0..F-1 are G and F..2F-1 are U."""
+    cols = np.arange(F) if cols is None else np.asarray(cols)
+    g = lm_head_int4g64(x_bits, Wq[cols], S_bits[cols], threads=threads)
+    u = lm_head_int4g64(x_bits, Wq[F + cols], S_bits[F + cols], threads=threads)
+    return silu_mul(g, u)

@@ -52,6 +52,10 @@ def load() -> ctypes.CDLL:
         "mtpv_lm_head_smallm": ([P, I, I, I, P, P, I, P, P, Z, P], I),
         "mtpv_lm_head_pair_workspace_bytes": ([I, I, I, I], Z),
         "mtpv_lm_head_pair": ([P, I, P, P, P, I, P, P, P, I, I, P, Z, P], I),
+        "mtpv_int4_proj_workspace_bytes": ([I, I, I], Z),
+        "mtpv_int4_proj": ([P, I, I, I, P, P, P, P, Z, P], I),
+        "mtpv_int4_gate_up_workspace_bytes": ([I, I, I], Z),
+        "mtpv_int4_gate_up": ([P, I, I, I, P, P, P, P, Z, P], I),
         "mtpv_verify_workspace_bytes": ([I, I, I], Z),
         "mtpv_verify": ([P, P, P, P, P, I, I, I, F, F, P, P, P, P, Z, P], I),
         "mtpv_sample_workspace_bytes": ([I, I], Z),
@@ -151,6 +155,28 @@ def lm_head_pair(xt, w, yt, xd, wq, scales, yd, ws=None, stream=None):
         _ptr(xt), Mt, _ptr(w), _ptr(yt), _ptr(xd), Md, _ptr(wq), _ptr(scales), _ptr(yd), Kd, N,
         _ptr(ws), wsb, _stream(stream)))
     return yt, yd
+
+
+def int4_proj(x, wq, scales, y, ws=None, stream=None):
+    """y[M, N] (fp32) = x[M, Kd] (bf16) . deq(wq, scales)^T, split-K for decoder projections."""
+    M, Kd = x.shape
+    N = wq.shape[0]
+    if ws is None:
+        ws = workspace(load().mtpv_int4_proj_workspace_bytes(M, Kd, N), x.device)
+    _check("mtpv_int4_proj", load().mtpv_int4_proj(
+        _ptr(x), M, Kd, N, _ptr(wq), _ptr(scales), _ptr(y), _ptr(ws), ws.numel(), _stream(stream)))
+    return y
+
+
+def int4_gate_up(x, wq, scales, h, ws=None, stream=None):
+    """h[M, F] = silu(x . G^T) * (x . U^T) with G, U the two halves of the [2F, Kd] int4 head."""
+    M, Kd = x.shape
+    F = wq.shape[0] // 2
+    if ws is None:
+        ws = workspace(load().mtpv_int4_gate_up_workspace_bytes(M, Kd, F), x.device)
+    _check("mtpv_int4_gate_up", load().mtpv_int4_gate_up(
+        _ptr(x), M, Kd, F, _ptr(wq), _ptr(scales), _ptr(h), _ptr(ws), ws.numel(), _stream(stream)))
+    return h
 
 
 def verify(target_logits, draft_logits, draft_tokens, u_accept, u_sample, temperature: float,

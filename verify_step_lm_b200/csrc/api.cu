@@ -197,6 +197,41 @@ mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt, 
     return cuda_status(launch_heads(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, ws, (cudaStream_t)stream));
 }
 
+size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N) {
+    if (M < 1 || M > 64 || Kd < 64 || Kd % 64 || N < 1) return 0;
+    return mtpv::int4_proj_workspace_bytes(M, Kd, N);
+}
+
+static mtpv_status int4_proj_common(const void *x, int M, int Kd, int N, const void *wq,
+                                    const void *scales, float *y, int ldy, bool silu_mul, void *ws,
+                                    size_t ws_bytes, mtpv_stream stream) {
+    if (!x || !wq || !scales || !y) return MTPV_ERR_INVALID_ARG;
+    const size_t need = mtpv_int4_proj_workspace_bytes(M, Kd, N);
+    if (need == 0) return MTPV_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(scales, 2) || !aligned(y, 4))
+        return MTPV_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return MTPV_ERR_WORKSPACE;
+    return cuda_status(
+        mtpv::launch_int4_proj(x, M, Kd, N, wq, scales, y, ldy, silu_mul, ws, (cudaStream_t)stream));
+}
+
+mtpv_status mtpv_int4_proj(const void *x, int M, int Kd, int N, const void *wq, const void *scales,
+                           float *y, void *ws, size_t ws_bytes, mtpv_stream stream) {
+    return int4_proj_common(x, M, Kd, N, wq, scales, y, N, false, ws, ws_bytes, stream);
+}
+
+size_t mtpv_int4_gate_up_workspace_bytes(int M, int Kd, int F) {
+    if (F < 1 || F > (1 << 28)) return 0;
+    return mtpv_int4_proj_workspace_bytes(M, Kd, 2 * F);
+}
+
+mtpv_status mtpv_int4_gate_up(const void *x, int M, int Kd, int F, const void *wq,
+                              const void *scales, float *h, void *ws, size_t ws_bytes,
+                              mtpv_stream stream) {
+    if (F < 1 || F > (1 << 28)) return MTPV_ERR_INVALID_ARG;
+    return int4_proj_common(x, M, Kd, 2 * F, wq, scales, h, F, true, ws, ws_bytes, stream);
+}
+
 size_t mtpv_verify_workspace_bytes(int B, int K, int V) {
     if (!verify_shape_ok(B, K, V)) return 0;
     return verify_layout(B, K, V).total;

@@ -45,9 +45,19 @@ __device__ __forceinline__ int swz8(int k) {
 // Staging: every thread of the block takes part.
 template <int M>
 __device__ __forceinline__ void bf16_stage_x(float *xsf, const uint16_t *__restrict__ x, int Kd) {
-    for (int i = threadIdx.x; i < M * Kd; i += blockDim.x) {
-        const int m = i / Kd, k = i - m * Kd;
-        xsf[m * Kd + swz8(k)] = __uint_as_float((uint32_t)x[i] << 16);
+    // 8 activations per step: one 16-byte load, two float4 stores (the
+    // chunk's two halves swap places when (c >> 2) & 1, as swz8)
+    const int nch = Kd >> 3;
+#pragma unroll
+    for (int m = 0; m < M; ++m) {
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)m * Kd);
+        float4 *dst = reinterpret_cast<float4 *>(xsf + (size_t)m * Kd);
+        for (int c = threadIdx.x; c < nch; c += blockDim.x) {
+            const uint4 v = xr[c];
+            const int sw = (c >> 2) & 1;
+            dst[2 * c + sw] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
+            dst[2 * c + (sw ^ 1)] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
+        }
     }
 }
 
@@ -316,8 +326,25 @@ __device__ __forceinline__ void int4_f16_stage_x(uint16_t *xb, float *xs, unsign
     const int rowc = Gt * 8 + 1;
     if (threadIdx.x < 8) row_amax[threadIdx.x] = 0u;
     __syncthreads();
-    for (int i = threadIdx.x; i < M * Kd; i += blockDim.x)
-        atomicMax(&row_amax[i / Kd], ((uint32_t)x[i] << 16) & 0x7fffffffu);
+    {
+        // row maxima of |x| as bit patterns: per thread, then per warp, then
+        // one shared atomic per warp and row
+        const int lane = threadIdx.x & 31;
+        for (int m = 0; m < M; ++m) {
+            const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)m * Kd);
+            uint32_t a = 0u;
+            for (int c = threadIdx.x; c < (Kd >> 3); c += blockDim.x) {
+                const uint4 v = xr[c];
+                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                    a = max(a, max((w4[q] << 16) & 0x7fffffffu, (w4[q] >> 16) << 16 & 0x7fffffffu));
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
+            if (lane == 0 && a) atomicMax(&row_amax[m], a);
+        }
+    }
     if (zero_row)
         for (int i = threadIdx.x; i < rowc * 8; i += blockDim.x) xb[M * rowc * 8 + i] = 0;
     __syncthreads();
@@ -331,22 +358,43 @@ __device__ __forceinline__ void int4_f16_stage_x(uint16_t *xb, float *xs, unsign
         row_amax[threadIdx.x] = (uint32_t)sh;  // read back as int
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < M * Kd; i += blockDim.x) {
-        const int m = i / Kd, k = i - m * Kd;
+    // 8 activations per step (k = 8c .. 8c+7, one 16-byte load): in the
+    // layout of mma_x_pos, value w of the chunk goes to group position
+    // 16 ((c >> 1) & 3) + 4 (w & 3) + 2 (c & 1) + (w >> 2), so values w and
+    // w + 4 are adjacent: four 32-bit stores of fp16 pairs
+    for (int m = 0; m < M; ++m) {
         const int sh = (int)row_amax[m] + 4;  // the row's scale, then / 16
-        const float v = __uint_as_float((uint32_t)x[i] << 16) * __uint_as_float((uint32_t)(127 - sh) << 23);
-        xb[m * rowc * 8 + mma_x_pos(k)] = __half_as_ushort(__float2half_rn(v));
+        const float f = __uint_as_float((uint32_t)(127 - sh) << 23);
+        const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)m * Kd);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(xb + (size_t)m * rowc * 8);
+        for (int c = threadIdx.x; c < (Kd >> 3); c += blockDim.x) {
+            const uint4 v = xr[c];
+            const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+            const int base = (c >> 3) * 64 + ((c >> 1) & 3) * 16 + 2 * (c & 1);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const __half2 h = __floats2half2_rn(e[j] * f, e[j + 4] * f);
+                dst[(base + 4 * j) >> 1] = *reinterpret_cast<const uint32_t *>(&h);
+            }
+        }
     }
     __syncthreads();
-    for (int i = threadIdx.x; i < Gt * 8; i += blockDim.x) {
-        const int G = i >> 3, m = i & 7;
-        float sum = 0.0f;
-        if (m < M)
-            for (int k = G * 64; k < G * 64 + 64; ++k) {
-                const float b = __half2float(__ushort_as_half(xb[m * rowc * 8 + mma_x_pos(k)]));
-                sum = fmaf(1152.0f, b, sum);
+    {
+        // offset sums, one warp per (group, row): 1152 x (sum of the group's
+        // staged activations), summed by a fixed shuffle tree
+        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+        for (int i = warp; i < Gt * 8; i += nw) {
+            const int G = i >> 3, m = i & 7;
+            float v = 0.0f;
+            if (m < M) {
+                const uint16_t *r = xb + (size_t)m * rowc * 8 + G * 64;  // the group's 64 staged values
+                v = __half2float(__ushort_as_half(r[lane])) + __half2float(__ushort_as_half(r[lane + 32]));
             }
-        xs[i] = sum;
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+            if (lane == 0) xs[i] = 1152.0f * v;
+        }
     }
     __syncthreads();
 }
@@ -502,23 +550,22 @@ __global__ void __launch_bounds__(NT) lm_head_int4_f16_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// Both heads of a verify step in one persistent launch.  Every warp takes
-// work items from one list in which the int4 tasks (RB 16-row tiles each) are
-// spread evenly among the bf16 row groups, so at any moment most warps stream
-// the bf16 head while a few dequantise the int4 head: the int4 head's
-// dequantisation and latency hide behind the bf16 stream instead of running
-// as a launch of its own.  The int4 task loads its nibbles straight into
-// registers (8 bytes per lane and row per group) and computes exactly as the
-// fp16 ring kernel does (same MMA operands, order and epilogue), and the bf16
-// group is the bf16 kernel's, so each head's logits are bit-identical to its
-// own kernel's.
+// Direct-load form of the fp16 int4 kernel: each lane loads its nibbles
+// straight into registers (8 bytes per row and group) and computes exactly as
+// the ring kernel does (same MMA operands, order and epilogue), so both forms
+// give the same bits.  Used where the ring does not fit and, over slices of
+// the reduction, by the split-K projection kernel.
 // ---------------------------------------------------------------------------
+// Groups [gbeg, gend) of the RB tiles of task `task`, scaled back by the
+// rows' power-of-two factors and stored to y (partial sums when the range
+// is a slice of the reduction).
 template <int RB, int UI>
 __device__ __forceinline__ void int4_f16_direct_task(const uint4 *xstage, const float *xs,
                                                      const float *row_unscale, int M, int Kd, int N,
                                                      const uint8_t *__restrict__ Wq,
                                                      const uint16_t *__restrict__ S,
-                                                     float *__restrict__ y, int ldy, int task) {
+                                                     float *__restrict__ y, int ldy, int task,
+                                                     int gbeg, int gend) {
     const int Gt = Kd >> 6;
     const int rowc = Gt * 8 + 1;
     const int lane = threadIdx.x & 31;
@@ -542,7 +589,7 @@ __device__ __forceinline__ void int4_f16_direct_task(const uint4 *xstage, const 
     for (int rb = 0; rb < RB; ++rb)
 #pragma unroll
         for (int e = 0; e < 4; ++e) acc[rb][e] = 0.0f;
-    for (int G0 = 0; G0 < Gt; G0 += UI) {
+    for (int G0 = gbeg; G0 < gend; G0 += UI) {
         uint2 wv[UI][RB][2];
         float sc[UI][RB][2];
 #pragma unroll
@@ -552,13 +599,13 @@ __device__ __forceinline__ void int4_f16_direct_task(const uint4 *xstage, const 
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                     const int G = G0 + u;
-                    wv[u][rb][h] = G < Gt ? ld_stream8(wr[rb][h] + G * 32) : make_uint2(0, 0);
-                    sc[u][rb][h] = G < Gt ? __uint_as_float((uint32_t)__ldg(sr[rb][h] + G) << 16) : 0.0f;
+                    wv[u][rb][h] = G < gend ? ld_stream8(wr[rb][h] + G * 32) : make_uint2(0, 0);
+                    sc[u][rb][h] = G < gend ? __uint_as_float((uint32_t)__ldg(sr[rb][h] + G) << 16) : 0.0f;
                 }
 #pragma unroll
         for (int u = 0; u < UI; ++u) {
             const int G = G0 + u;
-            if (G < Gt) {
+            if (G < gend) {
                 const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
                 const uint4 bA = has_row ? xrow[G * 8] : z4;
                 const uint4 bB = has_row ? xrow[G * 8 + 1] : z4;
@@ -630,7 +677,61 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_int4_f16_direct_kernel(
     int4_f16_stage_x(xb, xs, row_amax, row_unscale, x, M, Kd, false);
     const int tasks = ((N + 15) / 16 + RB - 1) / RB;
     for (int task = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); task < tasks; task += gridDim.x * kGemvWarps)
-        int4_f16_direct_task<RB, UI>(smem_dir, xs, row_unscale, M, Kd, N, Wq, S, y, ldy, task);
+        int4_f16_direct_task<RB, UI>(smem_dir, xs, row_unscale, M, Kd, N, Wq, S, y, ldy, task, 0, Kd >> 6);
+}
+
+// ---------------------------------------------------------------------------
+// Split-K int4 projection for decoder layers (few output rows per tile, long
+// reductions: N of a few thousand gives too few 16-row tiles to fill 148
+// SMs).  A work item is one task (RB tiles) over one slice of the 64-weight
+// groups; its partial sums go to part[slice][M][N], and a second kernel adds
+// the slices in a fixed order (deterministic), optionally applying the SiLU
+// gate of a gate||up projection.
+// ---------------------------------------------------------------------------
+template <int RB, int UI>
+__global__ void __launch_bounds__(kGemvThreads) lm_head_int4_splitk_kernel(
+    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint8_t *__restrict__ Wq,
+    const uint16_t *__restrict__ S, float *__restrict__ part, int slices, int gps) {
+    extern __shared__ uint4 smem_sk[];
+    __shared__ unsigned int row_amax[8];
+    __shared__ float row_unscale[8];
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    uint16_t *xb = reinterpret_cast<uint16_t *>(smem_sk);               // [M][rowc * 8]
+    float *xs = reinterpret_cast<float *>(smem_sk + (size_t)M * rowc);  // [Gt][8]
+    int4_f16_stage_x(xb, xs, row_amax, row_unscale, x, M, Kd, false);
+    const int tasks = ((N + 15) / 16 + RB - 1) / RB;
+    const int items = tasks * slices;
+    for (int item = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); item < items;
+         item += gridDim.x * kGemvWarps) {
+        const int task = item / slices, sl = item - task * slices;
+        const int gbeg = sl * gps, gend = min(Gt, gbeg + gps);
+        int4_f16_direct_task<RB, UI>(smem_sk, xs, row_unscale, M, Kd, N, Wq, S,
+                                     part + (size_t)sl * M * N, N, task, gbeg, gend);
+    }
+}
+
+// y[m][j] = sum over slices of part[s][m][j] (s in order); with silu_mul the
+// N columns are a gate half and an up half and y[m][j] = silu(g) * u for
+// j < N/2, g = column j, u = column j + N/2, silu(g) = g / (1 + e^-g).
+__global__ void __launch_bounds__(kGemvThreads) splitk_reduce_kernel(const float *__restrict__ part,
+                                                                     int slices, int M, int N,
+                                                                     float *__restrict__ y, int ldy,
+                                                                     int silu_mul) {
+    const int cols = silu_mul ? N / 2 : N;
+    const size_t plane = (size_t)M * N;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < M * cols; i += gridDim.x * blockDim.x) {
+        const int m = i / cols, j = i - m * cols;
+        const float *p = part + (size_t)m * N + j;
+        float a = 0.0f;
+        for (int sl = 0; sl < slices; ++sl) a += p[sl * plane];
+        if (silu_mul) {
+            float b = 0.0f;
+            for (int sl = 0; sl < slices; ++sl) b += p[sl * plane + cols];
+            a = a / (1.0f + expf(-a)) * b;
+        }
+        y[(size_t)m * ldy + j] = a;
+    }
 }
 
 constexpr int kMixWarps = 16;      // per CTA, one CTA per SM
@@ -805,6 +906,68 @@ cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *y
         case 3: return launch_pair<3>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
         default: return launch_pair<4>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
     }
+}
+
+// ---- split-K projection ----------------------------------------------------
+constexpr int kSplitRB = 2, kSplitUI = 4;
+
+// Rows of activations one split-K pass stages (fp16, plus the offset sums).
+static int splitk_rows(int Kd) {
+    const size_t per_row = ((size_t)Kd / 8 + 1) * 16, fixed = (size_t)Kd / 2;
+    const size_t cap = (size_t)227 * 1024 - 256;  // leaves room for the static shared memory
+    return cap > fixed ? (int)std::min<size_t>(8, (cap - fixed) / per_row) : 0;
+}
+
+// Slices of the reduction for a pass over N outputs: enough items to give
+// every warp of the GPU about two, at least kSplitUI groups per slice.
+static void splitk_plan(int Kd, int N, int *slices, int *gps) {
+    const int Gt = Kd / 64;
+    const int tasks = ((N + 15) / 16 + kSplitRB - 1) / kSplitRB;
+    int sl = (2 * kSMs * kGemvWarps + tasks - 1) / tasks;
+    sl = std::max(1, std::min({sl, 16, std::max(1, Gt / kSplitUI)}));
+    const int g = (Gt + sl - 1) / sl;
+    *gps = g;
+    *slices = (Gt + g - 1) / g;
+}
+
+size_t int4_proj_workspace_bytes(int M, int Kd, int N) {
+    const int rows = splitk_rows(Kd);
+    if (rows < 1) return 0;
+    int slices, gps;
+    splitk_plan(Kd, N, &slices, &gps);
+    return (size_t)slices * std::min(M, rows) * N * sizeof(float);
+}
+
+cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq, const void *scales,
+                             float *y, int ldy, bool silu_mul, void *ws, cudaStream_t s) {
+    const int rows = splitk_rows(Kd);
+    if (rows < 1) return cudaErrorInvalidValue;
+    int slices, gps;
+    splitk_plan(Kd, N, &slices, &gps);
+    auto k = lm_head_int4_splitk_kernel<kSplitRB, kSplitUI>;
+    const uint16_t *xb = static_cast<const uint16_t *>(x);
+    float *part = static_cast<float *>(ws);
+    for (int m0 = 0; m0 < M; m0 += rows) {
+        const int mm = std::min(rows, M - m0);
+        const size_t smem = int4_direct_smem(mm, Kd);
+        int occ = 0;
+        cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ);
+        if (e != cudaSuccess) return e;
+        const int tasks = ((N + 15) / 16 + kSplitRB - 1) / kSplitRB;
+        const int need = (tasks * slices + kGemvWarps - 1) / kGemvWarps;
+        k<<<std::min(need, kSMs * occ), kGemvThreads, smem, s>>>(
+            xb + (size_t)m0 * Kd, mm, Kd, N, static_cast<const uint8_t *>(wq),
+            static_cast<const uint16_t *>(scales), part, slices, gps);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        const int cols = silu_mul ? N / 2 : N;
+        const int blocks = std::min(kSMs * 4, (mm * cols + kGemvThreads - 1) / kGemvThreads);
+        splitk_reduce_kernel<<<blocks, kGemvThreads, 0, s>>>(part, slices, mm, N, y + (size_t)m0 * ldy,
+                                                            ldy, silu_mul ? 1 : 0);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+    }
+    return cudaSuccess;
 }
 
 size_t lm_head_max_smem_rows(int Kd) {
