@@ -174,10 +174,10 @@ MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, fl
  *   x       device bf16 [M, Kd] (16-byte aligned), 1 <= M <= 64.
  *   wq      device uint8 [N, Kd/2] (N = 2F for gate_up), MTPV_W_INT4_G64
  *           nibble order; scales device bf16 [N, Kd/64].
- *   Kd      a positive multiple of 64, at most 92864.  A pass stages up to
- *           8 activation rows in shared memory as fp16: 8 rows per pass up
- *           to Kd = 14016, 6 at Kd = 17408, fewer beyond (the weights are
- *           read once per pass).
+ *   Kd      a positive multiple of 64, at most 2^20.  Passes of up to 8
+ *           rows (one MMA n-tile); the weights are read once per pass.  The
+ *           activations of a pass are staged once, as fp16 in the MMA
+ *           operand order, into the workspace.
  *   y, h    device fp32 [M, N] / [M, F], fully overwritten.
  * The reduction over Kd is split into slices when N alone gives too few
  * 16-row tiles to fill the GPU; the slices' partial sums (workspace) are

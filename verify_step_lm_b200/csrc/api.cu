@@ -198,7 +198,7 @@ mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt, 
 }
 
 size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N) {
-    if (M < 1 || M > 64 || Kd < 64 || Kd % 64 || N < 1) return 0;
+    if (M < 1 || M > 64 || Kd < 64 || Kd % 64 || Kd > (1 << 20) || N < 1 || N > (1 << 28)) return 0;
     return mtpv::int4_proj_workspace_bytes(M, Kd, N);
 }
 

@@ -319,84 +319,123 @@ __device__ __forceinline__ void nib_pairs_f16(uint32_t w, uint32_t (&p)[4]) {
 // Activation staging of the fp16 int4 kernels: per-row power-of-two
 // prescale, fp16, permuted (plus, with zero_row, a row of zeros at index M),
 // and the per-group offset sums.  Every thread of the block takes part; the block synchronises inside.
+// Per-row pieces of the staging, shared by the block-wide staging below and
+// the one-CTA-per-row staging kernel of the split-K projection.
+// Largest |x| of the row as an fp32 bit pattern, per calling warp (every
+// thread of the block walks the row; reduce the warps' values with max).
+__device__ __forceinline__ uint32_t int4_row_absmax_warp(const uint16_t *__restrict__ xrow, int Kd) {
+    const uint4 *xr = reinterpret_cast<const uint4 *>(xrow);
+    uint32_t a = 0u;
+    for (int c = threadIdx.x; c < (Kd >> 3); c += blockDim.x) {
+        const uint4 v = xr[c];
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            a = max(a, max((w4[q] << 16) & 0x7fffffffu, ((w4[q] >> 16) << 16) & 0x7fffffffu));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
+    return a;
+}
+// sh: the row's largest |x| times 2^-sh lies in [2^9, 2^10) (e: the largest
+// exponent with 2^e <= max|x|); an all-zero row keeps sh = 0.
+__device__ __forceinline__ int int4_row_shift(uint32_t amax) {
+    const int sh = amax ? (int)(amax >> 23) - 127 - 9 : 0;
+    return max(-100, min(100, sh));
+}
+// 8 activations per step (k = 8c .. 8c+7, one 16-byte load): in the layout
+// of mma_x_pos, value w of the chunk goes to group position
+// 16 ((c >> 1) & 3) + 4 (w & 3) + 2 (c & 1) + (w >> 2), so values w and w + 4
+// are adjacent: four 32-bit stores of fp16 pairs.  Scale 2^-(sh + 4): the
+// row's power-of-two factor, then / 16.
+__device__ __forceinline__ void int4_row_convert(const uint16_t *__restrict__ xrow, int Kd, int sh,
+                                                 uint16_t *dst_row) {
+    const float f = __uint_as_float((uint32_t)(127 - (sh + 4)) << 23);
+    const uint4 *xr = reinterpret_cast<const uint4 *>(xrow);
+    uint32_t *dst = reinterpret_cast<uint32_t *>(dst_row);
+    for (int c = threadIdx.x; c < (Kd >> 3); c += blockDim.x) {
+        const uint4 v = xr[c];
+        const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
+                            bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
+        const int base = (c >> 3) * 64 + ((c >> 1) & 3) * 16 + 2 * (c & 1);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __half2 h = __floats2half2_rn(e[j] * f, e[j + 4] * f);
+            dst[(base + 4 * j) >> 1] = *reinterpret_cast<const uint32_t *>(&h);
+        }
+    }
+}
+// Offset sum of group G of a staged row: 1152 x (sum of the group's 64 staged
+// activations), by a fixed shuffle tree; the calling warp's lane 0 gets it.
+__device__ __forceinline__ float int4_group_offset(const uint16_t *staged_row, int G) {
+    const int lane = threadIdx.x & 31;
+    const uint16_t *r = staged_row + G * 64;
+    float v = __half2float(__ushort_as_half(r[lane])) + __half2float(__ushort_as_half(r[lane + 32]));
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return 1152.0f * v;
+}
+
 __device__ __forceinline__ void int4_f16_stage_x(uint16_t *xb, float *xs, unsigned int *row_amax,
                                                  float *row_unscale, const uint16_t *__restrict__ x,
                                                  int M, int Kd, bool zero_row) {
     const int Gt = Kd >> 6;
     const int rowc = Gt * 8 + 1;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
     if (threadIdx.x < 8) row_amax[threadIdx.x] = 0u;
     __syncthreads();
-    {
-        // row maxima of |x| as bit patterns: per thread, then per warp, then
-        // one shared atomic per warp and row
-        const int lane = threadIdx.x & 31;
-        for (int m = 0; m < M; ++m) {
-            const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)m * Kd);
-            uint32_t a = 0u;
-            for (int c = threadIdx.x; c < (Kd >> 3); c += blockDim.x) {
-                const uint4 v = xr[c];
-                const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-                for (int q = 0; q < 4; ++q)
-                    a = max(a, max((w4[q] << 16) & 0x7fffffffu, (w4[q] >> 16) << 16 & 0x7fffffffu));
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) a = max(a, __shfl_xor_sync(0xffffffffu, a, o));
-            if (lane == 0 && a) atomicMax(&row_amax[m], a);
-        }
+    for (int m = 0; m < M; ++m) {  // row maxima: per warp, then one shared atomic per warp
+        const uint32_t a = int4_row_absmax_warp(x + (size_t)m * Kd, Kd);
+        if (lane == 0 && a) atomicMax(&row_amax[m], a);
     }
     if (zero_row)
         for (int i = threadIdx.x; i < rowc * 8; i += blockDim.x) xb[M * rowc * 8 + i] = 0;
     __syncthreads();
     if (threadIdx.x < 8) {
-        // sh: the row's largest |x| times 2^-sh lies in [2^9, 2^10) (e: the
-        // largest exponent with 2^e <= max|x|); an all-zero row keeps sh = 0
-        const uint32_t amax = row_amax[threadIdx.x];
-        int sh = amax ? (int)(amax >> 23) - 127 - 9 : 0;
-        sh = max(-100, min(100, sh));
+        const int sh = int4_row_shift(row_amax[threadIdx.x]);
         row_unscale[threadIdx.x] = __uint_as_float((uint32_t)(127 + sh) << 23);
         row_amax[threadIdx.x] = (uint32_t)sh;  // read back as int
     }
     __syncthreads();
-    // 8 activations per step (k = 8c .. 8c+7, one 16-byte load): in the
-    // layout of mma_x_pos, value w of the chunk goes to group position
-    // 16 ((c >> 1) & 3) + 4 (w & 3) + 2 (c & 1) + (w >> 2), so values w and
-    // w + 4 are adjacent: four 32-bit stores of fp16 pairs
-    for (int m = 0; m < M; ++m) {
-        const int sh = (int)row_amax[m] + 4;  // the row's scale, then / 16
-        const float f = __uint_as_float((uint32_t)(127 - sh) << 23);
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)m * Kd);
-        uint32_t *dst = reinterpret_cast<uint32_t *>(xb + (size_t)m * rowc * 8);
-        for (int c = threadIdx.x; c < (Kd >> 3); c += blockDim.x) {
-            const uint4 v = xr[c];
-            const float e[8] = {bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y),
-                                bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w)};
-            const int base = (c >> 3) * 64 + ((c >> 1) & 3) * 16 + 2 * (c & 1);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const __half2 h = __floats2half2_rn(e[j] * f, e[j + 4] * f);
-                dst[(base + 4 * j) >> 1] = *reinterpret_cast<const uint32_t *>(&h);
-            }
-        }
+    for (int m = 0; m < M; ++m)
+        int4_row_convert(x + (size_t)m * Kd, Kd, (int)row_amax[m], xb + (size_t)m * rowc * 8);
+    __syncthreads();
+    for (int i = warp; i < Gt * 8; i += nw) {  // offset sums, one warp per (group, row)
+        const int G = i >> 3, m = i & 7;
+        const float v = m < M ? int4_group_offset(xb + (size_t)m * rowc * 8, G) : 0.0f;
+        if (lane == 0) xs[i] = v;
     }
     __syncthreads();
-    {
-        // offset sums, one warp per (group, row): 1152 x (sum of the group's
-        // staged activations), summed by a fixed shuffle tree
-        const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-        for (int i = warp; i < Gt * 8; i += nw) {
-            const int G = i >> 3, m = i & 7;
-            float v = 0.0f;
-            if (m < M) {
-                const uint16_t *r = xb + (size_t)m * rowc * 8 + G * 64;  // the group's 64 staged values
-                v = __half2float(__ushort_as_half(r[lane])) + __half2float(__ushort_as_half(r[lane + 32]));
-            }
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-            if (lane == 0) xs[i] = 1152.0f * v;
-        }
-    }
+}
+
+// The same staging for the split-K projection, once per call into global
+// memory: one CTA per activation row (row blockIdx.x); xs entries of rows
+// past M are zeroed by CTA 0.
+__global__ void __launch_bounds__(kGemvThreads) int4_f16_stage_rows_kernel(
+    const uint16_t *__restrict__ x, int M, int Kd, uint16_t *__restrict__ xb, float *__restrict__ xs,
+    float *__restrict__ row_unscale) {
+    __shared__ unsigned int s_amax;
+    const int m = blockIdx.x;
+    const int Gt = Kd >> 6;
+    const int rowc = Gt * 8 + 1;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+    if (threadIdx.x == 0) s_amax = 0u;
     __syncthreads();
+    const uint32_t a = int4_row_absmax_warp(x + (size_t)m * Kd, Kd);
+    if (lane == 0 && a) atomicMax(&s_amax, a);
+    __syncthreads();
+    const int sh = int4_row_shift(s_amax);
+    if (threadIdx.x == 0) row_unscale[m] = __uint_as_float((uint32_t)(127 + sh) << 23);
+    uint16_t *dst = xb + (size_t)m * rowc * 8;
+    int4_row_convert(x + (size_t)m * Kd, Kd, sh, dst);
+    __syncthreads();
+    for (int G = warp; G < Gt; G += nw) {
+        const float v = int4_group_offset(dst, G);
+        if (lane == 0) xs[G * 8 + m] = v;
+    }
+    if (m == 0)
+        for (int i = threadIdx.x; i < Gt * 8; i += blockDim.x)
+            if ((i & 7) >= M) xs[i] = 0.0f;
 }
 
 // The 16-row tiles of warp gw of nw warps (grid-wide numbering), streamed
@@ -683,31 +722,27 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_int4_f16_direct_kernel(
 // ---------------------------------------------------------------------------
 // Split-K int4 projection for decoder layers (few output rows per tile, long
 // reductions: N of a few thousand gives too few 16-row tiles to fill 148
-// SMs).  A work item is one task (RB tiles) over one slice of the 64-weight
-// groups; its partial sums go to part[slice][M][N], and a second kernel adds
+// SMs).  The activations are staged once per call into global memory (one
+// CTA per row), where every work item reads its fragments through the
+// caches; a work item is one task (RB tiles) over one slice of the 64-weight
+// groups; its partial sums go to part[slice][M][N], and a third kernel adds
 // the slices in a fixed order (deterministic), optionally applying the SiLU
 // gate of a gate||up projection.
 // ---------------------------------------------------------------------------
 template <int RB, int UI>
 __global__ void __launch_bounds__(kGemvThreads) lm_head_int4_splitk_kernel(
-    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint8_t *__restrict__ Wq,
-    const uint16_t *__restrict__ S, float *__restrict__ part, int slices, int gps) {
-    extern __shared__ uint4 smem_sk[];
-    __shared__ unsigned int row_amax[8];
-    __shared__ float row_unscale[8];
+    const uint4 *__restrict__ xstage, const float *__restrict__ xs, const float *__restrict__ unscale,
+    int M, int Kd, int N, const uint8_t *__restrict__ Wq, const uint16_t *__restrict__ S,
+    float *__restrict__ part, int slices, int gps) {
     const int Gt = Kd >> 6;
-    const int rowc = Gt * 8 + 1;
-    uint16_t *xb = reinterpret_cast<uint16_t *>(smem_sk);               // [M][rowc * 8]
-    float *xs = reinterpret_cast<float *>(smem_sk + (size_t)M * rowc);  // [Gt][8]
-    int4_f16_stage_x(xb, xs, row_amax, row_unscale, x, M, Kd, false);
     const int tasks = ((N + 15) / 16 + RB - 1) / RB;
     const int items = tasks * slices;
     for (int item = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); item < items;
          item += gridDim.x * kGemvWarps) {
         const int task = item / slices, sl = item - task * slices;
         const int gbeg = sl * gps, gend = min(Gt, gbeg + gps);
-        int4_f16_direct_task<RB, UI>(smem_sk, xs, row_unscale, M, Kd, N, Wq, S,
-                                     part + (size_t)sl * M * N, N, task, gbeg, gend);
+        int4_f16_direct_task<RB, UI>(xstage, xs, unscale, M, Kd, N, Wq, S, part + (size_t)sl * M * N, N,
+                                     task, gbeg, gend);
     }
 }
 
@@ -909,14 +944,7 @@ cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *y
 }
 
 // ---- split-K projection ----------------------------------------------------
-constexpr int kSplitRB = 2, kSplitUI = 4;
-
-// Rows of activations one split-K pass stages (fp16, plus the offset sums).
-static int splitk_rows(int Kd) {
-    const size_t per_row = ((size_t)Kd / 8 + 1) * 16, fixed = (size_t)Kd / 2;
-    const size_t cap = (size_t)227 * 1024 - 256;  // leaves room for the static shared memory
-    return cap > fixed ? (int)std::min<size_t>(8, (cap - fixed) / per_row) : 0;
-}
+constexpr int kSplitRB = 2, kSplitUI = 4, kSplitRows = 8;  // rows per pass: one MMA n-tile
 
 // Slices of the reduction for a pass over N outputs: enough items to give
 // every warp of the GPU about two, at least kSplitUI groups per slice.
@@ -930,33 +958,51 @@ static void splitk_plan(int Kd, int N, int *slices, int *gps) {
     *slices = (Gt + g - 1) / g;
 }
 
-size_t int4_proj_workspace_bytes(int M, int Kd, int N) {
-    const int rows = splitk_rows(Kd);
-    if (rows < 1) return 0;
+// Workspace: [staged activations: kSplitRows x rowc x 16 B][offset sums: Gt x
+// 8 fp32][row scales: 8 fp32][partial sums: slices x rows x N fp32]
+struct SplitWs {
+    size_t xb, xs, us, part, total;
+};
+static SplitWs splitk_layout(int M, int Kd, int N) {
+    const size_t Gt = (size_t)Kd / 64, rowc = Gt * 8 + 1;
     int slices, gps;
     splitk_plan(Kd, N, &slices, &gps);
-    return (size_t)slices * std::min(M, rows) * N * sizeof(float);
+    auto up = [](size_t n) { return (n + 255) / 256 * 256; };
+    SplitWs l;
+    l.xb = 0;
+    l.xs = l.xb + up((size_t)kSplitRows * rowc * 16);
+    l.us = l.xs + up(Gt * 8 * sizeof(float));
+    l.part = l.us + up(8 * sizeof(float));
+    l.total = l.part + up((size_t)slices * std::min(M, kSplitRows) * N * sizeof(float));
+    return l;
 }
+
+size_t int4_proj_workspace_bytes(int M, int Kd, int N) { return splitk_layout(M, Kd, N).total; }
 
 cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq, const void *scales,
                              float *y, int ldy, bool silu_mul, void *ws, cudaStream_t s) {
-    const int rows = splitk_rows(Kd);
-    if (rows < 1) return cudaErrorInvalidValue;
     int slices, gps;
     splitk_plan(Kd, N, &slices, &gps);
+    const SplitWs l = splitk_layout(M, Kd, N);
+    char *w = static_cast<char *>(ws);
+    uint16_t *xb = reinterpret_cast<uint16_t *>(w + l.xb);
+    float *xs = reinterpret_cast<float *>(w + l.xs);
+    float *us = reinterpret_cast<float *>(w + l.us);
+    float *part = reinterpret_cast<float *>(w + l.part);
     auto k = lm_head_int4_splitk_kernel<kSplitRB, kSplitUI>;
-    const uint16_t *xb = static_cast<const uint16_t *>(x);
-    float *part = static_cast<float *>(ws);
-    for (int m0 = 0; m0 < M; m0 += rows) {
-        const int mm = std::min(rows, M - m0);
-        const size_t smem = int4_direct_smem(mm, Kd);
+    const uint16_t *x16 = static_cast<const uint16_t *>(x);
+    for (int m0 = 0; m0 < M; m0 += kSplitRows) {
+        const int mm = std::min(kSplitRows, M - m0);
+        int4_f16_stage_rows_kernel<<<mm, kGemvThreads, 0, s>>>(x16 + (size_t)m0 * Kd, mm, Kd, xb, xs, us);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
         int occ = 0;
-        cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ);
+        e = kernel_setup((const void *)k, kGemvThreads, 0, &occ);
         if (e != cudaSuccess) return e;
         const int tasks = ((N + 15) / 16 + kSplitRB - 1) / kSplitRB;
         const int need = (tasks * slices + kGemvWarps - 1) / kGemvWarps;
-        k<<<std::min(need, kSMs * occ), kGemvThreads, smem, s>>>(
-            xb + (size_t)m0 * Kd, mm, Kd, N, static_cast<const uint8_t *>(wq),
+        k<<<std::min(need, kSMs * occ), kGemvThreads, 0, s>>>(
+            reinterpret_cast<const uint4 *>(xb), xs, us, mm, Kd, N, static_cast<const uint8_t *>(wq),
             static_cast<const uint16_t *>(scales), part, slices, gps);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
