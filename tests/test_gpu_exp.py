@@ -1,5 +1,8 @@
-"""Accuracy of the sampler's own fp64 exp (Cody-Waite reduction + Taylor
-series) against CUDA's exp: at most 2 ulp apart on [-745, 0], exact at 0, and
+"""Accuracy of the sampler's own fp64 exp (Tang's table-driven method: a
+64-entry table of 2^(j/64) built with CUDA's exp2, a degree-5 Taylor series
+on |r| <= ln2/128) against CUDA's exp: at most 3 ulp apart on [-745, 0]
+(table entries within exp2's 1-ulp bound, the series and the final multiply
+within about 1 ulp, CUDA's exp within its own 1-ulp bound), exact at 0, and
 0 below the subnormal range."""
 import ctypes
 import os
@@ -41,13 +44,15 @@ def ulps(a, b):
     return np.abs(ia - ib)
 
 
-def test_exp_within_two_ulp_of_cuda(exp_pair):
+def test_exp_within_three_ulp_of_cuda(exp_pair):
     rng = np.random.default_rng(0)
     x = np.concatenate([-rng.random(1_000_000) * 745.0, -rng.random(1_000_000) * 40.0,
                         -rng.random(100_000) * 1e-6, -np.arange(0, 746, 0.5)])
     mine, ref = exp_pair(x)
     normal = ref > 2.3e-308
-    assert ulps(mine[normal], ref[normal]).max() <= 2
+    d = ulps(mine[normal], ref[normal])
+    print(f"max ulp difference {d.max()}, mean {d.mean():.3f}")
+    assert d.max() <= 3
     # subnormal results: agree to the subnormal spacing
     assert np.abs(mine[~normal] - ref[~normal]).max() <= 4 * 5e-324
 

@@ -60,19 +60,22 @@ constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kBins = 2048;
 constexpr int kCandCap = 4096;
-constexpr int kCacheFloats = 16384;  // logits slice kept in shared memory (64 KB)
-constexpr int kBatch = 8;            // loads in flight per thread in streaming loops
+constexpr int kCacheFloats = 9728;  // logits slice kept in shared memory (38 KB), and its exps
+constexpr int kBatch = 8;           // loads in flight per thread in streaming loops
+constexpr int kExpTab = 64;         // entries of the exp table (2^(j/64))
 
-// Dynamic shared memory: a large region reused phase by phase, then the
-// small bookkeeping struct.
-//   region: [logits slice cache: kCacheFloats fp32][hist_mass: kBins fp64]
-//           [hist_cnt: kBins int][cand: kCandCap u64][cand_e: kCandCap fp64]
-//   during the draw the whole region is the weight buffer (fp64).
-constexpr size_t kOffHistMass = kCacheFloats * sizeof(float);
+// Dynamic shared memory of the statistics kernel: a region reused phase by
+// phase, then the small bookkeeping struct.
+//   region: [logits slice: kCacheFloats fp32][their exps: kCacheFloats fp64]
+//           [hist_mass: kBins fp64][hist_cnt: kBins int][cand: kCandCap u64]
+//           [cand_e: kCandCap fp64]
+constexpr size_t kOffExp = kCacheFloats * sizeof(float);
+constexpr size_t kOffHistMass = kOffExp + kCacheFloats * sizeof(double);
 constexpr size_t kOffHistCnt = kOffHistMass + kBins * sizeof(double);
 constexpr size_t kOffCand = kOffHistCnt + kBins * sizeof(int);
 constexpr size_t kOffCandE = kOffCand + kCandCap * sizeof(unsigned long long);
 constexpr size_t kRegionBytes = kOffCandE + kCandCap * sizeof(double);
+static_assert(kOffExp % 16 == 0 && kOffHistMass % 16 == 0, "region alignment");
 constexpr int kDrawBufDoubles = 16384;  // the draw kernel's weight buffer (128 KB)
 constexpr size_t kDrawBufBytes = kDrawBufDoubles * sizeof(double);
 
@@ -104,6 +107,7 @@ struct SamplerSmem {
     int wstar, x_found, first_fail, cut_idx;
     float cut_l;
     int res_x, res_acc;  // draw kernel: the position's token and acceptance, in CTA 0
+    double exp_tab[kExpTab];  // 2^(j/64), for exp_neg
 };
 
 constexpr size_t kStatsSmemBytes = kRegionBytes + sizeof(SamplerSmem);
@@ -111,6 +115,7 @@ constexpr size_t kDrawSmemBytes = kDrawBufBytes + sizeof(SamplerSmem);
 
 struct Region {
     float *cache;
+    double *ecache;
     double *hist_mass;
     int *hist_cnt;
     unsigned long long *cand;
@@ -140,45 +145,46 @@ __device__ __forceinline__ int key_index(unsigned long long k) {
     return (int)(0xffffffffu - (unsigned)(k & 0xffffffffu));
 }
 
-// exp(x) in fp64 for x <= 0.  Cody-Waite range reduction (Cody and Waite,
-// "Software Manual for the Elementary Functions", 1980): k = rint(x / ln 2),
-// r = x - k ln 2 with ln 2 split into a 32-bit head (k * head is exact) and
-// the double nearest the remainder, |r| <= ln 2 / 2; exp(r) from its Taylor
-// series to degree 14 (truncation below 4e-18 relative); 2^k assembled in the
-// exponent field (two steps below 2^-1022).  Arguments below -745.2 give 0.
-__device__ __forceinline__ double exp_neg(double x) {
+// exp(x) in fp64 for x <= 0, table-driven (P. T. P. Tang, "Table-driven
+// implementation of the exponential function in IEEE floating-point
+// arithmetic", ACM TOMS 15, 1989): x = (64 k' + j) ln2/64 + r with
+// |r| <= ln2/128, exp(x) = 2^k' * 2^(j/64) * exp(r).  k = 64 k' + j is
+// rint(64 x / ln 2); r = x - k ln2/64 with ln2/64 split into a 36-bit head
+// (k times it is exact, |k| < 2^17) and the double nearest the rest;
+// exp(r) - 1 from its Taylor series to degree 5 (truncation below 4e-17
+// relative at |r| = ln2/128); tab[j] = 2^(j/64), built with exp2 by
+// build_exp_table.  2^k' is assembled in the exponent field (two steps below
+// 2^-1022).  Arguments below -745.2 give 0.
+__device__ __forceinline__ void build_exp_table(double *tab) {
+    if (threadIdx.x < kExpTab) tab[threadIdx.x] = exp2((double)threadIdx.x / kExpTab);
+}
+
+__device__ __forceinline__ double exp_neg(double x, const double *tab) {
     if (!(x > -745.2)) return 0.0;
-    const double kLog2e = 1.4426950408889634;
-    const double kLn2Head = 0x1.62e42ff000000p-1;
-    const double kLn2Tail = -0x1.718432a1b0e26p-35;
+    const double kInv = 0x1.71547652b82fep+6;  // 64 / ln 2
+    const double kL1 = 0x1.62e42fefa0000p-7;   // ln 2 / 64, its first 36 bits
+    const double kL2 = 0x1.cf79abc9e3b3ap-46;  // ln 2 / 64 - kL1
     const double kRound = 6755399441055744.0;  // 1.5 * 2^52: adding it rounds to an integer
-    const double t = __fma_rn(x, kLog2e, kRound);
+    const double t = __fma_rn(x, kInv, kRound);
     const double kd = __dsub_rn(t, kRound);
     const int k = (int)__double2loint(t);
-    double r = __fma_rn(-kd, kLn2Head, x);
-    r = __fma_rn(-kd, kLn2Tail, r);
-    double q = 1.1470745597729725e-11;  // 1/14!
-    q = __fma_rn(q, r, 1.6059043836821613e-10);
-    q = __fma_rn(q, r, 2.08767569878681e-09);
-    q = __fma_rn(q, r, 2.505210838544172e-08);
-    q = __fma_rn(q, r, 2.755731922398589e-07);
-    q = __fma_rn(q, r, 2.7557319223985893e-06);
-    q = __fma_rn(q, r, 2.48015873015873e-05);
-    q = __fma_rn(q, r, 0.0001984126984126984);
-    q = __fma_rn(q, r, 0.001388888888888889);
-    q = __fma_rn(q, r, 0.008333333333333333);
-    q = __fma_rn(q, r, 0.041666666666666664);
-    q = __fma_rn(q, r, 0.16666666666666666);
+    double r = __fma_rn(-kd, kL1, x);
+    r = __fma_rn(-kd, kL2, r);
+    double q = 0.008333333333333333;    // 1/5!
+    q = __fma_rn(q, r, 0.041666666666666664);  // 1/4!
+    q = __fma_rn(q, r, 0.16666666666666666);   // 1/3!
     q = __fma_rn(q, r, 0.5);
     q = __fma_rn(q, r, 1.0);
-    q = __fma_rn(q, r, 1.0);
-    if (k >= -1022) return q * __hiloint2double((k + 1023) << 20, 0);
-    return (q * __hiloint2double((k + 1023 + 54) << 20, 0)) * 0x1p-54;
+    const double tj = tab[k & (kExpTab - 1)];
+    const double v = __fma_rn(tj, __dmul_rn(q, r), tj);  // 2^(j/64) exp(r)
+    const int e = k >> 6;                                 // floor(k / 64)
+    if (e >= -1022) return v * __hiloint2double((e + 1023) << 20, 0);
+    return (v * __hiloint2double((e + 1023 + 54) << 20, 0)) * 0x1p-54;
 }
 
 // e_j = exp((l_j - m) / T), with 1/T precomputed.
-__device__ __forceinline__ double e_of(float l, double m, double invT) {
-    return exp_neg(__dmul_rn(__dsub_rn((double)l, m), invT));
+__device__ __forceinline__ double e_of(float l, double m, double invT, const double *tab) {
+    return exp_neg(__dmul_rn(__dsub_rn((double)l, m), invT), tab);
 }
 
 // Level-1 bin of a logit: linear in (m - l) over the row's range; monotone
@@ -193,11 +199,11 @@ __device__ __forceinline__ bool is_kept(const RowStats &st, float l, int j) {
 
 // p'_j of one row given its statistics (logits read from global memory).
 __device__ __forceinline__ double warped_prob(const RowStats &st, const float *L, int j, double T,
-                                              double invT) {
+                                              double invT, const double *tab) {
     if (T == 0.0) return j == st.argmax ? 1.0 : 0.0;
     const float l = L[j];
     if (!is_kept(st, l, j)) return 0.0;
-    return e_of(l, (double)st.m, invT) / st.Zk;
+    return e_of(l, (double)st.m, invT, tab) / st.Zk;
 }
 
 // Fixed-tree block sum (deterministic for a given launch shape).
@@ -327,6 +333,7 @@ struct DrawSrc {
     RowStats st_t, st_d;
     const float *Lt, *Ld;
     const double *Et, *Ed;
+    const double *tab;  // exp table
     double rho;
     int kind;
 };
@@ -340,10 +347,10 @@ __device__ __forceinline__ double draw_combine(const DrawSrc &d, double wt, doub
 __device__ __forceinline__ double draw_weight(const DrawSrc &d, int j, double invT) {
     if (d.Et) return draw_combine(d, d.Et[j], d.kind == 1 ? d.Ed[j] : 0.0);
     const float lt = d.Lt[j];
-    const double wt = is_kept(d.st_t, lt, j) ? e_of(lt, (double)d.st_t.m, invT) : 0.0;
+    const double wt = is_kept(d.st_t, lt, j) ? e_of(lt, (double)d.st_t.m, invT, d.tab) : 0.0;
     if (d.kind == 0) return wt;
     const float ld = d.Ld[j];
-    const double wd = is_kept(d.st_d, ld, j) ? e_of(ld, (double)d.st_d.m, invT) : 0.0;
+    const double wd = is_kept(d.st_d, ld, j) ? e_of(ld, (double)d.st_d.m, invT, d.tab) : 0.0;
     return draw_combine(d, wt, wd);
 }
 
@@ -373,9 +380,9 @@ __device__ __forceinline__ void draw_weights_batch(const DrawSrc &d, int v1, int
 #pragma unroll
     for (int q = 0; q < kBatch; ++q) {
         const int j = j0 + q * kThreads;
-        const double wt = (j < v1 && is_kept(d.st_t, lt[q], j)) ? e_of(lt[q], (double)d.st_t.m, invT) : 0.0;
+        const double wt = (j < v1 && is_kept(d.st_t, lt[q], j)) ? e_of(lt[q], (double)d.st_t.m, invT, d.tab) : 0.0;
         const double wd = (d.kind == 1 && j < v1 && is_kept(d.st_d, ld[q], j))
-                              ? e_of(ld[q], (double)d.st_d.m, invT) : 0.0;
+                              ? e_of(ld[q], (double)d.st_d.m, invT, d.tab) : 0.0;
         w[q] = draw_combine(d, wt, wd);
     }
 }
@@ -505,6 +512,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     SamplerSmem &s = *reinterpret_cast<SamplerSmem *>(smem_raw + kRegionBytes);
     Region rg;
     rg.cache = reinterpret_cast<float *>(smem_raw);
+    rg.ecache = reinterpret_cast<double *>(smem_raw + kOffExp);
     rg.hist_mass = reinterpret_cast<double *>(smem_raw + kOffHistMass);
     rg.hist_cnt = reinterpret_cast<int *>(smem_raw + kOffHistCnt);
     rg.cand = reinterpret_cast<unsigned long long *>(smem_raw + kOffCand);
@@ -525,6 +533,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     const double invT = T > 0.0 ? 1.0 / T : 0.0;
     const bool topp_all = !(p.top_p < 1.0f);
     double *erow = p.ecache ? p.ecache + (size_t)row * V : nullptr;
+    build_exp_table(s.exp_tab);  // first used after the P1 barriers
     if (p.verify && row == 0 && rank == 0)  // ticket counters of the draw kernel
         for (int k = tid; k < p.B; k += kThreads) p.counters[k] = 0u;
     auto lval = [&](int j) -> float { return cached ? cache[j - v0] : L[j]; };
@@ -624,12 +633,13 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 lv[q] = j < v1 ? lval(j) : m;
             }
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) ev[q] = e_of(lv[q], md, invT);
+            for (int q = 0; q < kBatch; ++q) ev[q] = e_of(lv[q], md, invT, s.exp_tab);
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
                 const int j = j0 + q * kThreads;
                 if (j < v1) {
                     zt += ev[q];
+                    if (cached) rg.ecache[j - v0] = ev[q];
                     if (!topp_all) {
                         const int b = bin_of(lv[q], m, inv_w);
                         atomicAdd(&rg.hist_mass[b], ev[q]);
@@ -776,7 +786,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                             __syncthreads();
                         }
                     }
-                    for (int i = tid; i < n; i += kThreads) rg.cand_e[i] = e_of(key_logit(rg.cand[i]), md, invT);
+                    for (int i = tid; i < n; i += kThreads) rg.cand_e[i] = e_of(key_logit(rg.cand[i]), md, invT, s.exp_tab);
                     // exclusive prefix over the sorted candidates: sequential
                     // chunks per thread, thread totals chained by warp 0
                     const int ch = (n + kThreads - 1) / kThreads;
@@ -848,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                             const unsigned long long key = rank_key(l, j);
                             if ((key & mask) != prefix) continue;
                             const int d = (int)((key >> shift) & 255ull);
-                            const double e = e_of(l, md, invT);
+                            const double e = cached ? rg.ecache[j - v0] : e_of(l, md, invT, s.exp_tab);
                             if (d != cur) {
                                 if (cur >= 0) { atomicAdd(&s.rad_mass[cur], cacc); atomicAdd(&s.rad_cnt[cur], ccnt); }
                                 cur = d; cacc = 0.0; ccnt = 0;
@@ -892,7 +902,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 }
                 st.lstar = key_logit(prefix);
                 st.idxstar = key_index(prefix);
-                st.Zk = __dadd_rn(above, e_of(st.lstar, md, invT));
+                st.Zk = __dadd_rn(above, e_of(st.lstar, md, invT, s.exp_tab));
             }
         }
     }
@@ -901,17 +911,22 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     if (rank == 0 && tid == 0) p.slots[row].st = st;
     if (erow && !bad && T > 0.0) {
         const double md = (double)m;
-        for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
-            float lv[kBatch];
+        if (cached) {
+            for (int j = v0 + tid; j < v1; j += kThreads)
+                erow[j] = is_kept(st, rg.cache[j - v0], j) ? rg.ecache[j - v0] : 0.0;
+        } else {
+            for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
+                float lv[kBatch];
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                const int j = j0 + q * kThreads;
-                lv[q] = j < v1 ? lval(j) : -INFINITY;
-            }
+                for (int q = 0; q < kBatch; ++q) {
+                    const int j = j0 + q * kThreads;
+                    lv[q] = j < v1 ? lval(j) : -INFINITY;
+                }
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
-                const int j = j0 + q * kThreads;
-                if (j < v1) erow[j] = is_kept(st, lv[q], j) ? e_of(lv[q], md, invT) : 0.0;
+                for (int q = 0; q < kBatch; ++q) {
+                    const int j = j0 + q * kThreads;
+                    if (j < v1) erow[j] = is_kept(st, lv[q], j) ? e_of(lv[q], md, invT, s.exp_tab) : 0.0;
+                }
             }
         }
     }
@@ -951,6 +966,8 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
         s.res_x = -1;
         s.res_acc = 0;
     }
+    build_exp_table(s.exp_tab);
+    __syncthreads();
     const RowStats st_t = p.slots[rt].st;
     const RowStats st_d = p.slots[rd].st;
     const float *Lt = row_ptr(p, rt), *Ld = row_ptr(p, rd);
@@ -969,8 +986,8 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
                 pt = Et[d] / st_t.Zk;
                 qd = Ed[d] / st_d.Zk;
             } else {
-                pt = warped_prob(st_t, Lt, d, T, invT);
-                qd = warped_prob(st_d, Ld, d, T, invT);
+                pt = warped_prob(st_t, Lt, d, T, invT, s.exp_tab);
+                qd = warped_prob(st_d, Ld, d, T, invT, s.exp_tab);
             }
             const double ratio = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
             s.res_acc = (double)p.u_acc[(size_t)b * K + i] < ratio ? 1 : 0;
@@ -991,6 +1008,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
         src.Ld = residual ? Ld : Lt;
         src.Et = Et;
         src.Ed = residual ? Ed : Et;
+        src.tab = s.exp_tab;
         src.rho = residual ? st_t.Zk / st_d.Zk : 1.0;
         src.kind = residual ? 1 : 0;
         const float u = p.verify ? p.u_samp[(size_t)b * (K + 1) + i] : p.u_samp[c];
