@@ -261,8 +261,8 @@ def run_gpu(args, c, rank, world, local_rank):
     rs = torch.empty((B,), dtype=torch.int32, device=dev)
     ws = mtpv.workspace(mtpv.verify_step_workspace_bytes(B, K, V, h), dev)
     # the step runs both heads in one launch when the fused kernel takes the shapes
-    fused = B * (K + 1) <= 4 and B * K <= 8 and h % 512 == 0 and \
-        (B * (K + 1) * h * 4 + (B * K + 1) * (h // 8 + 1) * 16 + h // 2 + 4 * 13056) <= 227 * 1024 - 256
+    fused = B * (K + 1) <= 8 and B * K <= 8 and h % 512 == 0 and \
+        (2 * B * (K + 1) * (h + 32) + (B * K + 1) * (h // 8 + 1) * 16 + h // 2 + 3 * 13056) <= 227 * 1024 - 256
     pws = mtpv.workspace(mtpv.load().mtpv_lm_head_pair_workspace_bytes(B * (K + 1), B * K, h, V), dev)
     vws = mtpv.workspace(mtpv.verify_workspace_bytes(B, K, V), dev)
     stream = torch.cuda.current_stream(dev)

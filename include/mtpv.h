@@ -91,13 +91,14 @@ MTPV_API const char *mtpv_status_string(mtpv_status st);
  *   y[m][n] = sum_k x[m][k] * Wd[n][k],  0 <= m < M, 0 <= n < N   (fp32 out)
  *
  *   x       device, bf16 [M, Kd] row-major (activations / hidden states).
- *   M       rows, 1 <= M <= 64.  MTPV_W_BF16 with M <= 8 streams the head on
- *           the CUDA cores; with M > 8 (and Kd <= 7232) it runs on the tensor
- *           cores (mma.sync bf16, fp32 accumulation), 16 rows per pass.
- *           Other shapes go in groups of min(8, floor(232448 / (4 Kd)))
- *           rows.  The weights are re-read once per pass or group.
- *   Kd      reduction length, a positive multiple of 64, at most 58112 (the
- *           kernels stage each activation row in shared memory as fp32).
+ *   M       rows, 1 <= M <= 64.  MTPV_W_BF16 runs on the tensor cores
+ *           (mma.sync bf16, fp32 accumulation) in passes of up to 8 rows, or
+ *           16 when M > 8 and Kd <= 7232; a pass stages its rows as bf16 in
+ *           shared memory, so at most floor(232448 / (2 (Kd + 32))) rows go
+ *           in one pass.  MTPV_W_INT4_G64 goes in passes of
+ *           min(8, floor(232448 / (4 Kd))) rows.  The weights are re-read
+ *           once per pass.
+ *   Kd      reduction length, a positive multiple of 64, at most 58112.
  *           MTPV_W_INT4_G64 runs on the tensor cores (fp16 MMA of exactly
  *           dequantised nibbles, fp32 accumulation per 64-weight group):
  *           through per-warp shared-memory rings when Kd is a multiple of
@@ -136,15 +137,16 @@ MTPV_API mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, co
  * Passage: hazakura.dev MTPLX notes, Layer 0 (the target head at full
  * precision, the draft through a 4-bit copy) and its cached-graph item (one
  * fixed launch sequence per step).  Arguments as in mtpv_lm_head_smallm, the
- * same Kd and N for both heads.  When 1 <= Mt <= 4, 1 <= Md <= 8, Kd is a
+ * same Kd and N for both heads.  When 1 <= Mt <= 8, 1 <= Md <= 8, Kd is a
  * multiple of 512, the scales are 16-byte aligned and the staging fits in
- * shared memory (4 Mt Kd + (Md + 1)(2 Kd + 16) + Kd/2 + 52224 <= 232192
- * bytes; Mt = 4, Md = 3 at Kd = 5120 does), both heads run in ONE persistent
- * kernel: 4 of every CTA's 16 warps first stream the int4 head through their
- * shared-memory rings (bound by dequantisation, not by HBM) and then join
- * the other 12 on the bf16 head, whose row groups every warp takes one at a
- * time from a counter in `ws`, so the bf16 stream keeps HBM busy to the
- * end.  Otherwise the call makes the two mtpv_lm_head_smallm launches.
+ * shared memory (2 Mt (Kd + 32) + (Md + 1)(2 Kd + 16) + Kd/2 + 39168 <=
+ * 232192 bytes; Mt = 8, Md = 8 at Kd = 5120 does), both heads run in ONE
+ * persistent kernel: 3 of every CTA's 16 warps first stream the int4 head
+ * through their shared-memory rings (bound by dequantisation, not by HBM) and
+ * then join the other 13 on the bf16 head, whose 16-row tiles every warp
+ * takes one at a time from a counter in `ws`, so the bf16 stream keeps HBM
+ * busy to the end.  Otherwise the call makes the two mtpv_lm_head_smallm
+ * launches.
  * Either way the values are those mtpv_lm_head_smallm gives (same
  * arithmetic, bit for bit).
  * ws, ws_bytes: at least mtpv_lm_head_pair_workspace_bytes() bytes (256),

@@ -30,7 +30,8 @@ def hidden(M, Kd, seed):
 
 # (Mt, Md, Kd, N): fused shapes, then shapes that take two launches
 SHAPES = [(4, 3, 5120, 151936), (2, 1, 5120, 151936), (3, 2, 512, 4096), (1, 1, 512, 1000),
-          (4, 4, 1024, 4099), (4, 3, 640, 4096), (8, 6, 512, 4096), (4, 8, 5120, 20000)]
+          (4, 4, 1024, 4099), (8, 6, 512, 4096), (4, 8, 5120, 20000), (8, 8, 5120, 20011),
+          (4, 3, 640, 4096), (12, 3, 512, 4096), (9, 9, 1024, 3000)]
 
 
 @pytest.mark.parametrize("Mt,Md,Kd,N", SHAPES)

@@ -44,7 +44,8 @@ def test_int4_tiny_config_all_M(M):
 
 @pytest.mark.parametrize("fmt", [0, 1])
 @pytest.mark.parametrize("M,Kd,N", [(3, 64, 1), (4, 192, 999), (2, 1024, 4097), (16, 512, 300),
-                                    (32, 256, 77), (12, 5120, 513), (6, 17408, 130), (8, 17408, 64)])
+                                    (32, 256, 77), (12, 5120, 513), (6, 17408, 130), (8, 17408, 64),
+                                    (3, 58112, 40)])
 def test_ragged_shapes(fmt, M, Kd, N):
     # N not a multiple of the rows per warp, Kd not a multiple of the lane
     # stride, M above 8 (row groups), long Kd limited by shared memory

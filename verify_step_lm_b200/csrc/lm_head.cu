@@ -7,18 +7,18 @@
 // (gist.science BaseRT explainer, methodology: specialisation).
 //
 // At M <= 8 every weight is used M times, so the work is an HBM stream and the
-// kernels are built around keeping enough bytes in flight:
-//   bf16 head   CUDA cores.  Each warp owns RW consecutive weight rows and
-//               sweeps the whole reduction with 16-byte non-allocating loads,
-//               U chunks per row in flight; activations staged once per CTA
-//               as fp32 in an XOR-swizzled shared-memory layout; fp32
-//               accumulation, one warp-shuffle reduction per row.
-//   int4 head   tensor cores (mma.sync m16n8k16, fp32 accumulate).  On CUDA
-//               cores the dequantisation plus M FMAs per weight left the ALU
-//               and FMA pipes as the limit at a third of HBM bandwidth, so the
-//               weights are dequantised straight into MMA A registers and the
-//               activations are the B operand.  Each warp streams 16-row
-//               tiles through its own cp.async ring in shared memory.
+// kernels are built around keeping enough bytes in flight with as few
+// instructions as possible; both heads run on the tensor cores (mma.sync
+// m16n8k16, fp32 accumulate), the weights as the A operand straight from
+// global loads, the activations as the B operand from shared memory:
+//   bf16 head   one MMA stands for 64 FMAs and 16 bf16 widenings per lane,
+//               which leaves the warps free to keep 8 KB of loads in flight
+//               each (16-byte non-allocating loads, 16-row tiles).
+//   int4 head   on CUDA cores the dequantisation plus M FMAs per weight left
+//               the ALU and FMA pipes as the limit at a third of HBM
+//               bandwidth, so the weights are dequantised straight into MMA A
+//               registers.  Each warp streams 16-row tiles through its own
+//               cp.async ring in shared memory.
 // A persistent grid of (SMs x resident CTAs) walks the row blocks.
 #include <algorithm>
 
@@ -32,117 +32,21 @@ namespace mtpv {
 constexpr int kGemvThreads = 256;
 constexpr int kGemvWarps = kGemvThreads / 32;
 
-// Shared-memory layout of the bf16 kernel's fp32 activations, XOR-swizzled so
-// that a warp's 128-bit loads (one 8-weight chunk per lane, consecutive chunks
-// in consecutive lanes) spread over all 32 banks: float4 j of chunk c is
-// stored at position j ^ ((c >> 2) & 1).
-__device__ __forceinline__ int swz8(int k) {
-    const int c = k >> 3, j = (k >> 2) & 1;
-    return (c << 3) | ((j ^ ((c >> 2) & 1)) << 2) | (k & 3);
-}
-
-// bf16 weights with the activations staged as fp32 (no per-use widening).
-// Staging: every thread of the block takes part.
-template <int M>
-__device__ __forceinline__ void bf16_stage_x(float *xsf, const uint16_t *__restrict__ x, int Kd) {
-    // 8 activations per step: one 16-byte load, two float4 stores (the
-    // chunk's two halves swap places when (c >> 2) & 1, as swz8)
-    const int nch = Kd >> 3;
-#pragma unroll
-    for (int m = 0; m < M; ++m) {
-        const uint4 *xr = reinterpret_cast<const uint4 *>(x + (size_t)m * Kd);
-        float4 *dst = reinterpret_cast<float4 *>(xsf + (size_t)m * Kd);
-        for (int c = threadIdx.x; c < nch; c += blockDim.x) {
-            const uint4 v = xr[c];
-            const int sw = (c >> 2) & 1;
-            dst[2 * c + sw] = make_float4(bf16_lo(v.x), bf16_hi(v.x), bf16_lo(v.y), bf16_hi(v.y));
-            dst[2 * c + (sw ^ 1)] = make_float4(bf16_lo(v.z), bf16_hi(v.z), bf16_lo(v.w), bf16_hi(v.w));
-        }
-    }
-}
-
-// One group of RW consecutive weight rows (r0 = g * RW) for the calling warp.
-template <int M, int RW, int U>
-__device__ __forceinline__ void bf16_group(const float *xsf, int Kd, int N,
-                                           const uint16_t *__restrict__ W, float *__restrict__ y,
-                                           int ldy, int g) {
-    const int nch = Kd >> 3;
-    const int lane = threadIdx.x & 31;
-    const int r0 = g * RW;
-    const uint4 *wr[RW];
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-        wr[r] = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + r, N - 1) * Kd);
-    float acc[RW][M];
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-#pragma unroll
-        for (int m = 0; m < M; ++m) acc[r][m] = 0.0f;
-    for (int c0 = lane; c0 < nch; c0 += 32 * U) {
-        uint4 wv[U][RW];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = c0 + 32 * u;
-#pragma unroll
-            for (int r = 0; r < RW; ++r)
-                wv[u][r] = (c < nch) ? ld_stream16(wr[r] + c) : make_uint4(0, 0, 0, 0);
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int c = c0 + 32 * u;
-            if (c < nch) {
-#pragma unroll
-                for (int m = 0; m < M; ++m) {
-                    const int sw = (c >> 2) & 1;
-                    const float4 a = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 8 + (sw << 2));
-                    const float4 b = *reinterpret_cast<const float4 *>(xsf + m * Kd + c * 8 + ((sw ^ 1) << 2));
-#pragma unroll
-                    for (int r = 0; r < RW; ++r) {
-                        const uint4 w = wv[u][r];
-                        float t = acc[r][m];
-                        t = fmaf(a.x, bf16_lo(w.x), t); t = fmaf(a.y, bf16_hi(w.x), t);
-                        t = fmaf(a.z, bf16_lo(w.y), t); t = fmaf(a.w, bf16_hi(w.y), t);
-                        t = fmaf(b.x, bf16_lo(w.z), t); t = fmaf(b.y, bf16_hi(w.z), t);
-                        t = fmaf(b.z, bf16_lo(w.w), t); t = fmaf(b.w, bf16_hi(w.w), t);
-                        acc[r][m] = t;
-                    }
-                }
-            }
-        }
-    }
-#pragma unroll
-    for (int r = 0; r < RW; ++r)
-#pragma unroll
-        for (int m = 0; m < M; ++m) {
-            const float v = warp_sum(acc[r][m]);
-            if (lane == 0 && r0 + r < N) y[(size_t)m * ldy + r0 + r] = v;
-        }
-}
-
-template <int M, int RW, int U>
-__global__ void __launch_bounds__(kGemvThreads) lm_head_bf16_xf32_kernel(
-    const uint16_t *__restrict__ x, int Kd, int N, const uint16_t *__restrict__ W,
-    float *__restrict__ y, int ldy) {
-    extern __shared__ float xsf[];  // [M][Kd]
-    bf16_stage_x<M>(xsf, x, Kd);
-    __syncthreads();
-    const int groups = (N + RW - 1) / RW;
-    for (int g = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); g < groups; g += gridDim.x * kGemvWarps)
-        bf16_group<M, RW, U>(xsf, Kd, N, W, y, ldy, g);
-}
-
 // ---------------------------------------------------------------------------
-// bf16 head for 9..16 rows on the tensor cores (mma.sync m16n8k16 bf16, fp32
-// accumulate): the weights are the A operand (16 vocabulary rows x 16 k), the
-// activation rows the B operand (k x 8 rows, NT n-tiles).  The reduction
-// index is permuted inside every 32-k step so that each lane's fragments are
-// contiguous: lane (g, t) holds physical k 8t..8t+7 of the step, the first
-// four for the step's first MMA and the last four for its second (logical k
-// 2t, 2t+1, 2t+8, 2t+9 of an MMA are physical 8t + 0..3, or 8t + 4..7).
-// The A fragments are then one 16-byte global load per row, 64 contiguous
-// bytes per row per warp, and the B fragments one 16-byte shared-memory load
-// per n-tile; activation rows are padded by 64 bytes, which puts the two
-// rows of a quarter-warp on different halves of the banks.
+// bf16 head on the tensor cores (mma.sync m16n8k16 bf16, fp32 accumulate):
+// the weights are the A operand (16 vocabulary rows x 16 k), the activation
+// rows the B operand (k x 8 rows, NT n-tiles of 8 rows).  At M <= 8 the head
+// is an HBM stream and the MMA is there to save issue slots: one MMA does the
+// work of 64 FMAs plus 16 bf16 widenings per lane, so the warps spend their
+// time keeping loads in flight.  The reduction index is permuted inside every
+// 32-k step so that each lane's fragments are contiguous: lane (g, t) holds
+// physical k 8t..8t+7 of the step, the first four for the step's first MMA
+// and the last four for its second (logical k 2t, 2t+1, 2t+8, 2t+9 of an MMA
+// are physical 8t + 0..3, or 8t + 4..7).  The A fragments are then one
+// 16-byte global load per row, 64 contiguous bytes per row per warp, and the
+// B fragments one 16-byte shared-memory load per n-tile; activation rows are
+// staged as bf16 with a pitch of Kd + 32 elements (64 bytes of padding),
+// which puts the two rows of a quarter-warp on different halves of the banks.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
                                                uint32_t b1) {
@@ -154,73 +58,90 @@ __device__ __forceinline__ void mma_bf16_16816(float (&c)[4], const uint32_t (&a
 }
 
 constexpr int kBmmaThreads = 512;
+constexpr int kBmmaU = 8;  // 32-k steps in flight per lane: 8 KB of weights per warp
 
-template <int NT, int U>
-__global__ void __launch_bounds__(kBmmaThreads, 1) lm_head_bf16_mma_kernel(
-    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint16_t *__restrict__ W,
-    float *__restrict__ y, int ldy) {
-    extern __shared__ uint4 smem_bm[];
-    const int pitch = Kd + 32;  // bf16 elements per staged row (64 bytes of padding)
-    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_bm);
+// Stage M activation rows (bf16 [M, Kd]) at xs with pitch Kd + 32; every
+// thread of the block takes part, the caller places the barrier.
+__device__ __forceinline__ void bf16_mma_stage_x(uint16_t *xs, const uint16_t *__restrict__ x, int M,
+                                                 int Kd) {
+    const int pitch = Kd + 32;
     for (int i = threadIdx.x; i < M * (Kd / 8); i += blockDim.x) {
         const int m = i / (Kd / 8), c = i - m * (Kd / 8);
         *reinterpret_cast<uint4 *>(xs + (size_t)m * pitch + c * 8) =
             *reinterpret_cast<const uint4 *>(x + (size_t)m * Kd + c * 8);
     }
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+}
+
+// One 16-row tile (rows 16 tile .. 16 tile + 15) of y[M, N] for the calling warp.
+template <int NT, int U>
+__device__ __forceinline__ void bf16_mma_tile(const uint16_t *xs, int M, int Kd, int N,
+                                              const uint16_t *__restrict__ W, float *__restrict__ y,
+                                              int ldy, int tile) {
+    const int pitch = Kd + 32;
+    const int lane = threadIdx.x & 31;
     const int g = lane >> 2, t = lane & 3;
-    const int nwarps = blockDim.x >> 5;
-    const int ntiles = (N + 15) / 16;
     const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-    for (int tile = blockIdx.x * nwarps + warp; tile < ntiles; tile += gridDim.x * nwarps) {
-        const int r0 = tile * 16;
-        const uint4 *wa = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + g, N - 1) * Kd) + t;
-        const uint4 *wb = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + g + 8, N - 1) * Kd) + t;
-        float acc[NT][4];
+    const int r0 = tile * 16;
+    const uint4 *wa = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + g, N - 1) * Kd) + t;
+    const uint4 *wb = reinterpret_cast<const uint4 *>(W + (size_t)min(r0 + g + 8, N - 1) * Kd) + t;
+    float acc[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt)
+    for (int nt = 0; nt < NT; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
-        for (int k0 = 0; k0 < Kd; k0 += 32 * U) {
-            uint4 va[U], vb[U];
+        for (int e = 0; e < 4; ++e) acc[nt][e] = 0.0f;
+    for (int k0 = 0; k0 < Kd; k0 += 32 * U) {
+        uint4 va[U], vb[U];
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const bool in = k0 + 32 * u < Kd;
-                va[u] = in ? ld_stream16(wa + (k0 + 32 * u) / 8) : z4;
-                vb[u] = in ? ld_stream16(wb + (k0 + 32 * u) / 8) : z4;
-            }
+        for (int u = 0; u < U; ++u) {
+            const bool in = k0 + 32 * u < Kd;
+            va[u] = in ? ld_stream16(wa + (k0 + 32 * u) / 8) : z4;
+            vb[u] = in ? ld_stream16(wb + (k0 + 32 * u) / 8) : z4;
+        }
 #pragma unroll
-            for (int u = 0; u < U; ++u) {
-                const int k = k0 + 32 * u;
-                if (k < Kd) {
+        for (int u = 0; u < U; ++u) {
+            const int k = k0 + 32 * u;
+            if (k < Kd) {
 #pragma unroll
-                    for (int nt = 0; nt < NT; ++nt) {
-                        const int n = nt * 8 + g;
-                        const uint4 xv = n < M ? *reinterpret_cast<const uint4 *>(xs + (size_t)n * pitch + k + 8 * t)
-                                               : z4;
-                        const uint32_t a0[4] = {va[u].x, vb[u].x, va[u].y, vb[u].y};
-                        const uint32_t a1[4] = {va[u].z, vb[u].z, va[u].w, vb[u].w};
-                        mma_bf16_16816(acc[nt], a0, xv.x, xv.y);
-                        mma_bf16_16816(acc[nt], a1, xv.z, xv.w);
-                    }
+                for (int nt = 0; nt < NT; ++nt) {
+                    const int n = nt * 8 + g;
+                    const uint4 xv = n < M ? *reinterpret_cast<const uint4 *>(xs + (size_t)n * pitch + k + 8 * t)
+                                           : z4;
+                    const uint32_t a0[4] = {va[u].x, vb[u].x, va[u].y, vb[u].y};
+                    const uint32_t a1[4] = {va[u].z, vb[u].z, va[u].w, vb[u].w};
+                    mma_bf16_16816(acc[nt], a0, xv.x, xv.y);
+                    mma_bf16_16816(acc[nt], a1, xv.z, xv.w);
                 }
             }
         }
-        const int ra = r0 + g, rb = ra + 8;
+    }
+    const int ra = r0 + g, rb = ra + 8;
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-            const int m0 = nt * 8 + 2 * t, m1 = m0 + 1;
-            if (m0 < M) {
-                if (ra < N) y[(size_t)m0 * ldy + ra] = acc[nt][0];
-                if (rb < N) y[(size_t)m0 * ldy + rb] = acc[nt][2];
-            }
-            if (m1 < M) {
-                if (ra < N) y[(size_t)m1 * ldy + ra] = acc[nt][1];
-                if (rb < N) y[(size_t)m1 * ldy + rb] = acc[nt][3];
-            }
+    for (int nt = 0; nt < NT; ++nt) {
+        const int m0 = nt * 8 + 2 * t, m1 = m0 + 1;
+        if (m0 < M) {
+            if (ra < N) y[(size_t)m0 * ldy + ra] = acc[nt][0];
+            if (rb < N) y[(size_t)m0 * ldy + rb] = acc[nt][2];
+        }
+        if (m1 < M) {
+            if (ra < N) y[(size_t)m1 * ldy + ra] = acc[nt][1];
+            if (rb < N) y[(size_t)m1 * ldy + rb] = acc[nt][3];
         }
     }
+}
+
+// M <= 8 * NT rows: the CTA stages x, then its warps walk the 16-row tiles.
+template <int NT, int U>
+__global__ void __launch_bounds__(kBmmaThreads, 1) lm_head_bf16_mma_kernel(
+    const uint16_t *__restrict__ x, int M, int Kd, int N, const uint16_t *__restrict__ W,
+    float *__restrict__ y, int ldy) {
+    extern __shared__ uint4 smem_bm[];
+    uint16_t *xs = reinterpret_cast<uint16_t *>(smem_bm);
+    bf16_mma_stage_x(xs, x, M, Kd);
+    __syncthreads();
+    const int warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+    const int ntiles = (N + 15) / 16;
+    for (int tile = blockIdx.x * nwarps + warp; tile < ntiles; tile += gridDim.x * nwarps)
+        bf16_mma_tile<NT, U>(xs, M, Kd, N, W, y, ldy, tile);
 }
 
 // ---------------------------------------------------------------------------
@@ -770,20 +691,20 @@ __global__ void __launch_bounds__(kGemvThreads) splitk_reduce_kernel(const float
 }
 
 constexpr int kMixWarps = 16;      // per CTA, one CTA per SM
-constexpr int kMixInt4Warps = 4;   // the last 4 warps of a CTA own int4 rings
+constexpr int kMixInt4Warps = 3;   // the last 3 warps of a CTA own int4 rings
 constexpr int kMixThreads = 32 * kMixWarps;
 
 // Both heads of a verify step in one persistent launch.  The last
 // kMixInt4Warps warps of every CTA first stream their share of the int4 head
 // through their cp.async rings (bound by dequantisation and copy latency, not
-// by HBM), then join the other warps on the bf16 head, whose 4-row groups all
+// by HBM), then join the other warps on the bf16 head, whose 16-row tiles all
 // warps take one at a time from a global counter (`work`, zero on entry), so
 // the bf16 stream keeps every SM busy to the end whatever the int4 warps'
 // speed.  Each head's values are bit-identical to its own kernel's (same
-// device functions).
-template <int MT, int RW, int U, int GPS, int NST>
+// device functions, same tile shapes).
+template <int GPS, int NST>
 __global__ void __launch_bounds__(kMixThreads, 1) lm_heads_mixed_kernel(
-    const uint16_t *__restrict__ xt, const uint16_t *__restrict__ W, float *__restrict__ yt,
+    const uint16_t *__restrict__ xt, int Mt, const uint16_t *__restrict__ W, float *__restrict__ yt,
     const uint16_t *__restrict__ xd, int Md, const uint8_t *__restrict__ Wq,
     const uint16_t *__restrict__ S, float *__restrict__ yd, int Kd, int N, unsigned int *work) {
     using R = Int4Ring<GPS, NST>;
@@ -792,12 +713,12 @@ __global__ void __launch_bounds__(kMixThreads, 1) lm_heads_mixed_kernel(
     __shared__ float row_unscale[8];
     const int Gt = Kd >> 6;
     const int rowc = Gt * 8 + 1;
-    float *xsf = reinterpret_cast<float *>(smem_mix);                         // [MT][Kd] fp32
-    uint4 *x4 = smem_mix + (size_t)MT * Kd / 4;                               // int4 staging
+    uint16_t *xst = reinterpret_cast<uint16_t *>(smem_mix);                   // [Mt][Kd + 32] bf16
+    uint4 *x4 = smem_mix + (size_t)Mt * (Kd + 32) / 8;                        // int4 staging
     uint16_t *xb = reinterpret_cast<uint16_t *>(x4);                          // [Md + 1][rowc * 8]
     float *xs = reinterpret_cast<float *>(x4 + (size_t)(Md + 1) * rowc);      // [Gt][8]
     unsigned char *rings = reinterpret_cast<unsigned char *>(xs + Gt * 8);    // [int4 warps][NST][stage]
-    bf16_stage_x<MT>(xsf, xt, Kd);
+    bf16_mma_stage_x(xst, xt, Mt, Kd);
     int4_f16_stage_x(xb, xs, row_amax, row_unscale, xd, Md, Kd, true);  // ends with a block barrier
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int w4 = warp - (kMixWarps - kMixInt4Warps);
@@ -805,44 +726,26 @@ __global__ void __launch_bounds__(kMixThreads, 1) lm_heads_mixed_kernel(
         int4_f16_tiles<GPS, NST>(x4, xs, row_unscale, rings + (size_t)w4 * R::kWarpBytes, Md, Kd, N,
                                  Wq, S, yd, N, blockIdx.x * kMixInt4Warps + w4,
                                  gridDim.x * kMixInt4Warps);
-    const unsigned groups = (unsigned)((N + RW - 1) / RW);
+    const unsigned tiles = (unsigned)((N + 15) / 16);
     for (;;) {
         unsigned g = 0;
         if (lane == 0) g = atomicAdd(work, 1u);
         g = __shfl_sync(0xffffffffu, g, 0);
-        if (g >= groups) break;
-        bf16_group<MT, RW, U>(xsf, Kd, N, W, yt, N, (int)g);
+        if (g >= tiles) break;
+        bf16_mma_tile<1, kBmmaU>(xst, Mt, Kd, N, W, yt, N, (int)g);
     }
 }
 
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int M>
-static cudaError_t launch_bf16(const uint16_t *x, int Kd, int N, const uint16_t *W, float *y,
-                               int ldy, cudaStream_t s) {
-    constexpr int RW = M <= 4 ? 4 : 2;
-    constexpr int U = M <= 4 ? 4 : 2;
-    auto k = lm_head_bf16_xf32_kernel<M, RW, U>;
-    const size_t smem = (size_t)M * Kd * sizeof(float);
-    int occ = 0;
-    cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ);
-    if (e != cudaSuccess) return e;
-    const int groups = (N + RW - 1) / RW;
-    const int need = (groups + kGemvWarps - 1) / kGemvWarps;
-    const int grid = std::min(need, kSMs * occ);
-    k<<<grid, kGemvThreads, smem, s>>>(x, Kd, N, W, y, ldy);
-    return cudaGetLastError();
-}
-
 // Shared memory of the tensor-core bf16 kernel for M (<= 16) rows.
 static size_t bf16_mma_smem(int M, int Kd) { return (size_t)M * (Kd + 32) * 2; }
 
 template <int NT>
 static cudaError_t launch_bf16_mma(const uint16_t *x, int M, int Kd, int N, const uint16_t *W,
                                    float *y, int ldy, cudaStream_t s) {
-    constexpr int U = 8;
-    auto k = lm_head_bf16_mma_kernel<NT, U>;
+    auto k = lm_head_bf16_mma_kernel<NT, kBmmaU>;
     const size_t smem = bf16_mma_smem(M, Kd);
     int occ = 0;
     cudaError_t e = kernel_setup((const void *)k, kBmmaThreads, smem, &occ);
@@ -903,44 +806,32 @@ static cudaError_t launch_int4_direct(const uint16_t *x, int M, int Kd, int N, c
 
 static size_t heads_pair_smem(int Mt, int Md, int Kd) {
     const size_t Gt = (size_t)Kd / 64;
-    return (size_t)Mt * Kd * sizeof(float) + (size_t)(Md + 1) * (Gt * 8 + 1) * 16 +
-           Gt * 8 * sizeof(float) + (size_t)kMixInt4Warps * Int4Ring<kF16Gps, kF16Nst>::kWarpBytes;
+    return bf16_mma_smem(Mt, Kd) + (size_t)(Md + 1) * (Gt * 8 + 1) * 16 + Gt * 8 * sizeof(float) +
+           (size_t)kMixInt4Warps * Int4Ring<kF16Gps, kF16Nst>::kWarpBytes;
 }
 
 bool lm_heads_pair_ok(int Mt, int Md, int Kd, const void *scales) {
-    return Mt >= 1 && Mt <= 4 && Md >= 1 && Md <= 8 && Kd % (64 * kF16Gps) == 0 &&
+    return Mt >= 1 && Mt <= 8 && Md >= 1 && Md <= 8 && Kd % (64 * kF16Gps) == 0 &&
            ((uintptr_t)scales & 15) == 0 && heads_pair_smem(Mt, Md, Kd) <= (size_t)227 * 1024 - 256;
-}
-
-template <int MT>
-static cudaError_t launch_pair(const uint16_t *xt, const uint16_t *W, float *yt, const uint16_t *xd,
-                               int Md, const uint8_t *Wq, const uint16_t *S, float *yd, int Kd,
-                               int N, unsigned int *work, cudaStream_t s) {
-    auto k = lm_heads_mixed_kernel<MT, 4, 4, kF16Gps, kF16Nst>;
-    const size_t smem = heads_pair_smem(MT, Md, Kd);
-    int occ = 0;
-    cudaError_t e = kernel_setup((const void *)k, kMixThreads, smem, &occ);
-    if (e != cudaSuccess) return e;
-    e = cudaMemsetAsync(work, 0, sizeof(unsigned int), s);
-    if (e != cudaSuccess) return e;
-    k<<<kSMs * occ, kMixThreads, smem, s>>>(xt, W, yt, xd, Md, Wq, S, yd, Kd, N, work);
-    return cudaGetLastError();
 }
 
 cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
                                  int Md, const void *wq, const void *scales, float *yd, int Kd,
                                  int N, void *work, cudaStream_t s) {
     if (!lm_heads_pair_ok(Mt, Md, Kd, scales) || !work) return cudaErrorInvalidValue;
-    const uint16_t *xt16 = static_cast<const uint16_t *>(xt), *xd16 = static_cast<const uint16_t *>(xd);
-    const uint16_t *W = static_cast<const uint16_t *>(w), *S = static_cast<const uint16_t *>(scales);
-    const uint8_t *Wq = static_cast<const uint8_t *>(wq);
+    auto k = lm_heads_mixed_kernel<kF16Gps, kF16Nst>;
+    const size_t smem = heads_pair_smem(Mt, Md, Kd);
+    int occ = 0;
+    cudaError_t e = kernel_setup((const void *)k, kMixThreads, smem, &occ);
+    if (e != cudaSuccess) return e;
     unsigned int *wk = static_cast<unsigned int *>(work);
-    switch (Mt) {
-        case 1: return launch_pair<1>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
-        case 2: return launch_pair<2>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
-        case 3: return launch_pair<3>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
-        default: return launch_pair<4>(xt16, W, yt, xd16, Md, Wq, S, yd, Kd, N, wk, s);
-    }
+    e = cudaMemsetAsync(wk, 0, sizeof(unsigned int), s);
+    if (e != cudaSuccess) return e;
+    k<<<kSMs * occ, kMixThreads, smem, s>>>(
+        static_cast<const uint16_t *>(xt), Mt, static_cast<const uint16_t *>(w), yt,
+        static_cast<const uint16_t *>(xd), Md, static_cast<const uint8_t *>(wq),
+        static_cast<const uint16_t *>(scales), yd, Kd, N, wk);
+    return cudaGetLastError();
 }
 
 // ---- split-K projection ----------------------------------------------------
@@ -1017,18 +908,23 @@ cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq
 }
 
 size_t lm_head_max_smem_rows(int Kd) {
-    // rows of fp32 activations that fit in 227 KB of shared memory
+    // rows of 4 Kd bytes that fit in 227 KB of shared memory: the shape bound
+    // of both heads (Kd <= 58112) and the int4 row grouping
     return (size_t)(227 * 1024) / ((size_t)Kd * sizeof(float));
 }
 
 cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, const void *scales,
                            int fmt, float *y, cudaStream_t s) {
     const uint16_t *xb = static_cast<const uint16_t *>(x);
-    if (fmt == MTPV_W_BF16 && M > 8 && bf16_mma_smem(16, Kd) <= (size_t)227 * 1024) {
-        // more than 8 rows: the tensor-core kernel, up to 16 rows per pass
+    if (fmt == MTPV_W_BF16) {
+        // the tensor-core kernel: 16 rows per pass when more than 8 rows come
+        // and 16 staged rows fit, else passes of up to 8 rows
         const uint16_t *W = static_cast<const uint16_t *>(w);
-        for (int m0 = 0; m0 < M; m0 += 16) {
-            const int mm = std::min(16, M - m0);
+        const size_t fit = (size_t)227 * 1024 / bf16_mma_smem(1, Kd);
+        if (fit < 1) return cudaErrorInvalidValue;
+        const int step = (M > 8 && fit >= 16) ? 16 : (int)std::min<size_t>(8, fit);
+        for (int m0 = 0; m0 < M; m0 += step) {
+            const int mm = std::min(step, M - m0);
             const cudaError_t e =
                 mm > 8 ? launch_bf16_mma<2>(xb + (size_t)m0 * Kd, mm, Kd, N, W, y + (size_t)m0 * N, N, s)
                        : launch_bf16_mma<1>(xb + (size_t)m0 * Kd, mm, Kd, N, W, y + (size_t)m0 * N, N, s);
@@ -1036,40 +932,23 @@ cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, c
         }
         return cudaSuccess;
     }
+    // int4 group-64: passes of up to 8 rows, each on the ring kernel when it
+    // takes the shape, else on the direct-load kernel (same bits)
     const int step = (int)std::min<size_t>(8, lm_head_max_smem_rows(Kd));
     if (step < 1) return cudaErrorInvalidValue;
+    const uint8_t *Wq = static_cast<const uint8_t *>(w);
+    const uint16_t *S = static_cast<const uint16_t *>(scales);
     for (int m0 = 0; m0 < M; m0 += step) {
         const int mm = std::min(step, M - m0);
         const uint16_t *xm = xb + (size_t)m0 * Kd;
         float *ym = y + (size_t)m0 * N;
-        cudaError_t e = cudaSuccess;
-        if (fmt == MTPV_W_BF16) {
-            const uint16_t *W = static_cast<const uint16_t *>(w);
-            switch (mm) {
-                case 1: e = launch_bf16<1>(xm, Kd, N, W, ym, N, s); break;
-                case 2: e = launch_bf16<2>(xm, Kd, N, W, ym, N, s); break;
-                case 3: e = launch_bf16<3>(xm, Kd, N, W, ym, N, s); break;
-                case 4: e = launch_bf16<4>(xm, Kd, N, W, ym, N, s); break;
-                case 5: e = launch_bf16<5>(xm, Kd, N, W, ym, N, s); break;
-                case 6: e = launch_bf16<6>(xm, Kd, N, W, ym, N, s); break;
-                case 7: e = launch_bf16<7>(xm, Kd, N, W, ym, N, s); break;
-                default: e = launch_bf16<8>(xm, Kd, N, W, ym, N, s); break;
-            }
-        } else {
-            const uint8_t *Wq = static_cast<const uint8_t *>(w);
-            const uint16_t *S = static_cast<const uint16_t *>(scales);
-            if (int4_f16_ok(mm, Kd, S)) {
-                e = launch_int4_f16(xm, mm, Kd, N, Wq, S, ym, N, s);
-                if (e != cudaSuccess) return e;
-                continue;
-            }
-            if (int4_direct_smem(mm, Kd) <= (size_t)227 * 1024) {
-                e = launch_int4_direct(xm, mm, Kd, N, Wq, S, ym, N, s);
-                if (e != cudaSuccess) return e;
-                continue;
-            }
+        cudaError_t e;
+        if (int4_f16_ok(mm, Kd, S))
+            e = launch_int4_f16(xm, mm, Kd, N, Wq, S, ym, N, s);
+        else if (int4_direct_smem(mm, Kd) <= (size_t)227 * 1024)
+            e = launch_int4_direct(xm, mm, Kd, N, Wq, S, ym, N, s);
+        else
             return cudaErrorInvalidValue;  // no int4 kernel for this shape
-        }
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;

@@ -6,7 +6,8 @@
 
 namespace mtpv {
 
-// Rows of activations of length Kd that one launch can stage (as fp32) in shared memory.
+// Rows of 4 Kd bytes that fit in 227 KB of shared memory: at least 1 for every
+// supported Kd (<= 58112); the int4 path takes passes of min(8, this) rows.
 size_t lm_head_max_smem_rows(int Kd);
 
 // y[M, N] = x[M, Kd] . Wd[N, Kd]^T; fmt is an mtpv_wfmt.  Arguments are

@@ -67,12 +67,11 @@ constexpr int kExpTab = 64;         // entries of the exp table (2^(j/64))
 // Dynamic shared memory of the statistics kernel: a region reused phase by
 // phase, then the small bookkeeping struct.
 //   region: [logits slice: kCacheFloats fp32][their exps: kCacheFloats fp64]
-//           [hist_mass: kBins fp64][hist_cnt: kBins int][cand: kCandCap u64]
+//           [hist_mass: kBins fp64][cand: kCandCap u64]
 //           [cand_e: kCandCap fp64]
 constexpr size_t kOffExp = kCacheFloats * sizeof(float);
 constexpr size_t kOffHistMass = kOffExp + kCacheFloats * sizeof(double);
-constexpr size_t kOffHistCnt = kOffHistMass + kBins * sizeof(double);
-constexpr size_t kOffCand = kOffHistCnt + kBins * sizeof(int);
+constexpr size_t kOffCand = kOffHistMass + kBins * sizeof(double);
 constexpr size_t kOffCandE = kOffCand + kCandCap * sizeof(unsigned long long);
 constexpr size_t kRegionBytes = kOffCandE + kCandCap * sizeof(double);
 static_assert(kOffExp % 16 == 0 && kOffHistMass % 16 == 0, "region alignment");
@@ -96,7 +95,7 @@ struct SamplerSmem {
     int pub_arg, pub_bad;
     double pub_Z, pub_range_total, pub_partial;
     // broadcast into every CTA of the cluster
-    int bc_bin, bc_cnt, bc_last;
+    int bc_bin;
     double bc_A;
     unsigned int cand_count;
     unsigned int local_n, local_base;
@@ -117,7 +116,6 @@ struct Region {
     float *cache;
     double *ecache;
     double *hist_mass;
-    int *hist_cnt;
     unsigned long long *cand;
     double *cand_e;
 };
@@ -514,7 +512,6 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     rg.cache = reinterpret_cast<float *>(smem_raw);
     rg.ecache = reinterpret_cast<double *>(smem_raw + kOffExp);
     rg.hist_mass = reinterpret_cast<double *>(smem_raw + kOffHistMass);
-    rg.hist_cnt = reinterpret_cast<int *>(smem_raw + kOffHistCnt);
     rg.cand = reinterpret_cast<unsigned long long *>(smem_raw + kOffCand);
     rg.cand_e = reinterpret_cast<double *>(smem_raw + kOffCandE);
     float *cache = rg.cache;
@@ -620,7 +617,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
         float inv_w = (range > 0.0f) ? __fdiv_rn((float)kBins, range) : 0.0f;
         if (!isfinite(inv_w)) inv_w = 0.0f;
         if (!topp_all) {
-            for (int b = tid; b < kBins; b += kThreads) { rg.hist_mass[b] = 0.0; rg.hist_cnt[b] = 0; }
+            for (int b = tid; b < kBins; b += kThreads) rg.hist_mass[b] = 0.0;
             __syncthreads();
         }
         double zt = 0.0;
@@ -643,7 +640,6 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                     if (!topp_all) {
                         const int b = bin_of(lv[q], m, inv_w);
                         atomicAdd(&rg.hist_mass[b], ev[q]);
-                        atomicAdd(&rg.hist_cnt[b], 1);
                     }
                 }
             }
@@ -671,26 +667,16 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 constexpr int kPasses = kBins / kThreads;
                 const int bpp = kThreads / C, r = tid % C;
                 double vv[kPasses];
-                int cc[kPasses];
 #pragma unroll
                 for (int q = 0; q < kPasses; ++q) {
                     const int b = q * bpp + tid / C;
                     vv[q] = cluster.map_shared_rank(rg.hist_mass, r)[base + b];
-                    cc[q] = cluster.map_shared_rank(rg.hist_cnt, r)[base + b];
                 }
 #pragma unroll
                 for (int q = 0; q < kPasses; ++q) {
                     double v = vv[q];
-                    int cn = cc[q];
-                    for (int o = C >> 1; o > 0; o >>= 1) {
-                        v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-                        cn += __shfl_xor_sync(0xffffffffu, cn, o);
-                    }
-                    if (r == 0) {
-                        const int b = q * bpp + tid / C;
-                        s.own_mass[b] = v;
-                        s.own_cnt[b] = cn;
-                    }
+                    for (int o = C >> 1; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+                    if (r == 0) s.own_mass[q * bpp + tid / C] = v;
                 }
             }
             __syncthreads();
@@ -711,7 +697,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                     if (cstar < 0 && nx >= thr) { cstar = r; Pstar = P; }
                     P = nx;
                 }
-                int bstar = -2, cnt = 0;
+                int bstar = -2;
                 double A = P;
                 if (cstar == rank) {
                     int f;
@@ -719,26 +705,24 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                     warp_prefix_search(s.own_mass, per, Pstar, thr, true, &f, &bef);
                     if (f < 0) f = per - 1;  // not reachable: the range total reached thr
                     bstar = base + f;
-                    cnt = s.own_cnt[f];
                     A = bef;
                 } else if (cstar < 0 && rank == 0) {
                     bstar = -1;  // thr above the histogram total (top_p within rounding of 1)
                 }
                 if (bstar != -2 && lane < C) {
                     *cluster.map_shared_rank(&s.bc_bin, lane) = bstar;
-                    *cluster.map_shared_rank(&s.bc_cnt, lane) = cnt;
                     *cluster.map_shared_rank(&s.bc_A, lane) = A;
                 }
             }
             cluster.sync();
             const int bstar = s.bc_bin;
-            const int cnt = s.bc_cnt;
             const double A = s.bc_A;
-            if (bstar < 0 || cnt == 0) {
-                st.Zk = st.Z;  // nothing to cut (top_p within rounding of 1): keep all
-            } else if (cnt <= kCandCap) {
-                // gather the crossing bin's tokens into CTA 0: stage them
-                // locally, reserve a range with one remote atomic, copy
+            // gather the crossing bin's tokens into CTA 0: stage them
+            // locally, reserve a range with one remote atomic, copy.  The
+            // bin's size is known once every CTA has reserved its range; a bin
+            // above the candidate capacity takes the radix select instead.
+            unsigned total = 0u;
+            if (bstar >= 0) {
                 unsigned long long *stage = reinterpret_cast<unsigned long long *>(rg.cand_e);
                 if (tid == 0) s.local_n = 0u;
                 __syncthreads();
@@ -761,6 +745,11 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                         if (b0 + i < (unsigned)kCandCap) ck[b0 + i] = stage[i];
                 }
                 cluster.sync();
+                total = *cluster.map_shared_rank(&s.cand_count, 0);
+            }
+            if (bstar < 0 || total == 0u) {
+                st.Zk = st.Z;  // nothing to cut (top_p within rounding of 1): keep all
+            } else if (total <= (unsigned)kCandCap) {
                 if (rank == 0) {
                     const int n = min((int)s.cand_count, kCandCap);
                     int n2 = 1;
