@@ -63,6 +63,7 @@ constexpr int kCandCap = 4096;
 constexpr int kCacheFloats = 9728;  // logits slice kept in shared memory (38 KB), and its exps
 constexpr int kBatch = 8;           // loads in flight per thread in streaming loops
 constexpr int kExpTab = 64;         // entries of the exp table (2^(j/64))
+constexpr int kMaxCluster = 16;     // CTAs per cluster (16, or 8 where 16 cannot be resident)
 
 // Dynamic shared memory of the statistics kernel: a region reused phase by
 // phase, then the small bookkeeping struct.
@@ -90,10 +91,12 @@ struct SamplerSmem {
     int red_i2[kWarps];
     double warp_tot[kWarps];
     double thr_excl[kThreads];
-    // published to the other CTAs of the cluster
-    float pub_max, pub_min;
-    int pub_arg, pub_bad;
-    double pub_Z, pub_range_total, pub_partial;
+    // written by every CTA of the cluster into every CTA (slot = the writer's
+    // rank) before a cluster barrier, read locally after it
+    float all_max[kMaxCluster], all_min[kMaxCluster];
+    int all_arg[kMaxCluster], all_bad[kMaxCluster];
+    double all_Z[kMaxCluster], all_rt[kMaxCluster], all_part[kMaxCluster];
+    double my_partial;
     // broadcast into every CTA of the cluster
     int bc_bin;
     double bc_A;
@@ -222,14 +225,30 @@ __device__ double block_sum_d(double v, SamplerSmem &s) {
     return r;
 }
 
-// Sum over the CTAs of the cluster of the double at `addr` (one per CTA),
-// accumulated in rank order by every lane of the calling warp: lane r reads
-// rank r (the remote loads overlap), a broadcast shuffle chain adds them in a
-// fixed order.  *excl gets the sum of the ranks before `want`.
-__device__ __forceinline__ double cluster_sum_ordered(cg::cluster_group &cl, double *addr, int C,
-                                                      int want, double *excl) {
+// Programmatic dependent launch: wait until the grids this one depends on
+// have completed and their writes are visible; let dependents be scheduled.
+__device__ __forceinline__ void wait_for_producer() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Warp-wide (max with its lowest index, min, or) of per-lane partials; every
+// lane ends with the result.
+__device__ __forceinline__ void warp_max_min_arg(float &mx, int &arg, float &mn, int &bad) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+        const float om = __shfl_xor_sync(0xffffffffu, mx, o);
+        const int oa = __shfl_xor_sync(0xffffffffu, arg, o);
+        if (om > mx || (om == mx && oa < arg)) { mx = om; arg = oa; }
+        mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        bad |= __shfl_xor_sync(0xffffffffu, bad, o);
+    }
+}
+
+// Sum of vals[0..C) (one per CTA of the cluster, already in this CTA's shared
+// memory), accumulated in rank order by every lane of the calling warp (a
+// broadcast shuffle chain).  *excl gets the sum of the ranks before `want`.
+__device__ __forceinline__ double ordered_sum(const double *vals, int C, int want, double *excl) {
     const int lane = threadIdx.x & 31;
-    const double v = lane < C ? *cl.map_shared_rank(addr, lane) : 0.0;
+    const double v = lane < C ? vals[lane] : 0.0;
     double acc = 0.0, ex = 0.0;
     for (int r = 0; r < C; ++r) {
         const double vr = __shfl_sync(0xffffffffu, v, r);
@@ -238,6 +257,14 @@ __device__ __forceinline__ double cluster_sum_ordered(cg::cluster_group &cl, dou
     }
     if (excl) *excl = ex;
     return acc;
+}
+
+// Write v into slot `rank` of arr in every CTA of the cluster: lanes 0..C-1
+// of the calling warp each store to one CTA (v uniform over the warp).
+template <typename T>
+__device__ __forceinline__ void publish(cg::cluster_group &cl, T *arr, int rank, int C, T v) {
+    const int lane = threadIdx.x & 31;
+    if (lane < C) *cl.map_shared_rank(arr + rank, lane) = v;
 }
 
 // Warp-cooperative ordered prefix over a[0..n) (n a multiple of 32): lane l
@@ -438,28 +465,30 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
         }
         if (lane == 0) s.warp_tot[w] = acc;
         __syncthreads();
-        if (tid == 0) {
+        if (w == 0) {
             double a = 0.0;
             for (int i = 0; i < kWarps; ++i) a = __dadd_rn(a, s.warp_tot[i]);
-            s.pub_partial = a;
+            if (lane == 0) s.my_partial = a;
+            publish(cluster, s.all_part, rank, C, a);
         }
         cluster.sync();
         if (w == 0) {
             double pc = 0.0;
-            const double tot = cluster_sum_ordered(cluster, &s.pub_partial, C, rank, &pc);
+            const double tot = ordered_sum(s.all_part, C, rank, &pc);
             if (lane == 0) {
                 s.draw_Pc = pc;
                 s.draw_total = tot;
             }
         }
-        cluster.sync();  // all peers have read pub_partial
+        __syncthreads();
         const double Pc = s.draw_Pc, total = s.draw_total;
         if (total == 0.0 && allow_fallback && src.kind == 1) {
             src.kind = 0;  // p' == q' exactly: draw from p'_n
+            cluster.sync();  // every CTA has read all_part before the next attempt rewrites it
             continue;
         }
         const double target = __dmul_rn((double)u, total);
-        const double next = __dadd_rn(Pc, s.pub_partial);
+        const double next = __dadd_rn(Pc, s.my_partial);
         if (!(Pc <= target && target < next)) return;  // the crossing is in another CTA
         if (tid == 0) {
             double a = 0.0, om = 0.0;
@@ -531,6 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     const bool topp_all = !(p.top_p < 1.0f);
     double *erow = p.ecache ? p.ecache + (size_t)row * V : nullptr;
     build_exp_table(s.exp_tab);  // first used after the P1 barriers
+    allow_dependents();          // the draw kernel waits for this grid's completion itself
+    wait_for_producer();         // the logits
     if (p.verify && row == 0 && rank == 0)  // ticket counters of the draw kernel
         for (int k = tid; k < p.B; k += kThreads) p.counters[k] = 0u;
     auto lval = [&](int j) -> float { return cached ? cache[j - v0] : L[j]; };
@@ -560,39 +591,28 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 }
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            float om = __shfl_xor_sync(0xffffffffu, mx, o);
-            int oa = __shfl_xor_sync(0xffffffffu, arg, o);
-            if (om > mx || (om == mx && oa < arg)) { mx = om; arg = oa; }
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-            bad |= __shfl_xor_sync(0xffffffffu, bad, o);
-        }
+        warp_max_min_arg(mx, arg, mn, bad);
         if (lane == 0) { s.red_f[wid] = mx; s.red_f2[wid] = mn; s.red_i[wid] = arg; s.red_i2[wid] = bad; }
         __syncthreads();
-        if (tid == 0) {
-            mx = s.red_f[0]; arg = s.red_i[0]; mn = s.red_f2[0]; bad = s.red_i2[0];
-            for (int i = 1; i < kWarps; ++i) {
-                if (s.red_f[i] > mx || (s.red_f[i] == mx && s.red_i[i] < arg)) { mx = s.red_f[i]; arg = s.red_i[i]; }
-                mn = fminf(mn, s.red_f2[i]);
-                bad |= s.red_i2[i];
-            }
-            s.pub_max = mx; s.pub_min = mn; s.pub_arg = arg; s.pub_bad = bad;
+        // the CTA's result in every lane of warp 0, published into every CTA
+        if (wid == 0) {
+            float bm = lane < kWarps ? s.red_f[lane] : -INFINITY;
+            int ba = lane < kWarps ? s.red_i[lane] : INT_MAX;
+            float bn = lane < kWarps ? s.red_f2[lane] : INFINITY;
+            int bb = lane < kWarps ? s.red_i2[lane] : 0;
+            warp_max_min_arg(bm, ba, bn, bb);
+            publish(cluster, s.all_max, rank, C, bm);
+            publish(cluster, s.all_arg, rank, C, ba);
+            publish(cluster, s.all_min, rank, C, bn);
+            publish(cluster, s.all_bad, rank, C, bb);
         }
         cluster.sync();
         if (wid == 0) {
-            float gm = lane < C ? *cluster.map_shared_rank(&s.pub_max, lane) : -INFINITY;
-            int ga = lane < C ? *cluster.map_shared_rank(&s.pub_arg, lane) : INT_MAX;
-            float gn = lane < C ? *cluster.map_shared_rank(&s.pub_min, lane) : INFINITY;
-            int gb = lane < C ? *cluster.map_shared_rank(&s.pub_bad, lane) : 0;
-#pragma unroll
-            for (int o = 16; o > 0; o >>= 1) {
-                const float om = __shfl_xor_sync(0xffffffffu, gm, o);
-                const int oa = __shfl_xor_sync(0xffffffffu, ga, o);
-                if (om > gm || (om == gm && oa < ga)) { gm = om; ga = oa; }
-                gn = fminf(gn, __shfl_xor_sync(0xffffffffu, gn, o));
-                gb |= __shfl_xor_sync(0xffffffffu, gb, o);
-            }
+            float gm = lane < C ? s.all_max[lane] : -INFINITY;
+            int ga = lane < C ? s.all_arg[lane] : INT_MAX;
+            float gn = lane < C ? s.all_min[lane] : INFINITY;
+            int gb = lane < C ? s.all_bad[lane] : 0;
+            warp_max_min_arg(gm, ga, gn, gb);
             if (lane == 0) { s.g_m = gm; s.g_min = gn; s.g_arg = ga; s.g_bad = gb; }
         }
         __syncthreads();
@@ -644,11 +664,23 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 }
             }
         }
-        const double zc = block_sum_d(zt, s);
-        if (tid == 0) { s.pub_Z = zc; s.cand_count = 0u; }
+        const double zc = block_sum_d(zt, s);  // its barriers also complete the histogram
+        // publish Z, and send every CTA the part of this CTA's histogram that
+        // it owns (bins [r per, (r + 1) per) to CTA r, slot rank): warp r
+        // copies one contiguous run into CTA r's scratch (the candidate area,
+        // unused until the gather)
+        const int per = kBins / C;
+        if (wid == 0) publish(cluster, s.all_Z, rank, C, zc);
+        if (tid == 0) s.cand_count = 0u;
+        if (!topp_all) {
+            for (int r = wid; r < C; r += kWarps) {
+                double *dst = reinterpret_cast<double *>(cluster.map_shared_rank(rg.cand, r)) + rank * per;
+                for (int i = lane; i < per; i += 32) dst[i] = rg.hist_mass[r * per + i];
+            }
+        }
         cluster.sync();
         if (wid == 0) {
-            const double z = cluster_sum_ordered(cluster, &s.pub_Z, C, 0, nullptr);
+            const double z = ordered_sum(s.all_Z, C, 0, nullptr);
             if (lane == 0) s.g_Z = z;
         }
         __syncthreads();
@@ -658,25 +690,15 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
         if (!topp_all) {
             // ---------------- P3: crossing bin, exact cut ----------------
             const double thr = __dmul_rn((double)p.top_p, st.Z);
-            const int per = kBins / C;
             const int base = rank * per;
-            // merge the cluster's histograms for the bins this CTA owns: C
-            // lanes per bin, one remote load each (all issued together), a
-            // fixed shuffle tree
+            // the cluster's histogram on the bins this CTA owns: the C copies
+            // added in rank order
             {
-                constexpr int kPasses = kBins / kThreads;
-                const int bpp = kThreads / C, r = tid % C;
-                double vv[kPasses];
-#pragma unroll
-                for (int q = 0; q < kPasses; ++q) {
-                    const int b = q * bpp + tid / C;
-                    vv[q] = cluster.map_shared_rank(rg.hist_mass, r)[base + b];
-                }
-#pragma unroll
-                for (int q = 0; q < kPasses; ++q) {
-                    double v = vv[q];
-                    for (int o = C >> 1; o > 0; o >>= 1) v = __dadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
-                    if (r == 0) s.own_mass[q * bpp + tid / C] = v;
+                const double *scr = reinterpret_cast<const double *>(rg.cand);
+                for (int b = tid; b < per; b += kThreads) {
+                    double a = 0.0;
+                    for (int r = 0; r < C; ++r) a = __dadd_rn(a, scr[r * per + b]);
+                    s.own_mass[b] = a;
                 }
             }
             __syncthreads();
@@ -684,12 +706,12 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 int f;
                 double bef;
                 const double t = warp_prefix_search(s.own_mass, per, 0.0, 0.0, false, &f, &bef);
-                if (lane == 0) s.pub_range_total = t;
+                publish(cluster, s.all_rt, rank, C, t);
             }
             cluster.sync();
             if (wid == 0) {
                 // first range whose inclusive prefix reaches thr (same order everywhere)
-                const double v = lane < C ? *cluster.map_shared_rank(&s.pub_range_total, lane) : 0.0;
+                const double v = lane < C ? s.all_rt[lane] : 0.0;
                 double P = 0.0, Pstar = 0.0;
                 int cstar = -1;
                 for (int r = 0; r < C; ++r) {
@@ -957,6 +979,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
     }
     build_exp_table(s.exp_tab);
     __syncthreads();
+    wait_for_producer();  // the statistics kernel's rows and weights
     const RowStats st_t = p.slots[rt].st;
     const RowStats st_d = p.slots[rd].st;
     const float *Lt = row_ptr(p, rt), *Ld = row_ptr(p, rd);
@@ -1086,6 +1109,10 @@ int cluster_size_for(int which, Kern kernel, size_t smem) {
     return best;
 }
 
+// Both sampler kernels are launched as programmatic dependents of the work
+// before them on the stream: their CTAs may be scheduled while that work
+// drains, and each waits (griddepcontrol.wait) for it to complete before
+// reading its results.
 template <typename Kern>
 cudaError_t launch_clusters(Kern kernel, int C, int clusters, size_t smem, const SamplerParams &p,
                             cudaStream_t stream) {
@@ -1094,13 +1121,15 @@ cudaError_t launch_clusters(Kern kernel, int C, int clusters, size_t smem, const
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute at[1];
+    cudaLaunchAttribute at[2];
     at[0].id = cudaLaunchAttributeClusterDimension;
     at[0].val.clusterDim.x = C;
     at[0].val.clusterDim.y = 1;
     at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = at;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kernel, p);
 }
 
