@@ -73,6 +73,8 @@ typedef enum {
 #define MTPV_ROW_OK 0
 #define MTPV_ROW_BAD_DRAFT 1    /* a draft token id outside [0, V)          */
 #define MTPV_ROW_NONFINITE 2    /* a NaN or +-inf logit in one of its rows  */
+#define MTPV_ROW_TIMEOUT 3      /* a bounded device-side wait gave up: the  */
+                                /* sequence's outputs are not valid         */
 
 /* Library version: major*10000 + minor*100 + patch. */
 MTPV_API int mtpv_version(void);

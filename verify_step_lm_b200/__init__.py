@@ -23,7 +23,7 @@ LIB_PATH = os.path.join(_HERE, "libmtpv.so")
 OK = 0
 W_BF16 = 0
 W_INT4_G64 = 1
-ROW_OK, ROW_BAD_DRAFT, ROW_NONFINITE = 0, 1, 2
+ROW_OK, ROW_BAD_DRAFT, ROW_NONFINITE, ROW_TIMEOUT = 0, 1, 2, 3
 
 _lib = None
 

@@ -76,7 +76,7 @@ constexpr size_t kOffCand = kOffHistMass + kBins * sizeof(double);
 constexpr size_t kOffCandE = kOffCand + kCandCap * sizeof(unsigned long long);
 constexpr size_t kRegionBytes = kOffCandE + kCandCap * sizeof(double);
 static_assert(kOffExp % 16 == 0 && kOffHistMass % 16 == 0, "region alignment");
-constexpr int kDrawBufDoubles = 16384;  // the draw kernel's weight buffer (128 KB)
+constexpr int kDrawBufDoubles = 19456;  // the draw kernel's weight buffer (152 KB: two rows' slices)
 constexpr size_t kDrawBufBytes = kDrawBufDoubles * sizeof(double);
 
 struct SamplerSmem {
@@ -109,6 +109,8 @@ struct SamplerSmem {
     int wstar, x_found, first_fail, cut_idx;
     float cut_l;
     int res_x, res_acc;  // draw kernel: the position's token and acceptance, in CTA 0
+    int res_timeout;     // draw kernel, CTA 0: a CTA of the cluster gave up waiting for a copy
+    unsigned long long bar;  // mbarrier of the bulk copies
     double exp_tab[kExpTab];  // 2^(j/64), for exp_neg
 };
 
@@ -229,6 +231,51 @@ __device__ double block_sum_d(double v, SamplerSmem &s) {
 // have completed and their writes are visible; let dependents be scheduled.
 __device__ __forceinline__ void wait_for_producer() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void allow_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Bulk copies between global and shared memory (the copy engine moves a whole
+// contiguous run; both addresses 16-byte aligned, the size a multiple of 16).
+// Completion of loads is tracked by an mbarrier with a byte count; every wait
+// is bounded (kWaitLimit polls) and reports whether the copy landed.
+constexpr int kWaitLimit = 1 << 20;
+__device__ __forceinline__ unsigned smem_u32(const void *p) { return (unsigned)__cvta_generic_to_shared(p); }
+__device__ __forceinline__ void mbar_init(unsigned long long *bar) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_u32(bar)) : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_expect(unsigned long long *bar, unsigned bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned bytes, unsigned long long *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, unsigned phase) {
+    for (int i = 0; i < kWaitLimit; ++i) {
+        unsigned done;
+        asm volatile(
+            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done)
+            : "r"(smem_u32(bar)), "r"(phase)
+            : "memory");
+        if (done) return true;
+    }
+    return false;
+}
+__device__ __forceinline__ bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
+// Shared -> global: the writing threads fence their generic stores into the
+// async proxy and meet at a barrier first; one thread issues and waits.
+__device__ __forceinline__ void fence_to_async_proxy() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+__device__ __forceinline__ void bulk_store_wait(void *dst, const void *src, unsigned bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
+                 "r"(bytes)
+                 : "memory");
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
 
 // Warp-wide (max with its lowest index, min, or) of per-lane partials; every
 // lane ends with the result.
@@ -431,12 +478,39 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
     const int n = v1 - v0;
     const int ch = (n + kThreads - 1) / kThreads;
     const int t0 = min(v1, v0 + tid * ch), t1 = min(v1, t0 + ch);
-    // weights computed once, coalesced, into shared memory; thread t's
-    // sub-chunk lives at wbuf[t * P ..] with an odd stride P (no bank conflicts)
+    // With the statistics kernel's weights, aligned, and room for both rows:
+    // the copy engine brings the slices of e_t (and e_d) into shared memory
+    // in vocabulary order, and the residual weights are formed in e_d's place
+    // (e_t stays intact for the fallback to p'_n).
+    const bool bulk = src.Et && n > 0 && (n & 1) == 0 && 2 * n <= kDrawBufDoubles &&
+                      aligned16(src.Et + v0) && (src.kind == 0 || aligned16(src.Ed + v0));
+    double *bt = wbuf, *bd = wbuf + n;
+    bool landed = true;
+    if (bulk) {
+        if (tid == 0) {
+            mbar_init(&s.bar);
+            const unsigned bytes = (unsigned)n * 8u;
+            mbar_expect(&s.bar, src.kind == 1 ? 2u * bytes : bytes);
+            bulk_load(bt, src.Et + v0, bytes, &s.bar);
+            if (src.kind == 1) bulk_load(bd, src.Ed + v0, bytes, &s.bar);
+        }
+        __syncthreads();  // the barrier is initialised before anyone polls it
+        landed = mbar_wait(&s.bar, 0);
+        if (!landed) mbar_wait(&s.bar, 0);  // give the copies in flight a second bound
+        if (src.kind == 1)
+            for (int i = tid; i < n; i += kThreads) bd[i] = draw_combine(src, bt[i], bd[i]);
+        __syncthreads();
+    }
+    // Otherwise weights are computed once, coalesced, into shared memory;
+    // thread t's sub-chunk lives at wbuf[t * P ..] with an odd stride P (no
+    // bank conflicts).
     const int P = ch | 1;
-    const bool buffered = ch > 0 && (size_t)kThreads * P <= (size_t)kDrawBufDoubles;
+    const bool buffered = !bulk && ch > 0 && (size_t)kThreads * P <= (size_t)kDrawBufDoubles;
     const double *mine = wbuf + (size_t)tid * P;
-    auto wat = [&](int j) -> double { return buffered ? mine[j - t0] : draw_weight(src, j, invT); };
+    auto wat = [&](int j) -> double {
+        if (bulk) return (src.kind == 1 ? bd : bt)[j - v0];
+        return buffered ? mine[j - t0] : draw_weight(src, j, invT);
+    };
 
     for (int attempt = 0; attempt < 2; ++attempt) {
         if (buffered) {
@@ -472,6 +546,7 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
             publish(cluster, s.all_part, rank, C, a);
         }
         cluster.sync();
+        if (!landed && tid == 0) *cluster.map_shared_rank(&s.res_timeout, 0) = 1;
         if (w == 0) {
             double pc = 0.0;
             const double tot = ordered_sum(s.all_part, C, rank, &pc);
@@ -922,7 +997,15 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     if (rank == 0 && tid == 0) p.slots[row].st = st;
     if (erow && !bad && T > 0.0) {
         const double md = (double)m;
-        if (cached) {
+        const int n = v1 - v0;
+        if (cached && n > 0 && (n & 1) == 0 && aligned16(erow + v0)) {
+            // masked in place, then one bulk copy of the slice
+            for (int j = v0 + tid; j < v1; j += kThreads)
+                if (!is_kept(st, rg.cache[j - v0], j)) rg.ecache[j - v0] = 0.0;
+            fence_to_async_proxy();
+            __syncthreads();
+            if (tid == 0) bulk_store_wait(erow + v0, rg.ecache, (unsigned)n * 8u);
+        } else if (cached) {
             for (int j = v0 + tid; j < v1; j += kThreads)
                 erow[j] = is_kept(st, rg.cache[j - v0], j) ? rg.ecache[j - v0] : 0.0;
         } else {
@@ -976,6 +1059,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
     if (rank == 0 && tid == 0) {
         s.res_x = -1;
         s.res_acc = 0;
+        s.res_timeout = 0;
     }
     build_exp_table(s.exp_tab);
     __syncthreads();
@@ -1028,7 +1112,15 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
     }
     if (rank == 0 && tid == 0 && !p.verify && p.row_status) p.row_status[c] = status;
     cluster.sync();  // verify: res_x and res_acc are in CTA 0; no CTA exits while a peer reads it
-    if (!p.verify || rank != 0 || tid != 0) return;
+    if (rank != 0 || tid != 0) return;
+    if (s.res_timeout) status = MTPV_ROW_TIMEOUT;
+    if (!p.verify) {
+        if (status == MTPV_ROW_TIMEOUT) {
+            p.out_tokens[c] = -1;
+            if (p.row_status) p.row_status[c] = status;
+        }
+        return;
+    }
 
     // ---------------- record, ticket, and (last cluster) the sequence's outputs ----------------
     const int S = 2 * K + 1;
