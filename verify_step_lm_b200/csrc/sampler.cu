@@ -290,6 +290,36 @@ __device__ __forceinline__ void warp_max_min_arg(float &mx, int &arg, float &mn,
     }
 }
 
+// Block-wide scan of one double per thread: Kogge-Stone inside each warp, the
+// warp totals chained in order by one thread, so that every thread's
+// exclusive value (*excl) is bit for bit the previous thread's inclusive one
+// (the return value).  Uses warp_tot and red_d; ends with a barrier.
+__device__ double block_scan_d(double v, SamplerSmem &s, double *excl) {
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    double x = v;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double u = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x = __dadd_rn(u, x);
+    }
+    const double prev = __shfl_up_sync(0xffffffffu, x, 1);
+    if (lane == 31) s.warp_tot[w] = x;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        double a = 0.0;
+        for (int i = 0; i < kWarps; ++i) {
+            s.red_d[i] = a;
+            a = __dadd_rn(a, s.warp_tot[i]);
+        }
+    }
+    __syncthreads();
+    const double off = s.red_d[w];
+    *excl = lane > 0 ? __dadd_rn(off, prev) : off;
+    const double incl = __dadd_rn(off, x);
+    __syncthreads();
+    return incl;
+}
+
 // Sum of vals[0..C) (one per CTA of the cluster, already in this CTA's shared
 // memory), accumulated in rank order by every lane of the calling warp (a
 // broadcast shuffle chain).  *excl gets the sum of the ranks before `want`.
@@ -357,32 +387,6 @@ __device__ double warp_prefix_search(const double *a, int n, double base, double
         }
     }
     return acc;
-}
-
-// Bitonic sort of up to 512 keys held one per thread (block of 512), in
-// descending order; the stages that pair threads of the same warp use
-// shuffles, the rest go through `buf`.
-__device__ unsigned long long block_sort512_desc(unsigned long long key, unsigned long long *buf) {
-    const int tid = threadIdx.x;
-    for (int k = 2; k <= kThreads; k <<= 1) {
-        for (int jj = k >> 1; jj > 0; jj >>= 1) {
-            unsigned long long other;
-            if (jj >= 32) {
-                buf[tid] = key;
-                __syncthreads();
-                other = buf[tid ^ jj];
-                __syncthreads();
-            } else {
-                other = __shfl_xor_sync(0xffffffffu, key, jj);
-            }
-            const bool desc = (tid & k) == 0;
-            const bool lower = (tid & jj) == 0;
-            const unsigned long long mx = key > other ? key : other;
-            const unsigned long long mn = key > other ? other : key;
-            key = (desc == lower) ? mx : mn;
-        }
-    }
-    return key;
 }
 
 // Verify rows are ordered per sequence as K+1 target rows then K draft rows;
@@ -645,22 +649,37 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     {
         float mx = -INFINITY, mn = INFINITY;
         int arg = INT_MAX, bad = 0;
-        // batches of kBatch loads are issued before any use or store, so the
-        // L2 round trips overlap
+        // an aligned slice comes in with one bulk copy; otherwise batches of
+        // kBatch loads are issued before any use or store, so the L2 round
+        // trips overlap
+        const int n = v1 - v0;
+        const bool bulk = cached && n > 0 && (n & 3) == 0 && aligned16(L + v0);
+        if (bulk) {
+            if (tid == 0) {
+                mbar_init(&s.bar);
+                mbar_expect(&s.bar, (unsigned)n * 4u);
+                bulk_load(cache, L + v0, (unsigned)n * 4u, &s.bar);
+            }
+            __syncthreads();  // the barrier is initialised before anyone polls it
+            if (!mbar_wait(&s.bar, 0)) {
+                bad = 2;                 // the row is reported as timed out
+                mbar_wait(&s.bar, 0);    // a second bound for the copy in flight
+            }
+        }
         for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
             float lv[kBatch];
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
                 const int j = j0 + q * kThreads;
-                lv[q] = j < v1 ? __ldg(L + j) : 0.0f;
+                lv[q] = j < v1 ? (bulk ? cache[j - v0] : __ldg(L + j)) : 0.0f;
             }
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
                 const int j = j0 + q * kThreads;
                 if (j < v1) {
                     const float l = lv[q];
-                    if (cached) cache[j - v0] = l;
-                    if (!isfinite(l)) bad = 1;
+                    if (cached && !bulk) cache[j - v0] = l;
+                    if (!isfinite(l)) bad |= 1;
                     if (l > mx) { mx = l; arg = j; }
                     mn = fminf(mn, l);
                 }
@@ -699,7 +718,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     st.m = m;
     st.lmin = s.g_min;
     st.argmax = s.g_arg;
-    st.status = bad ? MTPV_ROW_NONFINITE : MTPV_ROW_OK;
+    st.status = (s.g_bad & 2) ? MTPV_ROW_TIMEOUT : bad ? MTPV_ROW_NONFINITE : MTPV_ROW_OK;
     st.Z = 1.0;
     st.Zk = 1.0;
     st.lstar = -INFINITY;
@@ -847,16 +866,46 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
             if (bstar < 0 || total == 0u) {
                 st.Zk = st.Z;  // nothing to cut (top_p within rounding of 1): keep all
             } else if (total <= (unsigned)kCandCap) {
-                if (rank == 0) {
+                if (rank == 0 && (int)total <= kThreads) {
+                    // one candidate per thread: its rank among the others (the
+                    // keys are distinct, they carry the token index) places it
+                    // and its exp in descending order; a block scan of the
+                    // sorted exps gives every candidate its preceding mass
+                    const int n = (int)total;
+                    const unsigned long long key = tid < n ? rg.cand[tid] : 0ull;
+                    int r = 0;
+                    if (tid < n)
+                        for (int j = 0; j < n; ++j) r += rg.cand[j] > key ? 1 : 0;
+                    const double e = tid < n ? e_of(key_logit(key), md, invT, s.exp_tab) : 0.0;
+                    __syncthreads();
+                    if (tid < n) {
+                        rg.cand[r] = key;
+                        rg.cand_e[r] = e;
+                    }
+                    if (tid == 0) s.first_fail = INT_MAX;
+                    __syncthreads();
+                    double excl;
+                    const double incl = block_scan_d(tid < n ? rg.cand_e[tid] : 0.0, s, &excl);
+                    if (tid < n && __dadd_rn(A, excl) >= thr) atomicMin(&s.first_fail, tid);
+                    __syncthreads();
+                    int cut = (s.first_fail == INT_MAX) ? n - 1 : s.first_fail - 1;
+                    if (cut < 0) cut = 0;  // A < thr by construction: the first is kept
+                    if (tid == cut) {
+                        s.cut_Zk = __dadd_rn(A, incl);
+                        s.cut_idx = key_index(rg.cand[cut]);
+                        s.cut_l = key_logit(rg.cand[cut]);
+                    }
+                    __syncthreads();
+                    if (wid == 0 && lane < C) {  // the cut, into every CTA of the cluster
+                        *cluster.map_shared_rank(&s.cut_Zk, lane) = s.cut_Zk;
+                        *cluster.map_shared_rank(&s.cut_idx, lane) = s.cut_idx;
+                        *cluster.map_shared_rank(&s.cut_l, lane) = s.cut_l;
+                    }
+                } else if (rank == 0) {
+                    // more candidates than threads: shared-memory bitonic sort
                     const int n = min((int)s.cand_count, kCandCap);
                     int n2 = 1;
                     while (n2 < n) n2 <<= 1;
-                    if (n2 <= kThreads) {
-                        unsigned long long key = tid < n ? rg.cand[tid] : 0ull;
-                        key = block_sort512_desc(key, reinterpret_cast<unsigned long long *>(rg.hist_mass));
-                        rg.cand[tid] = key;
-                        n2 = 1;  // sorted: skip the shared-memory network below
-                    }
                     for (int i = n + tid; i < n2; i += kThreads) rg.cand[i] = 0ull;
                     __syncthreads();
                     for (int k = 2; k <= n2; k <<= 1) {  // bitonic sort, descending
@@ -1075,7 +1124,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
     if (residual) {
         const int d = p.drafts[(size_t)b * K + i];
         if (d < 0 || d >= V) status = MTPV_ROW_BAD_DRAFT;
-        else if (st_d.status != MTPV_ROW_OK) status = MTPV_ROW_NONFINITE;
+        else if (st_d.status != MTPV_ROW_OK && status == MTPV_ROW_OK) status = st_d.status;
         if (status == MTPV_ROW_OK && rank == 0 && tid == 0) {
             double pt, qd;  // p'_i(d_i), q'_i(d_i)
             if (Et && T > 0.0) {
