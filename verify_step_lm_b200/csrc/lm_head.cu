@@ -711,6 +711,9 @@ __global__ void __launch_bounds__(kMixThreads, 1) lm_heads_mixed_kernel(
     extern __shared__ uint4 smem_mix[];
     __shared__ unsigned int row_amax[8];
     __shared__ float row_unscale[8];
+    // a dependent launch (the sampler) may be scheduled onto SMs as this
+    // grid's CTAs retire; it waits for the whole grid before reading y
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     const int Gt = Kd >> 6;
     const int rowc = Gt * 8 + 1;
     uint16_t *xst = reinterpret_cast<uint16_t *>(smem_mix);                   // [Mt][Kd + 32] bf16
