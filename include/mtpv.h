@@ -83,6 +83,21 @@ MTPV_API int mtpv_version(void);
 MTPV_API const char *mtpv_status_string(mtpv_status st);
 
 /* ------------------------------------------------------------------------
+ * mtpv_set_wait_polls -- bound of the sampler's device-side waits.
+ *
+ * The sampler kernels bring slices of logits and weights into shared memory
+ * with bulk copies and wait on an mbarrier for them.  Every such wait polls
+ * at most `polls` times (process-wide, taken at each launch); when the bound
+ * runs out the sequence (or sampled row) is reported as MTPV_ROW_TIMEOUT
+ * with out_accepted = -1 and tokens -1, and the kernel waits once more, with
+ * the default bound, for the copy it issued before it reads on or exits.
+ * polls < 0 restores the default (2^20 polls); 0 makes every first wait give
+ * up at once, which exercises the timeout path deterministically (tests).
+ * Not synchronised with launches in flight on other host threads.
+ * ---------------------------------------------------------------------- */
+MTPV_API void mtpv_set_wait_polls(int polls);
+
+/* ------------------------------------------------------------------------
  * mtpv_lm_head_smallm -- small-M weight-streaming projection.
  *
  * Passage: hazakura.dev MTPLX notes, Layer 0 (a matmul specialised for M=3..6

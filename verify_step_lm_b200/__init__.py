@@ -47,6 +47,7 @@ def load() -> ctypes.CDLL:
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
         "mtpv_version": ([], I),
+        "mtpv_set_wait_polls": ([I], None),
         "mtpv_status_string": ([I], ctypes.c_char_p),
         "mtpv_lm_head_workspace_bytes": ([I, I, I, I], Z),
         "mtpv_lm_head_smallm": ([P, I, I, I, P, P, I, P, P, Z, P], I),
@@ -96,6 +97,11 @@ def _check(fn: str, st: int):
 
 def version() -> int:
     return load().mtpv_version()
+
+
+def set_wait_polls(polls: int) -> None:
+    """Bound of the sampler's device-side waits (polls; < 0: the default)."""
+    load().mtpv_set_wait_polls(int(polls))
 
 
 def status_string(st: int) -> str:

@@ -152,6 +152,8 @@ extern "C" {
 
 int mtpv_version(void) { return 100; }
 
+void mtpv_set_wait_polls(int polls) { mtpv::set_wait_polls(polls); }
+
 const char *mtpv_status_string(mtpv_status st) {
     switch (st) {
         case MTPV_OK: return "ok";

@@ -47,6 +47,7 @@
 #include <limits.h>
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -253,8 +254,8 @@ __device__ __forceinline__ void bulk_load(void *dst, const void *src, unsigned b
         "l"(src), "r"(bytes), "r"(smem_u32(bar))
         : "memory");
 }
-__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, unsigned phase) {
-    for (int i = 0; i < kWaitLimit; ++i) {
+__device__ __forceinline__ bool mbar_wait(unsigned long long *bar, unsigned phase, int limit) {
+    for (int i = 0; i < limit; ++i) {
         unsigned done;
         asm volatile(
             "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
@@ -475,7 +476,8 @@ __device__ __forceinline__ void draw_weights_batch(const DrawSrc &d, int v1, int
 // every thread, warp and CTA equals the prefix the next level starts from.
 // ---------------------------------------------------------------------------
 __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double *wbuf, DrawSrc src,
-                             bool allow_fallback, double invT, float u, int v0, int v1, int *x_out) {
+                             bool allow_fallback, double invT, float u, int v0, int v1, int *x_out,
+                             int wait_polls) {
     const int C = (int)cluster.num_blocks();
     const int rank = (int)cluster.block_rank();
     const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
@@ -499,8 +501,8 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
             if (src.kind == 1) bulk_load(bd, src.Ed + v0, bytes, &s.bar);
         }
         __syncthreads();  // the barrier is initialised before anyone polls it
-        landed = mbar_wait(&s.bar, 0);
-        if (!landed) mbar_wait(&s.bar, 0);  // give the copies in flight a second bound
+        landed = mbar_wait(&s.bar, 0, wait_polls);
+        if (!landed) mbar_wait(&s.bar, 0, kWaitLimit);  // give the copies in flight a second bound
         if (src.kind == 1)
             for (int i = tid; i < n; i += kThreads) bd[i] = draw_combine(src, bt[i], bd[i]);
         __syncthreads();
@@ -661,9 +663,9 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 bulk_load(cache, L + v0, (unsigned)n * 4u, &s.bar);
             }
             __syncthreads();  // the barrier is initialised before anyone polls it
-            if (!mbar_wait(&s.bar, 0)) {
-                bad = 2;                 // the row is reported as timed out
-                mbar_wait(&s.bar, 0);    // a second bound for the copy in flight
+            if (!mbar_wait(&s.bar, 0, p.wait_polls)) {
+                bad = 2;                             // the row is reported as timed out
+                mbar_wait(&s.bar, 0, kWaitLimit);    // a second bound for the copy in flight
             }
         }
         for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
@@ -1157,7 +1159,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
         src.rho = residual ? st_t.Zk / st_d.Zk : 1.0;
         src.kind = residual ? 1 : 0;
         const float u = p.verify ? p.u_samp[(size_t)b * (K + 1) + i] : p.u_samp[c];
-        cluster_draw(cluster, s, wbuf, src, residual, invT, u, v0, v1, x_dst);
+        cluster_draw(cluster, s, wbuf, src, residual, invT, u, v0, v1, x_dst, p.wait_polls);
     }
     if (rank == 0 && tid == 0 && !p.verify && p.row_status) p.row_status[c] = status;
     cluster.sync();  // verify: res_x and res_acc are in CTA 0; no CTA exits while a peer reads it
@@ -1276,7 +1278,14 @@ cudaError_t launch_clusters(Kern kernel, int C, int clusters, size_t smem, const
 
 }  // namespace
 
-cudaError_t launch_sampler(const SamplerParams &p, int rows, cudaStream_t stream) {
+static std::atomic<int> g_wait_polls{-1};
+
+void set_wait_polls(int polls) { g_wait_polls.store(polls); }
+
+cudaError_t launch_sampler(const SamplerParams &params, int rows, cudaStream_t stream) {
+    SamplerParams p = params;
+    const int polls = g_wait_polls.load();
+    p.wait_polls = polls < 0 ? kWaitLimit : polls;
     const int C1 = cluster_size_for(0, sampler_stats_kernel, kStatsSmemBytes);
     cudaError_t e = launch_clusters(sampler_stats_kernel, C1, rows, kStatsSmemBytes, p, stream);
     if (e != cudaSuccess) return e;

@@ -49,7 +49,12 @@ struct SamplerParams {
     RowSlot *slots;       // [rows]
     unsigned int *counters;  // verify: [B]; zeroed by the statistics kernel
     double *ecache;       // [rows][V]: exp((l_j - m)/T) of kept tokens, 0 elsewhere (T > 0), or null
+    int wait_polls;       // polls of a bounded device-side wait before it gives up (set by launch_sampler)
 };
+
+// Process-wide bound of the sampler's device-side waits, in polls (< 0: the
+// default); see mtpv_set_wait_polls.
+void set_wait_polls(int polls);
 
 // Launches the statistics kernel over `rows` logits rows, then the draw
 // kernel (one cluster per draft position in verify mode, per row otherwise).
