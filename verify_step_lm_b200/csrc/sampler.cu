@@ -867,6 +867,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
             }
             if (bstar < 0 || total == 0u) {
                 st.Zk = st.Z;  // nothing to cut (top_p within rounding of 1): keep all
+                if (bstar >= 0) cluster.sync();  // every CTA has read CTA 0's count
             } else if (total <= (unsigned)kCandCap) {
                 if (rank == 0 && (int)total <= kThreads) {
                     // one candidate per thread: its rank among the others (the
@@ -1075,7 +1076,9 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
             }
         }
     }
-    cluster.sync();  // no CTA exits while a peer may still read its shared memory
+    // No closing cluster barrier: every access to a peer's shared memory above
+    // is followed by a cluster barrier that the peer also passes, so no CTA can
+    // leave while a peer still reads or writes its shared memory.
 }
 
 // ---------------------------------------------------------------------------
