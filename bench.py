@@ -220,6 +220,33 @@ def run_reference(args, c, rank):
     print(json.dumps(line), flush=True)
 
 
+class Replicas:
+    """Rank bookkeeping of an N-replica run: every rank runs the whole step on
+    its own batch (the verify step does not shard), ranks meet at barriers
+    around the timed region, the time is the max over ranks, and the
+    whole-job value counts every rank's steps.  Works on any process group
+    (NCCL with device tensors on the GPU machine, gloo with CPU tensors in the
+    tests); with world == 1 nothing is exchanged."""
+
+    def __init__(self, world: int, rank: int, device):
+        self.world, self.rank, self.device = world, rank, device
+
+    def barrier(self):
+        if self.world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(self, x: float) -> float:
+        if self.world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    def job_value(self, ms_per_step: float) -> float:
+        """Steps per second of the whole job: world steps per max-over-ranks step time."""
+        return self.world * 1e3 / ms_per_step
+
+
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
@@ -272,16 +299,8 @@ def run_gpu(args, c, rank, world, local_rank):
         mtpv.verify_step(W, Wq, S, ht[j], hd[j], dr[j], ua[j], us[j], B, K, T, top_p, ot, oa, rs,
                          tl, dl, ws)
 
-    def barrier():
-        if world > 1:
-            torch.distributed.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+    reps = Replicas(world, rank, dev)
+    barrier, max_over_ranks = reps.barrier, reps.max_over_ranks
 
     # --- warm-up
     for i in range(args.warmup):
@@ -340,7 +359,7 @@ def run_gpu(args, c, rank, world, local_rank):
     k_int4 = statistics.mean(e[1].elapsed_time(e[2]) for e in sev)
 
     step_ms = max_over_ranks(step_ms)
-    value = world * 1e3 / step_ms
+    value = reps.job_value(step_ms)
 
     # --- the same steps replayed from CUDA graphs (one captured graph per
     # pool entry; the library makes no allocation or host sync inside a step)
@@ -365,7 +384,7 @@ def run_gpu(args, c, rank, world, local_rank):
         torch.cuda.synchronize()
         barrier()
         graph_ms = max_over_ranks(g0.elapsed_time(g1) / args.steps)
-        graph = {"value": world * 1e3 / graph_ms, "unit": "steps/s", "ms_per_step": graph_ms,
+        graph = {"value": reps.job_value(graph_ms), "unit": "steps/s", "ms_per_step": graph_ms,
                  "graphs": POOL, "nodes_per_step": f"{3 if fused else 4} kernels"}
         del graphs
 
@@ -402,7 +421,7 @@ def run_gpu(args, c, rank, world, local_rank):
         e2e_ms = max_over_ranks(f0.elapsed_time(f1) / args.steps)
         h2d = (B * (K + 1) * h + B * K * h) * 2 + B * K * 4 + B * K * 4 + B * (K + 1) * 4
         d2h = B * (K + 1) * 4 + B * 4 + B * 4
-        e2e = {"value": world * 1e3 / e2e_ms, "unit": "steps/s", "h2d_bytes_per_step": h2d,
+        e2e = {"value": reps.job_value(e2e_ms), "unit": "steps/s", "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "api": "mtpv_verify_step_host (pinned host inputs/outputs)"}
 
