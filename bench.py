@@ -446,7 +446,7 @@ def run_gpu(args, c, rank, world, local_rank):
                                                  "lm_heads_mixed_qwen27b.md") if fused and
                                 args.config == "qwen27b" else None,
                      "kernel": "lm_heads_mixed_kernel (both heads, one launch)" if fused
-                               else "lm_head_bf16_xf32_kernel + lm_head_int4_f16_kernel",
+                               else "lm_head_bf16_mma_kernel + lm_head_int4_f16_kernel",
                      "algorithmic_bytes_per_launch": heads_bytes, "peak_source": peak_kind},
         "step_roofline": {"achieved": sb["total"] / (step_ms * 1e-3) / 1e9, "peak": peak,
                           "unit": "GB/s", "frac": sb["total"] / (step_ms * 1e-3) / 1e9 / peak,

@@ -14,11 +14,16 @@
 //
 // Design for sm_100a: two kernels, each a grid of thread-block clusters of C
 // CTAs (16, or 8 when a 16-CTA cluster cannot be resident); every cross-CTA
-// step goes through distributed shared memory and hardware cluster barriers
-// (no global flags, no spin loops).
+// step goes through distributed shared memory and hardware cluster barriers:
+// a CTA writes its share into a slot of every CTA of the cluster before the
+// barrier and reads the slots locally after it (no global flags).  Slices
+// move between global and shared memory by bulk copies where aligned; their
+// mbarrier waits are the only polling loops, each with a bound.  Both kernels
+// are programmatic dependents of the work before them on the stream.
 // Statistics kernel, one cluster per logits row; each CTA owns a contiguous
 // slice of the vocabulary and keeps it in shared memory:
-//   P1  the slice is read once (coalesced); max / min / argmax / finiteness
+//   P1  the slice is read once (one bulk copy when aligned, else coalesced
+//       loads); max / min / argmax / finiteness
 //   P2  e_j = exp((l_j - m)/T) in fp64 for every token: Z and a 2048-bin mass
 //       histogram on (m - l_j) over the row's own range
 //   P3  the bin where the descending cumulative mass reaches top_p * Z; its
