@@ -251,12 +251,16 @@ MTPV_API mtpv_status mtpv_int4_gate_up(const void *x, int M, int Kd, int F, cons
  *   temperature    >= 0 and finite; top_p in (0, 1] (values above 1 mean 1).
  *   out_tokens     device int32 [B, K+1];  out_accepted device int32 [B]
  *   row_status     device int32 [B] or NULL; MTPV_ROW_* per sequence.  A
- *                  sequence with a data error gets out_accepted = -1 and
- *                  out_tokens all -1.
+ *                  sequence with a data error, or whose device-side wait ran
+ *                  out of its bound (MTPV_ROW_TIMEOUT, mtpv_set_wait_polls),
+ *                  gets out_accepted = -1 and out_tokens all -1.
  *   ws, ws_bytes   workspace of at least mtpv_verify_workspace_bytes(B, K, V)
  *                  bytes, 256-byte aligned.  It need not be initialised: the
- *                  call clears what it needs on `stream` before the kernel.
+ *                  call's first kernel clears what it needs.
  * Arithmetic: exp, sums, ratios and CDFs in fp64 on fp32 logits.
+ * Launch: two kernels, each launched as a programmatic dependent of the work
+ * before it on `stream` (it may be scheduled while that work drains and
+ * waits for its completion before reading its results).
  * ---------------------------------------------------------------------- */
 MTPV_API size_t mtpv_verify_workspace_bytes(int B, int K, int V);
 MTPV_API mtpv_status mtpv_verify(const float *target_logits, const float *draft_logits,
@@ -289,7 +293,7 @@ MTPV_API mtpv_status mtpv_verify(const float *target_logits, const float *draft_
  *   (cudaGetSymbolAddress, which may load the library's GPU code); make that
  *   first call before any stream capture.
  *   Every call shares the one array and leaves its contents behind; each call
- *   clears the counters it needs on `stream` first.  Calls whose GPU work can
+ *   clears the counters it needs in its first kernel.  Calls whose GPU work can
  *   overlap in time (different streams without ordering) race on the array
  *   and give wrong results: order them on one stream.
  *   It calls no cudaMalloc, cudaFree or allocating library routine.
@@ -308,8 +312,10 @@ MTPV_API mtpv_status mtpv_verify_noalloc(const float *target_logits, const float
  * "Draft"), used to draw draft tokens from q'.
  *
  *   logits     device fp32 [R, V];  u device fp32 [R] in [0, 1)
- *   out        device int32 [R] (-1 for a row with a non-finite logit)
- *   row_status device int32 [R] or NULL (MTPV_ROW_OK / MTPV_ROW_NONFINITE)
+ *   out        device int32 [R] (-1 for a row with a non-finite logit or a
+ *              timed-out device wait)
+ *   row_status device int32 [R] or NULL (MTPV_ROW_OK / MTPV_ROW_NONFINITE /
+ *              MTPV_ROW_TIMEOUT)
  *   1 <= R <= 65535, 1 <= V <= 2^24; ws as returned by the query.
  * ---------------------------------------------------------------------- */
 MTPV_API size_t mtpv_sample_workspace_bytes(int R, int V);
