@@ -290,8 +290,13 @@ MTPV_API mtpv_status mtpv_verify(const float *target_logits, const float *draft_
  *   MTPV_ERR_UNSUPPORTED and launch nothing.  Other argument errors return
  *   MTPV_ERR_INVALID_ARG as in mtpv_verify.
  *   First call on a device: it looks up the array's device address once
- *   (cudaGetSymbolAddress, which may load the library's GPU code); make that
- *   first call before any stream capture.
+ *   (cudaGetSymbolAddress, which may load the library's GPU code) and keeps
+ *   it for the life of the process; make that first call before any stream
+ *   capture, and do not call it again on a device after cudaDeviceReset (the
+ *   kept address would then be stale).
+ *   With no room for mtpv_verify's cached token weights, the draw recomputes
+ *   each weight from the logits (one more fp64 exp per token it reads); the
+ *   results are the same bits.
  *   Every call shares the one array and leaves its contents behind; each call
  *   clears the counters it needs in its first kernel.  Calls whose GPU work can
  *   overlap in time (different streams without ordering) race on the array

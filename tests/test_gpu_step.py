@@ -92,8 +92,9 @@ def test_host_io_step_equals_device_step():
 
 
 def test_qwen_class_step_full_size():
-    """hidden 5120, vocab 151936, K = 3: the benchmark's step, checked on
-    sampled logits against the oracle and for self-consistency."""
+    """hidden 5120, vocab 151936, K = 3: the benchmark's step; logits against
+    the oracle (all draft rows; every 53rd vocabulary row and the ragged tail
+    of the target rows), tokens against the oracle run on the step's own logits."""
     B, K, V, h = 1, 3, 151936, 5120
     W, Wq, S, Ht, Hd, u = make_inputs(B, K, V, h, 11, 0.02, device="cuda")
     # drafts: the oracle's draft distribution needs the draft logits; compute
@@ -104,10 +105,15 @@ def test_qwen_class_step_full_size():
     d = d.reshape(B, K)
     tl, dl, ot, oa, rs = run_step(W, Wq, S, Ht, Hd, d, u, B, K)
     assert_logits_close(dl.reshape(B * K, V).cpu().numpy(), dl_ref)
-    Wc = W[:2048].cpu()
-    tl_ref = oracle.lm_head_bf16(synth.bf16_bits(Ht.cpu()), synth.bf16_bits(Wc), threads=8)
-    assert_logits_close(tl.reshape(B * (K + 1), V)[:, :2048].cpu().numpy(), tl_ref)
+    rows = torch.as_tensor(np.unique(np.concatenate([np.arange(0, V, 53), np.arange(V - 40, V)]))).cuda()
+    tl_ref = oracle.lm_head_bf16(synth.bf16_bits(Ht.cpu()), synth.bf16_bits(W[rows].cpu()), threads=8)
+    assert_logits_close(tl.reshape(B * (K + 1), V)[:, rows].cpu().numpy(), tl_ref)
     n = int(oa.item())
     assert 0 <= n <= K and int(rs.item()) == 0
     toks = ot.cpu().numpy()[0]
     assert list(toks[:n]) == list(d[0, :n]) and toks[n] >= 0 and (toks[n + 1:] == -1).all()
+    # the step's tokens against the oracle run on the step's own logits
+    ref = oracle.verify(tl.cpu().numpy(), dl.cpu().numpy(), d, u["u_accept"], u["u_sample"], f32(T),
+                        f32(TOP_P))
+    assert ref["flags"][0] != 0 or (np.array_equal(toks, ref["tokens"][0]) and n == ref["accepted"][0])
+    assert ref["status"][0] == 0

@@ -3,16 +3,19 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "args.cuh"
 #include "common.cuh"
 #include "lm_head.cuh"
 #include "sampler.cuh"
 
 namespace {
 
+using mtpv::kMaxRows;
+using mtpv::kMaxV;
+using mtpv::sampling_params_ok;
+using mtpv::verify_shape_ok;
+
 constexpr size_t kAlign = 256;
-constexpr int kMaxK = 16;
-constexpr int kMaxV = 1 << 24;
-constexpr int kMaxRows = 65535;
 
 size_t up(size_t n) { return (n + kAlign - 1) / kAlign * kAlign; }
 
@@ -90,15 +93,6 @@ DraftWs draft_layout(int B, int V, int h) {
     l.samp = l.tok + up(sizeof(int32_t) * (size_t)B);
     l.total = l.samp + sample_ws_bytes(B, V);
     return l;
-}
-
-bool verify_shape_ok(int B, int K, int V) {
-    return B >= 1 && K >= 1 && K <= kMaxK && V >= 1 && V <= kMaxV &&
-           (long long)B * (2 * K + 1) <= kMaxRows;
-}
-
-bool sampling_params_ok(float T, float top_p) {
-    return isfinite(T) && T >= 0.0f && !isnan(top_p) && top_p > 0.0f;
 }
 
 bool lm_head_shape_ok(int M, int Kd, int N) {

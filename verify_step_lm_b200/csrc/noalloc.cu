@@ -5,6 +5,7 @@
 // and caveats are documented with the declaration in include/mtpv.h.
 #include <mutex>
 
+#include "args.cuh"
 #include "common.cuh"
 #include "sampler.cuh"
 
@@ -13,9 +14,6 @@ namespace {
 constexpr size_t kScratchBytes = 64 * 1024;  // per device, held until process exit
 constexpr size_t kAlign = 256;
 constexpr int kMaxDevices = 64;
-constexpr int kMaxK = 16;
-constexpr int kMaxV = 1 << 24;
-constexpr int kMaxRows = 65535;
 static_assert(sizeof(mtpv::RowSlot) == 40, "the documented limit counts 40 bytes per row");
 
 // The library's own scratch.  In host code this name is only a stand-in for
@@ -56,9 +54,7 @@ extern "C" mtpv_status mtpv_verify_noalloc(const float *target_logits, const flo
     if (!target_logits || !draft_logits || !draft_tokens || !u_accept || !u_sample || !out_tokens ||
         !out_accepted)
         return MTPV_ERR_INVALID_ARG;
-    if (B < 1 || K < 1 || K > kMaxK || V < 1 || V > kMaxV || (long long)B * (2 * K + 1) > kMaxRows)
-        return MTPV_ERR_INVALID_ARG;
-    if (!isfinite(temperature) || temperature < 0.0f || isnan(top_p) || !(top_p > 0.0f))
+    if (!mtpv::verify_shape_ok(B, K, V) || !mtpv::sampling_params_ok(temperature, top_p))
         return MTPV_ERR_INVALID_ARG;
     if (((uintptr_t)target_logits & 3) || ((uintptr_t)draft_logits & 3)) return MTPV_ERR_INVALID_ARG;
 
