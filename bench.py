@@ -1,7 +1,8 @@
 """Benchmark of the speculative-decoding verify step on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--sigma S]
                     [--impl {mtpv,reference}] [--no-cpu-baseline] [--no-e2e] [--no-graph]
+                    [--no-extra]
     python bench.py --proj     (int4 decoder-layer projections at small M)
 
 One step = the whole verify step of one batch: the K+1 target rows through
@@ -15,7 +16,12 @@ step streams them from HBM.
 Multi-GPU: the verify step does not shard; N ranks run N independent
 replicas (weak scaling) and the time is the max over ranks.
 
-Prints one JSON line (rank 0).
+Prints one JSON line (rank 0).  Besides the headline workload (hidden 5120,
+vocabulary 151936, K = 3), a one-GPU run adds three keys, each timed the
+same way on its own synthetic inputs: "sweep" (draft depth K in {1, 2, 3} x
+T in {0.6, 0} x draft noise sigma in {0.1, 0.3, 1.0}: step time spread and
+acceptance per cell), "large_vocab_b8" (8 sequences, vocabulary 248320) and
+"projections" (the int4 decoder-layer projections at M = 1..8).
 """
 from __future__ import annotations
 
@@ -47,6 +53,7 @@ CONFIGS = {
     "tiny": dict(B=1, K=3, V=4096, h=512, T=0.6, top_p=0.95, sigma=0.3, wstd=0.05),
 }
 POOL = 64
+SWEEP_K, SWEEP_T, SWEEP_SIGMA = (1, 2, 3), (0.6, 0.0), (0.1, 0.3, 1.0)
 METRIC = "verify steps/s (K=3, V=151936, h=5120) and achieved HBM GB/s vs roofline"
 
 
@@ -212,7 +219,7 @@ def run_reference(args, c, rank):
         "impl": "reference", "metric": METRIC, "value": v, "unit": "steps/s", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * elapsed / steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": workload_name(c), "parallelism": "replicas"},
+        "data": "synthetic", "config": config_dict(c, args.config, args.gpus),
         "cpu_baseline": {"value": v, "unit": "steps/s", "cores": cores, "kind": "oracle",
                          "sample": f"{steps} whole verify steps of the workload, fp64 C oracle"},
         "e2e": {"value": v, "unit": "steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -250,16 +257,23 @@ class Replicas:
 # ---------------------------------------------------------------------------
 # the GPU arm
 # ---------------------------------------------------------------------------
-def build_pool(c, dev, mtpv):
-    B, K, V, h = c["B"], c["K"], c["V"], c["h"]
-    W = synth.make_head(V, h, c["wstd"], seed=12345, device=dev)
+def make_heads(c, dev):
+    W = synth.make_head(c["V"], c["h"], c["wstd"], seed=12345, device=dev)
     Wq, S = synth.quantize_int4_g64(W)
+    return W, Wq, S
+
+
+def build_pool(c, dev, mtpv, heads, n=POOL, sigma=None):
+    """n pre-generated steps: hidden states (draft noise sigma), uniforms, and
+    drafts drawn by the library's own sampler from q' (the draft phase)."""
+    B, K, V, h = c["B"], c["K"], c["V"], c["h"]
+    W, Wq, S = heads
+    sigma = c["sigma"] if sigma is None else sigma
     ht, hd, dr, ua, us = [], [], [], [], []
     dl = torch.empty((B * K, V), dtype=torch.float32, device=dev)
-    for i in range(POOL):
-        Ht, Hd = synth.make_hidden(B, K, h, c["sigma"], seed=i, device=dev)
+    for i in range(n):
+        Ht, Hd = synth.make_hidden(B, K, h, sigma, seed=i, device=dev)
         u = synth.step_uniforms(i, 0, B, K)
-        # drafts: the draft phase's own sampling from q' (library kernels)
         mtpv.lm_head_smallm(Hd, Wq, S, mtpv.W_INT4_G64, dl)
         d = torch.empty((B * K,), dtype=torch.int32, device=dev)
         mtpv.sample(dl, c["T"], c["top_p"], torch.as_tensor(u["u_draft"].reshape(-1)).to(dev), d)
@@ -269,7 +283,157 @@ def build_pool(c, dev, mtpv):
         ua.append(torch.as_tensor(u["u_accept"]).to(dev))
         us.append(torch.as_tensor(u["u_sample"]).to(dev))
     torch.cuda.synchronize()
-    return W, Wq, S, ht, hd, dr, ua, us
+    return ht, hd, dr, ua, us
+
+
+def spread(ms):
+    """median / p10 / p90 of per-step times (ms) in microseconds."""
+    a = np.asarray(ms, dtype=np.float64) * 1e3
+    return {"median": float(np.median(a)), "p10": float(np.percentile(a, 10)),
+            "p90": float(np.percentile(a, 90)), "n": int(a.size)}
+
+
+class StepRunner:
+    """One workload on one device: heads, a pool of steps, output buffers and
+    the workspace; step(i) runs pool entry i % n through mtpv_verify_step."""
+
+    def __init__(self, c, dev, mtpv, heads=None, sigma=None, n=POOL):
+        self.c, self.dev, self.mtpv = c, dev, mtpv
+        B, K, V, h = c["B"], c["K"], c["V"], c["h"]
+        self.heads = heads if heads is not None else make_heads(c, dev)
+        self.pool = build_pool(c, dev, mtpv, self.heads, n=n, sigma=sigma)
+        self.n = n
+        self.tl = torch.empty((B, K + 1, V), dtype=torch.float32, device=dev)
+        self.dl = torch.empty((B, K, V), dtype=torch.float32, device=dev)
+        self.ot = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
+        self.oa = torch.empty((B,), dtype=torch.int32, device=dev)
+        self.rs = torch.empty((B,), dtype=torch.int32, device=dev)
+        self.ws = mtpv.workspace(mtpv.verify_step_workspace_bytes(B, K, V, h), dev)
+        self.stream = torch.cuda.current_stream(dev)
+
+    def step(self, i):
+        c, (W, Wq, S) = self.c, self.heads
+        ht, hd, dr, ua, us = self.pool
+        j = i % self.n
+        self.mtpv.verify_step(W, Wq, S, ht[j], hd[j], dr[j], ua[j], us[j], c["B"], c["K"], c["T"],
+                              c["top_p"], self.ot, self.oa, self.rs, self.tl, self.dl, self.ws)
+
+    def timed(self, steps, barrier=lambda: None):
+        """(mean ms per step over the whole region, per-step ms list): events
+        on the launching stream after every step."""
+        ev = [torch.cuda.Event(enable_timing=True) for _ in range(steps + 1)]
+        barrier()
+        torch.cuda.synchronize()
+        ev[0].record(self.stream)
+        for i in range(steps):
+            self.step(i)
+            ev[i + 1].record(self.stream)
+        torch.cuda.synchronize()
+        barrier()
+        per = [ev[i].elapsed_time(ev[i + 1]) for i in range(steps)]
+        return ev[0].elapsed_time(ev[steps]) / steps, per
+
+    def acceptance(self):
+        """Accepted drafts over every pool step (untimed): rate = E[n] / K."""
+        acc = []
+        for j in range(self.n):
+            self.step(j)
+            acc.append(self.oa.clone())
+        torch.cuda.synchronize()
+        a = torch.cat(acc).double()
+        K = self.c["K"]
+        return {"rate": float(a.mean()) / K, "tokens_per_step": float(a.mean()) + 1.0,
+                "all_accepted": float((a == K).double().mean()), "steps": self.n,
+                "sequences": int(a.numel())}
+
+    def breakdown(self, steps, barrier=lambda: None):
+        """Mean ms of the heads launch and of the sampler, issued separately
+        with events between them, for `steps` steps."""
+        c, (W, Wq, S), mtpv = self.c, self.heads, self.mtpv
+        B, K, V = c["B"], c["K"], c["V"]
+        ht, hd, dr, ua, us = self.pool
+        pws = mtpv.workspace(mtpv.load().mtpv_lm_head_pair_workspace_bytes(B * (K + 1), B * K, c["h"], V),
+                             self.dev)
+        vws = mtpv.workspace(mtpv.verify_workspace_bytes(B, K, V), self.dev)
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+        barrier()
+        torch.cuda.synchronize()
+        for i in range(steps):
+            j = i % self.n
+            evs[i][0].record(self.stream)
+            mtpv.lm_head_pair(ht[j], W, self.tl.view(B * (K + 1), V), hd[j], Wq, S, self.dl.view(B * K, V),
+                              ws=pws)
+            evs[i][1].record(self.stream)
+            mtpv.verify(self.tl, self.dl, dr[j], ua[j], us[j], c["T"], c["top_p"], self.ot, self.oa, self.rs,
+                        ws=vws)
+            evs[i][2].record(self.stream)
+        torch.cuda.synchronize()
+        barrier()
+        heads = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+        samp = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+        return heads, samp
+
+
+def fused_heads(c):
+    """Whether the step runs both heads in one launch (the two-head kernel)."""
+    B, K, h = c["B"], c["K"], c["h"]
+    return B * (K + 1) <= 8 and B * K <= 8 and h % 512 == 0 and \
+        (2 * B * (K + 1) * (h + 32) + (B * K + 1) * (h // 8 + 1) * 16 + h // 2 + 3 * 13056) <= 227 * 1024 - 256
+
+
+def config_dict(c, name, world):
+    return {"workload": workload_name(c), "global_batch": c["B"] * world, "seq_len": c["K"] + 1,
+            "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+            "l2": f"inputs larger than L2: {step_bytes(c)['w_bf16'] + step_bytes(c)['w_int4']:.3g} B of "
+                  "head weights streamed per step",
+            "config_name": name, "draft_noise_sigma": c["sigma"]}
+
+
+def run_sweep(dev, mtpv, steps, warmup):
+    """The draft-depth sweep at the Qwen-class heads: K in {1, 2, 3}, T in
+    {0.6, 0 (greedy)}, draft noise sigma in {0.1, 0.3, 1.0}; per cell the
+    step time (mean, median, p10, p90) and the acceptance over 64 steps."""
+    base = CONFIGS["qwen27b"]
+    heads = make_heads(base, dev)
+    cells = []
+    for K in SWEEP_K:
+        for T in SWEEP_T:
+            for sigma in SWEEP_SIGMA:
+                c = dict(base, K=K, T=T, sigma=sigma)
+                r = StepRunner(c, dev, mtpv, heads=heads)
+                for i in range(warmup):
+                    r.step(i)
+                ms, per = r.timed(steps)
+                acc = r.acceptance()
+                cells.append({"K": K, "T": T, "sigma": sigma, "steps_per_s": 1e3 / ms, "ms_per_step": ms,
+                              "step_us": spread(per), "acceptance": acc,
+                              "tokens_per_s": (1e3 / ms) * acc["tokens_per_step"]})
+                del r
+    return {"workload": "hidden 5120, vocab 151936, B=1, top_p=0.95, head W ~ N(0, 0.02^2)",
+            "steps_per_cell": steps, "cells": cells}
+
+
+def run_extra_config(name, dev, mtpv, steps, warmup, peak):
+    """Steps/s, per-step spread, kernel breakdown and heads roofline of one
+    more workload (its own heads)."""
+    c = CONFIGS[name]
+    r = StepRunner(c, dev, mtpv)
+    for i in range(warmup):
+        r.step(i)
+    ms, per = r.timed(steps)
+    heads_ms, samp_ms = r.breakdown(steps)
+    sb = step_bytes(c)
+    hb = sb["bf16_launch"] + sb["int4_launch"]
+    out = {"config": config_dict(c, name, 1), "steps_per_s": 1e3 / ms, "ms_per_step": ms,
+           "step_us": spread(per), "kernels_ms": {"lm_heads": heads_ms, "sampler": samp_ms},
+           "heads_roofline": {"achieved": hb / (heads_ms * 1e-3) / 1e9, "peak": peak, "unit": "GB/s",
+                              "frac": hb / (heads_ms * 1e-3) / 1e9 / peak, "algorithmic_bytes": hb},
+           "step_roofline": {"achieved": sb["total"] / (ms * 1e-3) / 1e9, "peak": peak,
+                             "frac": sb["total"] / (ms * 1e-3) / 1e9 / peak,
+                             "algorithmic_bytes_per_step": sb["total"]},
+           "acceptance": r.acceptance()}
+    del r
+    return out
 
 
 def run_gpu(args, c, rank, world, local_rank):
@@ -280,64 +444,27 @@ def run_gpu(args, c, rank, world, local_rank):
     mtpv.load()
     B, K, V, h = c["B"], c["K"], c["V"], c["h"]
     T, top_p = c["T"], c["top_p"]
-    W, Wq, S, ht, hd, dr, ua, us = build_pool(c, dev, mtpv)
-    tl = torch.empty((B, K + 1, V), dtype=torch.float32, device=dev)
-    dl = torch.empty((B, K, V), dtype=torch.float32, device=dev)
-    ot = torch.empty((B, K + 1), dtype=torch.int32, device=dev)
-    oa = torch.empty((B,), dtype=torch.int32, device=dev)
-    rs = torch.empty((B,), dtype=torch.int32, device=dev)
-    ws = mtpv.workspace(mtpv.verify_step_workspace_bytes(B, K, V, h), dev)
-    # the step runs both heads in one launch when the fused kernel takes the shapes
-    fused = B * (K + 1) <= 8 and B * K <= 8 and h % 512 == 0 and \
-        (2 * B * (K + 1) * (h + 32) + (B * K + 1) * (h // 8 + 1) * 16 + h // 2 + 3 * 13056) <= 227 * 1024 - 256
-    pws = mtpv.workspace(mtpv.load().mtpv_lm_head_pair_workspace_bytes(B * (K + 1), B * K, h, V), dev)
-    vws = mtpv.workspace(mtpv.verify_workspace_bytes(B, K, V), dev)
-    stream = torch.cuda.current_stream(dev)
-
-    def step(i):
-        j = i % POOL
-        mtpv.verify_step(W, Wq, S, ht[j], hd[j], dr[j], ua[j], us[j], B, K, T, top_p, ot, oa, rs,
-                         tl, dl, ws)
-
+    r = StepRunner(c, dev, mtpv)
+    W, Wq, S = r.heads
+    fused = fused_heads(c)
+    stream = r.stream
     reps = Replicas(world, rank, dev)
     barrier, max_over_ranks = reps.barrier, reps.max_over_ranks
 
     # --- warm-up
     for i in range(args.warmup):
-        step(i)
+        r.step(i)
     torch.cuda.synchronize()
 
-    # --- timed region: K whole steps through the product entry point
+    # --- timed region: K whole steps through the product entry point (an
+    # event after every step gives the per-step spread)
     with ClockSampler(dev.index) as clk:
-        barrier()
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for i in range(args.steps):
-            step(i)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        barrier()
-        step_ms = e0.elapsed_time(e1) / args.steps
-
-        # --- per-kernel breakdown: the launches the step makes (both heads,
-        # then the sampler's two kernels) with events between them, on the
-        # launching stream, for the same count of steps
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-        barrier()
-        torch.cuda.synchronize()
-        for i in range(args.steps):
-            j = i % POOL
-            ev = evs[i]
-            ev[0].record(stream)
-            mtpv.lm_head_pair(ht[j], W, tl.view(B * (K + 1), V), hd[j], Wq, S, dl.view(B * K, V), ws=pws)
-            ev[1].record(stream)
-            mtpv.verify(tl, dl, dr[j], ua[j], us[j], T, top_p, ot, oa, rs, ws=vws)
-            ev[2].record(stream)
-        torch.cuda.synchronize()
-        barrier()
-
-        # --- each head alone through its own kernel (reference for the fused launch)
+        step_ms, per_step = r.timed(args.steps, barrier)
+        # per-kernel breakdown: the launches the step makes (both heads, then
+        # the sampler's two kernels) with events between them
+        k_heads, k_samp = r.breakdown(args.steps, barrier)
+        # each head alone through its own kernel (reference for the fused launch)
+        ht, hd = r.pool[0], r.pool[1]
         nalone = min(args.steps, 500)
         sev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(nalone)]
         barrier()
@@ -345,16 +472,13 @@ def run_gpu(args, c, rank, world, local_rank):
         for i in range(nalone):
             j = i % POOL
             sev[i][0].record(stream)
-            mtpv.lm_head_smallm(ht[j], W, None, mtpv.W_BF16, tl.view(B * (K + 1), V))
+            mtpv.lm_head_smallm(ht[j], W, None, mtpv.W_BF16, r.tl.view(B * (K + 1), V))
             sev[i][1].record(stream)
-            mtpv.lm_head_smallm(hd[j], Wq, S, mtpv.W_INT4_G64, dl.view(B * K, V))
+            mtpv.lm_head_smallm(hd[j], Wq, S, mtpv.W_INT4_G64, r.dl.view(B * K, V))
             sev[i][2].record(stream)
         torch.cuda.synchronize()
         barrier()
     clocks = clk.summary()
-    k_heads = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
-    k_samp = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
-    comp_ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
     k_bf16 = statistics.mean(e[0].elapsed_time(e[1]) for e in sev)
     k_int4 = statistics.mean(e[1].elapsed_time(e[2]) for e in sev)
 
@@ -369,7 +493,7 @@ def run_gpu(args, c, rank, world, local_rank):
         for j in range(POOL):
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g):
-                step(j)
+                r.step(j)
             graphs.append(g)
         torch.cuda.synchronize()
         for i in range(args.warmup):
@@ -392,11 +516,7 @@ def run_gpu(args, c, rank, world, local_rank):
     e2e = None
     if not args.no_e2e:
         pin = lambda t: t.cpu().contiguous().pin_memory()
-        hht = [pin(x) for x in ht]
-        hhd = [pin(x) for x in hd]
-        hdr = [pin(x) for x in dr]
-        hua = [pin(x) for x in ua]
-        hus = [pin(x) for x in us]
+        hht, hhd, hdr, hua, hus = ([pin(x) for x in lst] for lst in r.pool)
         hot = torch.empty((B, K + 1), dtype=torch.int32).pin_memory()
         hoa = torch.empty((B,), dtype=torch.int32).pin_memory()
         hrs = torch.empty((B,), dtype=torch.int32).pin_memory()
@@ -425,6 +545,7 @@ def run_gpu(args, c, rank, world, local_rank):
                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
                "api": "mtpv_verify_step_host (pinned host inputs/outputs)"}
 
+    acceptance = r.acceptance()
     if rank != 0:
         return
     peak, peak_kind = measured_peaks()
@@ -436,15 +557,12 @@ def run_gpu(args, c, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16/int4 weights, fp32 accumulate, f64 sampler",
         "data": "synthetic",
-        "config": {"workload": workload_name(c), "global_batch": B * world, "seq_len": K + 1,
-                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                   "l2": "inputs larger than L2: 1.98 GB of head weights streamed per step",
-                   "config_name": args.config},
+        "config": config_dict(c, args.config, world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                      "frac": achieved / peak,
                      "traffic": recorded_traffic("verify_step_lm_b200/csrc/lm_head.cu",
                                                  "lm_heads_mixed_qwen27b.md") if fused and
-                                args.config == "qwen27b" else None,
+                                args.config == "qwen27b" and args.sigma is None else None,
                      "kernel": "lm_heads_mixed_kernel (both heads, one launch)" if fused
                                else "lm_head_bf16_mma_kernel + lm_head_int4_f16_kernel",
                      "algorithmic_bytes_per_launch": heads_bytes, "peak_source": peak_kind},
@@ -452,16 +570,26 @@ def run_gpu(args, c, rank, world, local_rank):
                           "unit": "GB/s", "frac": sb["total"] / (step_ms * 1e-3) / 1e9 / peak,
                           "frac_of_8tbs": sb["total"] / (step_ms * 1e-3) / 8e12,
                           "algorithmic_bytes_per_step": sb["total"]},
-        "kernels_ms": {"lm_heads": k_heads, "sampler": k_samp, "sum": comp_ms},
+        "step_us": spread(per_step),
+        "kernels_ms": {"lm_heads": k_heads, "sampler": k_samp},
         "heads_alone_ms": {"lm_head_bf16": k_bf16, "lm_head_int4": k_int4,
                            "bf16_gbs": sb["bf16_launch"] / (k_bf16 * 1e-3) / 1e9,
                            "int4_gbs": sb["int4_launch"] / (k_int4 * 1e-3) / 1e9},
-        "acceptance_last_step": oa.cpu().tolist(),
+        "acceptance": acceptance,
         "gpu_launches": (3 if fused else 4) * args.steps,
         "clocks": clocks,
         "e2e": e2e,
         "graph": graph,
     }
+    if not args.no_extra and world == 1:
+        del r
+        torch.cuda.empty_cache()
+        n = max(50, min(args.steps, 200))
+        line["sweep"] = run_sweep(dev, mtpv, n, max(3, min(args.warmup, 10)))
+        torch.cuda.empty_cache()
+        line["large_vocab_b8"] = run_extra_config("b8_v248k", dev, mtpv, n, max(3, min(args.warmup, 10)), peak)
+        torch.cuda.empty_cache()
+        line["projections"] = run_proj(args, quiet=True)
     if not args.no_cpu_baseline and world == 1:
         steps, elapsed, cores = oracle_steps(c, seconds=10.0, min_steps=2, max_steps=30,
                                              heads=(W.cpu(), Wq.cpu(), S.cpu()))
@@ -479,10 +607,11 @@ PROJ_SHAPES = [  # name, Kd, N (gate_up: N = 2F, output F)
     ("qkv", 5120, 7168), ("o", 5120, 5120), ("gate_up", 5120, 2 * 17408), ("down", 17408, 5120)]
 
 
-def run_proj(args):
+def run_proj(args, quiet=False):
     """Each projection of a 27B-class decoder layer at M in {1..6, 8}, weights
     rotated over enough copies (>= 4x the L2) that every call streams them
-    from HBM; CUDA-event time per call, plain launches and CUDA-graph replay."""
+    from HBM; CUDA-event time per call, plain launches and CUDA-graph replay.
+    Prints one JSON line, or (quiet) returns it."""
     import verify_step_lm_b200 as mtpv
 
     dev = torch.device("cuda", 0)
@@ -552,6 +681,10 @@ def run_proj(args):
                                    "W ~ N(0, 0.02^2) -> int4 g64, activations N(0,1) bf16",
                        "weight_copies": copies, "l2": "weights rotated over >= 4x L2"},
             "peak_gbs": peak, "peak_source": peak_kind, "by_m": out}
+    del layers
+    torch.cuda.empty_cache()
+    if quiet:
+        return line
     print(json.dumps(line), flush=True)
 
 
@@ -565,12 +698,18 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the depth sweep, the large-vocabulary batch and the projections")
+    ap.add_argument("--sigma", type=float, default=None,
+                    help="draft-noise sigma of the workload (sets the acceptance rate)")
     ap.add_argument("--proj", action="store_true",
                     help="time the int4 decoder-layer projections instead of the verify step")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
-    c = CONFIGS[args.config]
+    c = dict(CONFIGS[args.config])
+    if args.sigma is not None:
+        c["sigma"] = args.sigma
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))

@@ -8,14 +8,16 @@
 
 namespace mtpv {
 
-constexpr int kSMs = 148;  // B200: 2 dies x 74 SMs
-
 // Launch setup of `kernel` on the current device: opts it into `smem` bytes of
 // dynamic shared memory and returns how many of its CTAs of `threads` threads
-// fit on one SM.  Cached per (kernel, device, threads, smem): once a first
-// call has run, later launches of the same shape make no CUDA API call here,
-// which also keeps them capturable into a CUDA graph.
-cudaError_t kernel_setup(const void *kernel, int threads, size_t smem, int *ctas_per_sm);
+// fit on one SM, and (sms) the device's SM count (148 on a B200), which sizes
+// the persistent grids.  Cached per (kernel, device, threads, smem): once a
+// first call has run, later launches of the same shape make no CUDA API call
+// here, which also keeps them capturable into a CUDA graph.
+cudaError_t kernel_setup(const void *kernel, int threads, size_t smem, int *ctas_per_sm, int *sms);
+
+// SM count of the current device (cached per device); 0 if it cannot be read.
+int current_device_sms();
 
 // ---------------------------------------------------------------------------
 // global loads

@@ -750,12 +750,12 @@ static cudaError_t launch_bf16_mma(const uint16_t *x, int M, int Kd, int N, cons
                                    float *y, int ldy, cudaStream_t s) {
     auto k = lm_head_bf16_mma_kernel<NT, kBmmaU>;
     const size_t smem = bf16_mma_smem(M, Kd);
-    int occ = 0;
-    cudaError_t e = kernel_setup((const void *)k, kBmmaThreads, smem, &occ);
+    int occ = 0, sms = 0;
+    cudaError_t e = kernel_setup((const void *)k, kBmmaThreads, smem, &occ, &sms);
     if (e != cudaSuccess) return e;
     const int ntiles = (N + 15) / 16;
     const int need = (ntiles + kBmmaThreads / 32 - 1) / (kBmmaThreads / 32);
-    const int grid = std::min(need, kSMs * occ);
+    const int grid = std::min(need, sms * occ);
     k<<<grid, kBmmaThreads, smem, s>>>(x, M, Kd, N, W, y, ldy);
     return cudaGetLastError();
 }
@@ -782,12 +782,12 @@ static cudaError_t launch_int4_f16(const uint16_t *x, int M, int Kd, int N, cons
                                    const uint16_t *S, float *y, int ldy, cudaStream_t s) {
     auto k = lm_head_int4_f16_kernel<kF16Gps, kF16Nst, kF16Threads>;
     const size_t smem = int4_f16_smem(M, Kd);
-    int occ = 0;
-    cudaError_t e = kernel_setup((const void *)k, kF16Threads, smem, &occ);
+    int occ = 0, sms = 0;
+    cudaError_t e = kernel_setup((const void *)k, kF16Threads, smem, &occ, &sms);
     if (e != cudaSuccess) return e;
     const int nblk = (N + 15) / 16;
     const int need = (nblk + kF16Threads / 32 - 1) / (kF16Threads / 32);
-    const int grid = std::min(need, kSMs * occ);
+    const int grid = std::min(need, sms * occ);
     k<<<grid, kF16Threads, smem, s>>>(x, M, Kd, N, Wq, S, y, ldy);
     return cudaGetLastError();
 }
@@ -797,12 +797,12 @@ static cudaError_t launch_int4_direct(const uint16_t *x, int M, int Kd, int N, c
     constexpr int RB = 2, UI = 4;
     auto k = lm_head_int4_f16_direct_kernel<RB, UI>;
     const size_t smem = int4_direct_smem(M, Kd);
-    int occ = 0;
-    cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ);
+    int occ = 0, sms = 0;
+    cudaError_t e = kernel_setup((const void *)k, kGemvThreads, smem, &occ, &sms);
     if (e != cudaSuccess) return e;
     const int ntask = ((N + 15) / 16 + RB - 1) / RB;
     const int need = (ntask + kGemvWarps - 1) / kGemvWarps;
-    const int grid = std::min(need, kSMs * occ);
+    const int grid = std::min(need, sms * occ);
     k<<<grid, kGemvThreads, smem, s>>>(x, M, Kd, N, Wq, S, y, ldy);
     return cudaGetLastError();
 }
@@ -824,13 +824,13 @@ cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *y
     if (!lm_heads_pair_ok(Mt, Md, Kd, scales) || !work) return cudaErrorInvalidValue;
     auto k = lm_heads_mixed_kernel<kF16Gps, kF16Nst>;
     const size_t smem = heads_pair_smem(Mt, Md, Kd);
-    int occ = 0;
-    cudaError_t e = kernel_setup((const void *)k, kMixThreads, smem, &occ);
+    int occ = 0, sms = 0;
+    cudaError_t e = kernel_setup((const void *)k, kMixThreads, smem, &occ, &sms);
     if (e != cudaSuccess) return e;
     unsigned int *wk = static_cast<unsigned int *>(work);
     e = cudaMemsetAsync(wk, 0, sizeof(unsigned int), s);
     if (e != cudaSuccess) return e;
-    k<<<kSMs * occ, kMixThreads, smem, s>>>(
+    k<<<sms * occ, kMixThreads, smem, s>>>(
         static_cast<const uint16_t *>(xt), Mt, static_cast<const uint16_t *>(w), yt,
         static_cast<const uint16_t *>(xd), Md, static_cast<const uint8_t *>(wq),
         static_cast<const uint16_t *>(scales), yd, Kd, N, wk);
@@ -841,11 +841,13 @@ cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *y
 constexpr int kSplitRB = 2, kSplitUI = 4, kSplitRows = 8;  // rows per pass: one MMA n-tile
 
 // Slices of the reduction for a pass over N outputs: enough items to give
-// every warp of the GPU about two, at least kSplitUI groups per slice.
+// every warp of the GPU about two, at least kSplitUI groups per slice (the
+// current device's SM count; 148 if it cannot be read).
 static void splitk_plan(int Kd, int N, int *slices, int *gps) {
     const int Gt = Kd / 64;
     const int tasks = ((N + 15) / 16 + kSplitRB - 1) / kSplitRB;
-    int sl = (2 * kSMs * kGemvWarps + tasks - 1) / tasks;
+    const int nsm = current_device_sms() > 0 ? current_device_sms() : 148;
+    int sl = (2 * nsm * kGemvWarps + tasks - 1) / tasks;
     sl = std::max(1, std::min({sl, 16, std::max(1, Gt / kSplitUI)}));
     const int g = (Gt + sl - 1) / sl;
     *gps = g;
@@ -890,18 +892,18 @@ cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq
         int4_f16_stage_rows_kernel<<<mm, kGemvThreads, 0, s>>>(x16 + (size_t)m0 * Kd, mm, Kd, xb, xs, us);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
-        int occ = 0;
-        e = kernel_setup((const void *)k, kGemvThreads, 0, &occ);
+        int occ = 0, sms = 0;
+        e = kernel_setup((const void *)k, kGemvThreads, 0, &occ, &sms);
         if (e != cudaSuccess) return e;
         const int tasks = ((N + 15) / 16 + kSplitRB - 1) / kSplitRB;
         const int need = (tasks * slices + kGemvWarps - 1) / kGemvWarps;
-        k<<<std::min(need, kSMs * occ), kGemvThreads, 0, s>>>(
+        k<<<std::min(need, sms * occ), kGemvThreads, 0, s>>>(
             reinterpret_cast<const uint4 *>(xb), xs, us, mm, Kd, N, static_cast<const uint8_t *>(wq),
             static_cast<const uint16_t *>(scales), part, slices, gps);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         const int cols = silu_mul ? N / 2 : N;
-        const int blocks = std::min(kSMs * 4, (mm * cols + kGemvThreads - 1) / kGemvThreads);
+        const int blocks = std::min(sms * 4, (mm * cols + kGemvThreads - 1) / kGemvThreads);
         splitk_reduce_kernel<<<blocks, kGemvThreads, 0, s>>>(part, slices, mm, N, y + (size_t)m0 * ldy,
                                                             ldy, silu_mul ? 1 : 0);
         e = cudaGetLastError();
