@@ -101,21 +101,18 @@ struct SamplerSmem {
     // rank) before a cluster barrier, read locally after it
     float all_max[kMaxCluster], all_min[kMaxCluster];
     int all_arg[kMaxCluster], all_bad[kMaxCluster];
-    double all_Z[kMaxCluster], all_rt[kMaxCluster], all_part[kMaxCluster];
+    double all_Z[kMaxCluster], all_rt[kMaxCluster], all_part[kMaxCluster], all_M[kMaxCluster];
     double my_partial;
     // broadcast into every CTA of the cluster
     int bc_bin;
-    double bc_A;
+    double bc_A;  // radix select: the mass above the selected digit
     unsigned int cand_count;
     unsigned int local_n, local_base;
     // derived by every CTA for itself
-    float g_m, g_min;
-    int g_arg, g_bad;
-    double g_Z, draw_Pc, draw_total, cut_Zk;
+    double draw_total, cut_Zk;
     int wstar, x_found, first_fail, cut_idx;
     float cut_l;
-    int res_x, res_acc;  // draw kernel: the position's token and acceptance, in CTA 0
-    int res_timeout;     // draw kernel, CTA 0: a CTA of the cluster gave up waiting for a copy
+    int res_acc;  // draw kernel, CTA 0: the position's acceptance
     unsigned long long bar;  // mbarrier of the bulk copies
     double exp_tab[kExpTab];  // 2^(j/64), for exp_neg
 };
@@ -472,15 +469,24 @@ __device__ __forceinline__ void draw_weights_batch(const DrawSrc &d, int v1, int
 // ---------------------------------------------------------------------------
 // Cluster-wide inverse-CDF draw over the row: x = min{k : C_k > u * total}.
 // Every CTA of the cluster calls it; the CTA holding the crossing writes
-// *x_out.  With allow_fallback, a residual whose total is exactly zero
-// (p' == q') is replaced by p'_t.
-// Summation order: each thread sums its contiguous sub-chunk sequentially
-// (tau), lanes are chained in lane order inside a warp (lp = prefix), warps in
-// warp order inside the CTA, CTAs in rank order.  Token j of thread t in warp
-// w has the cumulative value Pc + (Om_w + (lp_t + loc_j)), which at the end of
-// every thread, warp and CTA equals the prefix the next level starts from.
+// *x_out and returns kDrawWrote, the others kDrawNone; when a CTA of the
+// cluster gave up waiting for a copy, every CTA returns kDrawTimeout and
+// nobody writes.  With allow_fallback, a residual whose total is exactly
+// zero (p' == q') is replaced by p'_t.
+// Summation: each thread sums its contiguous sub-chunk sequentially (tau);
+// the lanes' sums are scanned inside the warp (a fixed shuffle tree), the
+// warps' totals chained in warp order, the CTAs' in rank order.  A token's
+// cumulative value is Pc + (Om_w + (lp_t + loc_j)); the search picks the
+// first warp, then lane, then token whose value passes the target, with the
+// very sums used for the totals, so it always lands on a token of the
+// crossing CTA (with a positive weight, or on its last positive one when the
+// target falls in a rounding gap between two lanes).
 // ---------------------------------------------------------------------------
-__device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double *wbuf, DrawSrc src,
+constexpr int kDrawNone = 0;     // this CTA did not write the token
+constexpr int kDrawWrote = 1;    // this CTA found the token and wrote it
+constexpr int kDrawTimeout = 2;  // a CTA of the cluster gave up waiting for a copy (nobody wrote)
+
+__device__ int cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double *wbuf, DrawSrc src,
                              bool allow_fallback, double invT, float u, int v0, int v1, int *x_out,
                              int wait_polls) {
     const int C = (int)cluster.num_blocks();
@@ -491,26 +497,23 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
     const int t0 = min(v1, v0 + tid * ch), t1 = min(v1, t0 + ch);
     // With the statistics kernel's weights, aligned, and room for both rows:
     // the copy engine brings the slices of e_t (and e_d) into shared memory
-    // in vocabulary order, and the residual weights are formed in e_d's place
+    // in vocabulary order; residual weights are combined where they are read
     // (e_t stays intact for the fallback to p'_n).
     const bool bulk = src.Et && n > 0 && (n & 1) == 0 && 2 * n <= kDrawBufDoubles &&
                       aligned16(src.Et + v0) && (src.kind == 0 || aligned16(src.Ed + v0));
-    double *bt = wbuf, *bd = wbuf + n;
+    const double *bt = wbuf, *bd = wbuf + n;
     bool landed = true;
     if (bulk) {
         if (tid == 0) {
             mbar_init(&s.bar);
             const unsigned bytes = (unsigned)n * 8u;
             mbar_expect(&s.bar, src.kind == 1 ? 2u * bytes : bytes);
-            bulk_load(bt, src.Et + v0, bytes, &s.bar);
-            if (src.kind == 1) bulk_load(bd, src.Ed + v0, bytes, &s.bar);
+            bulk_load(wbuf, src.Et + v0, bytes, &s.bar);
+            if (src.kind == 1) bulk_load(wbuf + n, src.Ed + v0, bytes, &s.bar);
         }
         __syncthreads();  // the barrier is initialised before anyone polls it
         landed = mbar_wait(&s.bar, 0, wait_polls);
         if (!landed) mbar_wait(&s.bar, 0, kWaitLimit);  // give the copies in flight a second bound
-        if (src.kind == 1)
-            for (int i = tid; i < n; i += kThreads) bd[i] = draw_combine(src, bt[i], bd[i]);
-        __syncthreads();
     }
     // Otherwise weights are computed once, coalesced, into shared memory;
     // thread t's sub-chunk lives at wbuf[t * P ..] with an odd stride P (no
@@ -519,7 +522,7 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
     const bool buffered = !bulk && ch > 0 && (size_t)kThreads * P <= (size_t)kDrawBufDoubles;
     const double *mine = wbuf + (size_t)tid * P;
     auto wat = [&](int j) -> double {
-        if (bulk) return (src.kind == 1 ? bd : bt)[j - v0];
+        if (bulk) return src.kind == 1 ? draw_combine(src, bt[j - v0], bd[j - v0]) : bt[j - v0];
         return buffered ? mine[j - t0] : draw_weight(src, j, invT);
     };
 
@@ -542,40 +545,39 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
         }
         double tau = 0.0;
         for (int j = t0; j < t1; ++j) tau = __dadd_rn(tau, wat(j));
-        double acc = 0.0, lp = 0.0;
-        for (int r = 0; r < 32; ++r) {
-            const double v = __shfl_sync(0xffffffffu, tau, r);
-            if (r == lane) lp = acc;
-            acc = __dadd_rn(acc, v);
+        // inclusive scan of the lanes' sums (fixed shuffle tree); lp = the
+        // lane's exclusive prefix, wtot = the warp's total
+        double incl = tau;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double v = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl = __dadd_rn(incl, v);
         }
-        if (lane == 0) s.warp_tot[w] = acc;
+        double lp = __shfl_up_sync(0xffffffffu, incl, 1);
+        if (lane == 0) lp = 0.0;
+        if (lane == 31) s.warp_tot[w] = incl;
         __syncthreads();
         if (w == 0) {
             double a = 0.0;
             for (int i = 0; i < kWarps; ++i) a = __dadd_rn(a, s.warp_tot[i]);
             if (lane == 0) s.my_partial = a;
             publish(cluster, s.all_part, rank, C, a);
+            publish(cluster, s.all_bad, rank, C, landed ? 0 : 1);
         }
         cluster.sync();
-        if (!landed && tid == 0) *cluster.map_shared_rank(&s.res_timeout, 0) = 1;
-        if (w == 0) {
-            double pc = 0.0;
-            const double tot = ordered_sum(s.all_part, C, rank, &pc);
-            if (lane == 0) {
-                s.draw_Pc = pc;
-                s.draw_total = tot;
-            }
-        }
-        __syncthreads();
-        const double Pc = s.draw_Pc, total = s.draw_total;
-        if (total == 0.0 && allow_fallback && src.kind == 1) {
+        double Pc = 0.0;
+        const double total = ordered_sum(s.all_part, C, rank, &Pc);  // every warp, same order
+        bool timed_out = false;
+        for (int r = 0; r < C; ++r) timed_out |= s.all_bad[r] != 0;
+        if (total == 0.0 && allow_fallback && src.kind == 1 && !timed_out) {
             src.kind = 0;  // p' == q' exactly: draw from p'_n
             cluster.sync();  // every CTA has read all_part before the next attempt rewrites it
             continue;
         }
         const double target = __dmul_rn((double)u, total);
         const double next = __dadd_rn(Pc, s.my_partial);
-        if (!(Pc <= target && target < next)) return;  // the crossing is in another CTA
+        if (timed_out) return kDrawTimeout;
+        if (!(Pc <= target && target < next)) return kDrawNone;  // the crossing is in another CTA
         if (tid == 0) {
             double a = 0.0, om = 0.0;
             int ws = kWarps - 1;
@@ -585,7 +587,7 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
                 a = nx;
             }
             s.wstar = ws;
-            s.draw_total = om;  // reused: prefix of the crossing warp
+            s.draw_total = om;  // prefix of the crossing warp
             s.x_found = -1;
         }
         __syncthreads();
@@ -607,14 +609,14 @@ __device__ void cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double 
         __syncthreads();
         if (tid == 0) {
             int x = s.x_found;
-            if (x < 0) {  // not reachable with the consistent sums above; stay valid
+            if (x < 0)  // the target fell in a rounding gap: this CTA's last positive weight
                 for (int j = v1 - 1; j >= v0; --j)
-                    if (draw_weight(src, j, invT) > 0.0) { x = j; break; }
-            }
+                    if (wat(j) > 0.0) { x = j; break; }
             *x_out = x;
         }
-        return;
+        return tid == 0 ? kDrawWrote : kDrawNone;
     }
+    return kDrawNone;
 }
 
 // ---------------------------------------------------------------------------
@@ -653,6 +655,8 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     auto lval = [&](int j) -> float { return cached ? cache[j - v0] : L[j]; };
 
     // ---------------- P1: read the slice; max, min, argmax, finiteness ----------------
+    float g_m, g_min;
+    int g_arg, g_bad;
     {
         float mx = -INFINITY, mn = INFINITY;
         int arg = INT_MAX, bad = 0;
@@ -708,24 +712,27 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
             publish(cluster, s.all_bad, rank, C, bb);
         }
         cluster.sync();
-        if (wid == 0) {
-            float gm = lane < C ? s.all_max[lane] : -INFINITY;
-            int ga = lane < C ? s.all_arg[lane] : INT_MAX;
-            float gn = lane < C ? s.all_min[lane] : INFINITY;
-            int gb = lane < C ? s.all_bad[lane] : 0;
-            warp_max_min_arg(gm, ga, gn, gb);
-            if (lane == 0) { s.g_m = gm; s.g_min = gn; s.g_arg = ga; s.g_bad = gb; }
-        }
-        __syncthreads();
+        // every warp combines the cluster's values itself, in the same order
+        // (so with the same result): no warp waits on another after the
+        // cluster barrier
+        float gm = lane < C ? s.all_max[lane] : -INFINITY;
+        int ga = lane < C ? s.all_arg[lane] : INT_MAX;
+        float gn = lane < C ? s.all_min[lane] : INFINITY;
+        int gb = lane < C ? s.all_bad[lane] : 0;
+        warp_max_min_arg(gm, ga, gn, gb);
+        g_m = gm;
+        g_min = gn;
+        g_arg = ga;
+        g_bad = gb;
     }
-    const float m = s.g_m;
-    const bool bad = s.g_bad != 0;
+    const float m = g_m;
+    const bool bad = g_bad != 0;
 
     RowStats st;
     st.m = m;
-    st.lmin = s.g_min;
-    st.argmax = s.g_arg;
-    st.status = (s.g_bad & 2) ? MTPV_ROW_TIMEOUT : bad ? MTPV_ROW_NONFINITE : MTPV_ROW_OK;
+    st.lmin = g_min;
+    st.argmax = g_arg;
+    st.status = (g_bad & 2) ? MTPV_ROW_TIMEOUT : bad ? MTPV_ROW_NONFINITE : MTPV_ROW_OK;
     st.Z = 1.0;
     st.Zk = 1.0;
     st.lstar = -INFINITY;
@@ -734,11 +741,24 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     if (!bad && T > 0.0) {
         // ---------------- P2: exps, Z, level-1 histogram, e-cache ----------------
         const double md = (double)m;
-        const float range = __fsub_rn(m, s.g_min);
+        const float range = __fsub_rn(m, g_min);
         float inv_w = (range > 0.0f) ? __fdiv_rn((float)kBins, range) : 0.0f;
         if (!isfinite(inv_w)) inv_w = 0.0f;
+        // The histogram only locates the crossing bin; the masses that decide
+        // the cut are exact fp64 sums taken afterwards.  Per bin: the token
+        // count and the tokens' excess over the bin's lower edge, e_j / e_lo - 1
+        // as a fraction of the bin's span eps = e_hi / e_lo - 1, in fixed point
+        // of at most qmax per token (32-bit integer atomics, exact and
+        // order-independent).  Bin b spans logits (m - (b + 1) bw, m - b bw].
+        const float bw = inv_w > 0.0f ? __frcp_rn(inv_w) : 0.0f;
+        const float xw = __fmul_rn(bw, (float)invT);            // a bin's span in exponent units
+        const float eps = xw > 0.0f ? expm1f(xw) : 0.0f;
+        const unsigned qmax = (unsigned)min(65536, (int)(4294967295u / (unsigned)max(1, v1 - v0)));
+        const float qscale = eps > 0.0f ? (float)qmax / eps : 0.0f;
+        unsigned *hcnt = reinterpret_cast<unsigned *>(rg.hist_mass);  // [kBins] counts
+        unsigned *hexc = hcnt + kBins;                                 // [kBins] excess
         if (!topp_all) {
-            for (int b = tid; b < kBins; b += kThreads) rg.hist_mass[b] = 0.0;
+            for (int b = tid; b < 2 * kBins; b += kThreads) hcnt[b] = 0u;
             __syncthreads();
         }
         double zt = 0.0;
@@ -760,7 +780,13 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                     if (cached) rg.ecache[j - v0] = ev[q];
                     if (!topp_all) {
                         const int b = bin_of(lv[q], m, inv_w);
-                        atomicAdd(&rg.hist_mass[b], ev[q]);
+                        // excess exp(x) - 1 over the lower edge, x in [0, xw] (xw is
+                        // small: a third-order series is ample for locating)
+                        const float lo = __fsub_rn(m, __fmul_rn((float)(b + 1), bw));
+                        const float x = fminf(xw, fmaxf(0.0f, __fmul_rn(__fsub_rn(lv[q], lo), (float)invT)));
+                        const float ex = __fmul_rn(x, __fmaf_rn(x, __fmaf_rn(x, 0.16666667f, 0.5f), 1.0f));
+                        atomicAdd(&hcnt[b], 1u);
+                        atomicAdd(&hexc[b], min(qmax, __float2uint_rn(__fmul_rn(ex, qscale))));
                     }
                 }
             }
@@ -775,31 +801,34 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
         if (tid == 0) s.cand_count = 0u;
         if (!topp_all) {
             for (int r = wid; r < C; r += kWarps) {
-                double *dst = reinterpret_cast<double *>(cluster.map_shared_rank(rg.cand, r)) + rank * per;
-                for (int i = lane; i < per; i += 32) dst[i] = rg.hist_mass[r * per + i];
+                uint2 *dst = reinterpret_cast<uint2 *>(cluster.map_shared_rank(rg.cand, r)) + rank * per;
+                for (int i = lane; i < per; i += 32)
+                    dst[i] = make_uint2(hcnt[r * per + i], hexc[r * per + i]);
             }
         }
         cluster.sync();
-        if (wid == 0) {
-            const double z = ordered_sum(s.all_Z, C, 0, nullptr);
-            if (lane == 0) s.g_Z = z;
-        }
-        __syncthreads();
-        st.Z = s.g_Z;
+        st.Z = ordered_sum(s.all_Z, C, 0, nullptr);  // every warp, same order
         st.Zk = st.Z;
 
         if (!topp_all) {
             // ---------------- P3: crossing bin, exact cut ----------------
             const double thr = __dmul_rn((double)p.top_p, st.Z);
             const int base = rank * per;
-            // the cluster's histogram on the bins this CTA owns: the C copies
-            // added in rank order
+            // the cluster's histogram on the bins this CTA owns: the C copies'
+            // integer sums, turned into an approximate mass
+            // e_lo (count + excess eps / qmax), e_lo = exp(-(b + 1) xw)
             {
-                const double *scr = reinterpret_cast<const double *>(rg.cand);
+                const uint2 *scr = reinterpret_cast<const uint2 *>(rg.cand);
+                const double kex = (double)eps / (double)qmax;
                 for (int b = tid; b < per; b += kThreads) {
-                    double a = 0.0;
-                    for (int r = 0; r < C; ++r) a = __dadd_rn(a, scr[r * per + b]);
-                    s.own_mass[b] = a;
+                    unsigned long long cn = 0ull, ex = 0ull;
+                    for (int r = 0; r < C; ++r) {
+                        const uint2 v = scr[r * per + b];
+                        cn += v.x;
+                        ex += v.y;
+                    }
+                    const double elo = exp_neg(-(double)(base + b + 1) * (double)xw, s.exp_tab);
+                    s.own_mass[b] = elo * ((double)cn + (double)ex * kex);
                 }
             }
             __syncthreads();
@@ -821,42 +850,53 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                     P = nx;
                 }
                 int bstar = -2;
-                double A = P;
                 if (cstar == rank) {
                     int f;
                     double bef;
                     warp_prefix_search(s.own_mass, per, Pstar, thr, true, &f, &bef);
                     if (f < 0) f = per - 1;  // not reachable: the range total reached thr
                     bstar = base + f;
-                    A = bef;
                 } else if (cstar < 0 && rank == 0) {
-                    bstar = -1;  // thr above the histogram total (top_p within rounding of 1)
+                    bstar = -1;  // thr above the histogram total (top_p within its rounding of 1)
                 }
-                if (bstar != -2 && lane < C) {
-                    *cluster.map_shared_rank(&s.bc_bin, lane) = bstar;
-                    *cluster.map_shared_rank(&s.bc_A, lane) = A;
-                }
+                if (bstar != -2 && lane < C) *cluster.map_shared_rank(&s.bc_bin, lane) = bstar;
             }
             cluster.sync();
             const int bstar = s.bc_bin;
-            const double A = s.bc_A;
-            // gather the crossing bin's tokens into CTA 0: stage them
-            // locally, reserve a range with one remote atomic, copy.  The
-            // bin's size is known once every CTA has reserved its range; a bin
-            // above the candidate capacity takes the radix select instead.
+            // One pass over the slice: the exact mass above the located bin (A)
+            // and in it (M), fp64 sums in a fixed order (each thread's tokens
+            // in index order, then fixed trees, then the CTAs in rank order), so
+            // they are the same bits in every run; and the located bin's tokens
+            // gathered into CTA 0: staged locally, a range reserved with one
+            // remote atomic, copied.  The bin's size is known once every CTA has
+            // reserved its range.
             unsigned total = 0u;
+            double A = 0.0, Mb = 0.0;
             if (bstar >= 0) {
                 unsigned long long *stage = reinterpret_cast<unsigned long long *>(rg.cand_e);
                 if (tid == 0) s.local_n = 0u;
                 __syncthreads();
+                double a_loc = 0.0, m_loc = 0.0;
                 for (int j = v0 + tid; j < v1; j += kThreads) {
                     const float l = lval(j);
-                    if (bin_of(l, m, inv_w) == bstar) {
-                        const unsigned slot = atomicAdd(&s.local_n, 1u);
-                        if (slot < (unsigned)kCandCap) stage[slot] = rank_key(l, j);
+                    const int b = bin_of(l, m, inv_w);
+                    if (b <= bstar) {
+                        const double e = cached ? rg.ecache[j - v0] : e_of(l, md, invT, s.exp_tab);
+                        if (b < bstar) {
+                            a_loc = __dadd_rn(a_loc, e);
+                        } else {
+                            m_loc = __dadd_rn(m_loc, e);
+                            const unsigned slot = atomicAdd(&s.local_n, 1u);
+                            if (slot < (unsigned)kCandCap) stage[slot] = rank_key(l, j);
+                        }
                     }
                 }
-                __syncthreads();
+                const double a_cta = block_sum_d(a_loc, s);  // also completes the staging
+                const double m_cta = block_sum_d(m_loc, s);
+                if (wid == 0) {
+                    publish(cluster, s.all_part, rank, C, a_cta);
+                    publish(cluster, s.all_M, rank, C, m_cta);
+                }
                 const unsigned nloc = min(s.local_n, (unsigned)kCandCap);
                 if (tid == 0)
                     s.local_base = nloc ? atomicAdd(cluster.map_shared_rank(&s.cand_count, 0), nloc) : 0u;
@@ -869,11 +909,15 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 }
                 cluster.sync();
                 total = *cluster.map_shared_rank(&s.cand_count, 0);
+                A = ordered_sum(s.all_part, C, 0, nullptr);  // every warp, same order
+                Mb = ordered_sum(s.all_M, C, 0, nullptr);
             }
-            if (bstar < 0 || total == 0u) {
-                st.Zk = st.Z;  // nothing to cut (top_p within rounding of 1): keep all
-                if (bstar >= 0) cluster.sync();  // every CTA has read CTA 0's count
-            } else if (total <= (unsigned)kCandCap) {
+            // The exact cut lies in the located bin iff A < thr <= A + M.  The
+            // approximate histogram can miss by a bin when thr falls within its
+            // rounding of a bin edge, and finds no bin when thr is within it of
+            // the total: the radix select then finds the cut from scratch.
+            const bool located = bstar >= 0 && total > 0u && A < thr && thr <= __dadd_rn(A, Mb);
+            if (located && total <= (unsigned)kCandCap) {
                 if (rank == 0 && (int)total <= kThreads) {
                     // one candidate per thread: its rank among the others (the
                     // keys are distinct, they carry the token index) places it
@@ -1115,47 +1159,52 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
         rd = i < K ? b * S + K + 1 + i : rt;
     }
     const bool residual = p.verify && i < K;
-    if (rank == 0 && tid == 0) {
-        s.res_x = -1;
-        s.res_acc = 0;
-        s.res_timeout = 0;
-    }
+    if (rank == 0 && tid == 0) s.res_acc = 0;
     build_exp_table(s.exp_tab);
     __syncthreads();
     wait_for_producer();  // the statistics kernel's rows and weights
-    const RowStats st_t = p.slots[rt].st;
-    const RowStats st_d = p.slots[rd].st;
     const float *Lt = row_ptr(p, rt), *Ld = row_ptr(p, rd);
     const double *Et = p.ecache ? p.ecache + (size_t)rt * V : nullptr;
     const double *Ed = p.ecache ? p.ecache + (size_t)rd * V : nullptr;
 
-    // ---------------- acceptance test of d_i ----------------
-    int status = st_t.status;
+    // ---------------- the position's status, acceptance test of d_i ----------------
+    // (verify: the slot of target row i becomes position i's record, whose
+    // first 12 bytes are written after the last cluster barrier below; the
+    // status field of the row statistics lies past them and is read first)
+    int status = p.slots[rt].st.status;
+    int d = 0;
     if (residual) {
-        const int d = p.drafts[(size_t)b * K + i];
+        d = p.drafts[(size_t)b * K + i];
+        const int sd = p.slots[rd].st.status;
         if (d < 0 || d >= V) status = MTPV_ROW_BAD_DRAFT;
-        else if (st_d.status != MTPV_ROW_OK && status == MTPV_ROW_OK) status = st_d.status;
-        if (status == MTPV_ROW_OK && rank == 0 && tid == 0) {
-            double pt, qd;  // p'_i(d_i), q'_i(d_i)
-            if (Et && T > 0.0) {
-                pt = Et[d] / st_t.Zk;
-                qd = Ed[d] / st_d.Zk;
-            } else {
-                pt = warped_prob(st_t, Lt, d, T, invT, s.exp_tab);
-                qd = warped_prob(st_d, Ld, d, T, invT, s.exp_tab);
-            }
-            const double ratio = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
-            s.res_acc = (double)p.u_acc[(size_t)b * K + i] < ratio ? 1 : 0;
+        else if (sd != MTPV_ROW_OK && status == MTPV_ROW_OK) status = sd;
+    }
+    const bool draws = status == MTPV_ROW_OK && T > 0.0;
+    RowStats st_t = {}, st_d = {};
+    if (draws || (rank == 0 && tid == 0)) {
+        st_t = p.slots[rt].st;
+        st_d = p.slots[rd].st;
+    }
+    if (residual && status == MTPV_ROW_OK && rank == 0 && tid == 0) {
+        double pt, qd;  // p'_i(d_i), q'_i(d_i)
+        if (Et && T > 0.0) {
+            pt = Et[d] / st_t.Zk;
+            qd = Ed[d] / st_d.Zk;
+        } else {
+            pt = warped_prob(st_t, Lt, d, T, invT, s.exp_tab);
+            qd = warped_prob(st_d, Ld, d, T, invT, s.exp_tab);
         }
+        const double ratio = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
+        s.res_acc = (double)p.u_acc[(size_t)b * K + i] < ratio ? 1 : 0;
     }
 
     // ---------------- this position's residual / bonus draw ----------------
-    int *x_dst = p.verify ? cluster.map_shared_rank(&s.res_x, 0) : &p.out_tokens[c];
-    if (status != MTPV_ROW_OK) {
-        if (rank == 0 && tid == 0) *x_dst = -1;
-    } else if (T == 0.0) {
-        if (rank == 0 && tid == 0) *x_dst = st_t.argmax;
-    } else {
+    // The CTA that finds the token writes it to global memory itself (verify:
+    // the record's x; sample: the output), so no CTA waits for another at the
+    // end.  CTA 0 writes it instead when no draw runs or the draw timed out.
+    int *x_dst = p.verify ? &p.slots[rt].rec.x : &p.out_tokens[c];
+    int drew = kDrawNone;
+    if (draws) {
         DrawSrc src;
         src.st_t = st_t;
         src.st_d = residual ? st_d : st_t;
@@ -1167,31 +1216,34 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
         src.rho = residual ? st_t.Zk / st_d.Zk : 1.0;
         src.kind = residual ? 1 : 0;
         const float u = p.verify ? p.u_samp[(size_t)b * (K + 1) + i] : p.u_samp[c];
-        cluster_draw(cluster, s, wbuf, src, residual, invT, u, v0, v1, x_dst, p.wait_polls);
+        drew = cluster_draw(cluster, s, wbuf, src, residual, invT, u, v0, v1, x_dst, p.wait_polls);
     }
-    if (rank == 0 && tid == 0 && !p.verify && p.row_status) p.row_status[c] = status;
-    cluster.sync();  // verify: res_x and res_acc are in CTA 0; no CTA exits while a peer reads it
-    if (rank != 0 || tid != 0) return;
-    if (s.res_timeout) status = MTPV_ROW_TIMEOUT;
-    if (!p.verify) {
-        if (status == MTPV_ROW_TIMEOUT) {
-            p.out_tokens[c] = -1;
+    if (drew == kDrawTimeout) status = MTPV_ROW_TIMEOUT;
+    const bool cta0_token = status != MTPV_ROW_OK || T == 0.0;
+    unsigned tickets = 0u;
+    if (rank == 0 && tid == 0) {
+        if (cta0_token) *x_dst = status == MTPV_ROW_OK ? st_t.argmax : -1;
+        if (!p.verify) {
             if (p.row_status) p.row_status[c] = status;
+            return;
         }
-        return;
+        // the record's other fields, and one ticket for them (two when
+        // this thread wrote the token as well)
+        p.slots[rt].rec.accept = s.res_acc;
+        p.slots[rt].rec.status = status;
+        tickets = cta0_token ? 2u : 1u;
     }
+    if (!p.verify) return;
+    if (drew == kDrawWrote && tid == 0) tickets += 1u;  // the token's ticket
+    if (tickets == 0u) return;
 
-    // ---------------- record, ticket, and (last cluster) the sequence's outputs ----------------
+    // ---------------- tickets, and (last) the sequence's outputs ----------------
+    // Two tickets per position; the thread that completes the sequence's
+    // 2 (K + 1) writes its outputs (nobody waits for anybody).
     const int S = 2 * K + 1;
-    PosRecord rec;
-    rec.x = s.res_x;
-    rec.accept = s.res_acc;
-    rec.status = status;
-    rec.pad = 0;
-    p.slots[rt].rec = rec;  // target row i's statistics are not read again
     __threadfence();
-    const unsigned old = atomicAdd(&p.counters[b], 1u);
-    if (old != (unsigned)K) return;  // another position of sequence b finishes last
+    const unsigned old = atomicAdd(&p.counters[b], tickets);
+    if (old + tickets != 2u * (unsigned)(K + 1)) return;
     __threadfence();
     int seq_status = MTPV_ROW_OK, n = K;
     for (int k = 0; k <= K; ++k) {
