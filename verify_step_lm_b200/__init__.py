@@ -143,6 +143,9 @@ def lm_head_smallm(x, w, scales, fmt: int, y, ws=None, stream=None):
     """y[M, N] (fp32) = x[M, Kd] (bf16) . Wd^T for a bf16 or int4-g64 head."""
     M, Kd = x.shape
     N = w.shape[0]
+    if ws is None:
+        need = lm_head_workspace_bytes(M, Kd, N, fmt)
+        ws = workspace(need, x.device) if need else None
     wsb = 0 if ws is None else ws.numel() * ws.element_size()
     _check("mtpv_lm_head_smallm", load().mtpv_lm_head_smallm(
         _ptr(x), M, Kd, N, _ptr(w), _ptr(scales), fmt, _ptr(y), _ptr(ws), wsb, _stream(stream)))

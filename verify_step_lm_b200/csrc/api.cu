@@ -44,13 +44,27 @@ VerifyWs verify_layout(int B, int K, int V) {
     return l;
 }
 
+// Both heads' scratch: the fused kernel's work counter, then each head's own
+// scratch when the two run as separate launches.
+struct HeadsWs {
+    size_t work, t, d, total;
+};
+HeadsWs heads_layout(int Mt, int Md, int Kd) {
+    HeadsWs l;
+    l.work = 0;
+    l.t = up(mtpv::kHeadsPairWorkBytes);
+    l.d = l.t + up(mtpv::lm_head_scratch_bytes(Mt, Kd, MTPV_W_BF16));
+    l.total = l.d + up(mtpv::lm_head_scratch_bytes(Md, Kd, MTPV_W_INT4_G64));
+    return l;
+}
+
 struct StepWs {
     size_t heads, tl, dl, verify, total;
 };
-StepWs step_layout(int B, int K, int V) {
+StepWs step_layout(int B, int K, int V, int h) {
     StepWs l;
-    l.heads = 0;  // the fused heads kernel's work counter
-    l.tl = l.heads + up(mtpv::kHeadsPairWorkBytes);
+    l.heads = 0;  // both heads' scratch
+    l.tl = l.heads + heads_layout(B * (K + 1), B * K, h).total;
     l.dl = l.tl + up(sizeof(float) * (size_t)B * (K + 1) * V);
     l.verify = l.dl + up(sizeof(float) * (size_t)B * K * V);
     l.total = l.verify + verify_layout(B, K, V).total;
@@ -63,7 +77,7 @@ struct HostWs {
 HostWs host_layout(int B, int K, int V, int h) {
     HostWs l;
     l.step = 0;
-    l.ht = step_layout(B, K, V).total;
+    l.ht = step_layout(B, K, V, h).total;
     l.hd = l.ht + up((size_t)B * (K + 1) * h * 2);
     l.drafts = l.hd + up((size_t)B * K * h * 2);
     l.ua = l.drafts + up(sizeof(int32_t) * (size_t)B * K);
@@ -79,7 +93,7 @@ HostWs host_layout(int B, int K, int V, int h) {
 // tokens (B > 1 only: gathered from / scattered to the [B, K] layouts), then
 // the sampler's workspace.
 struct DraftWs {
-    size_t x, y, u, tok, samp, total;
+    size_t x, y, u, tok, samp, head, total;
 };
 size_t sample_ws_bytes(int R, int V) {
     return up(sizeof(mtpv::RowSlot) * (size_t)R) + up(sizeof(double) * (size_t)R * V);
@@ -91,7 +105,8 @@ DraftWs draft_layout(int B, int V, int h) {
     l.u = l.y + up(sizeof(float) * (size_t)B * V);
     l.tok = l.u + up(sizeof(float) * (size_t)B);
     l.samp = l.tok + up(sizeof(int32_t) * (size_t)B);
-    l.total = l.samp + sample_ws_bytes(B, V);
+    l.head = l.samp + sample_ws_bytes(B, V);
+    l.total = l.head + up(mtpv::lm_head_scratch_bytes(B, h, MTPV_W_INT4_G64));
     return l;
 }
 
@@ -103,14 +118,16 @@ bool lm_head_shape_ok(int M, int Kd, int N) {
 char *at(void *ws, size_t off) { return static_cast<char *>(ws) + off; }
 
 // Both heads: one fused launch when the kernel takes the shapes, else two.
+// ws holds heads_layout(Mt, Md, Kd).total bytes.
 cudaError_t launch_heads(const void *xt, int Mt, const void *w, float *yt, const void *xd, int Md,
-                         const void *wq, const void *scales, float *yd, int Kd, int N, void *work,
+                         const void *wq, const void *scales, float *yd, int Kd, int N, void *ws,
                          cudaStream_t s) {
+    const HeadsWs l = heads_layout(Mt, Md, Kd);
     if (mtpv::lm_heads_pair_ok(Mt, Md, Kd, scales))
-        return mtpv::launch_lm_heads_pair(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, work, s);
-    cudaError_t e = mtpv::launch_lm_head(xt, Mt, Kd, N, w, nullptr, MTPV_W_BF16, yt, s);
+        return mtpv::launch_lm_heads_pair(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, at(ws, l.work), s);
+    cudaError_t e = mtpv::launch_lm_head(xt, Mt, Kd, N, w, nullptr, MTPV_W_BF16, yt, at(ws, l.t), s);
     if (e != cudaSuccess) return e;
-    return mtpv::launch_lm_head(xd, Md, Kd, N, wq, scales, MTPV_W_INT4_G64, yd, s);
+    return mtpv::launch_lm_head(xd, Md, Kd, N, wq, scales, MTPV_W_INT4_G64, yd, at(ws, l.d), s);
 }
 
 mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *drafts, const float *ua,
@@ -161,24 +178,25 @@ const char *mtpv_status_string(mtpv_status st) {
 }
 
 size_t mtpv_lm_head_workspace_bytes(int M, int Kd, int N, mtpv_wfmt fmt) {
-    (void)M; (void)Kd; (void)N; (void)fmt;
-    return 0;
+    if (!lm_head_shape_ok(M, Kd, N) || (fmt != MTPV_W_BF16 && fmt != MTPV_W_INT4_G64)) return 0;
+    return mtpv::lm_head_scratch_bytes(M, Kd, (int)fmt);
 }
 
 mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, const void *w,
                                 const void *scales, mtpv_wfmt fmt, float *y, void *ws,
                                 size_t ws_bytes, mtpv_stream stream) {
-    (void)ws; (void)ws_bytes;
     if (!x || !w || !y || !lm_head_shape_ok(M, Kd, N)) return MTPV_ERR_INVALID_ARG;
     if (fmt != MTPV_W_BF16 && fmt != MTPV_W_INT4_G64) return MTPV_ERR_INVALID_ARG;
     if (fmt == MTPV_W_INT4_G64 && (!scales || !aligned(scales, 2))) return MTPV_ERR_INVALID_ARG;
     if (!aligned(x, 16) || !aligned(w, 16) || !aligned(y, 4)) return MTPV_ERR_INVALID_ARG;
-    return cuda_status(mtpv::launch_lm_head(x, M, Kd, N, w, scales, (int)fmt, y, (cudaStream_t)stream));
+    const size_t need = mtpv::lm_head_scratch_bytes(M, Kd, (int)fmt);
+    if (need && (!ws || !aligned(ws, kAlign) || ws_bytes < need)) return MTPV_ERR_WORKSPACE;
+    return cuda_status(mtpv::launch_lm_head(x, M, Kd, N, w, scales, (int)fmt, y, ws, (cudaStream_t)stream));
 }
 
 size_t mtpv_lm_head_pair_workspace_bytes(int Mt, int Md, int Kd, int N) {
     if (!lm_head_shape_ok(Mt, Kd, N) || !lm_head_shape_ok(Md, Kd, N)) return 0;
-    return mtpv::kHeadsPairWorkBytes;
+    return heads_layout(Mt, Md, Kd).total;
 }
 
 mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt, const void *xd,
@@ -189,7 +207,7 @@ mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt, 
     if (!aligned(xt, 16) || !aligned(w, 16) || !aligned(yt, 4) || !aligned(xd, 16) ||
         !aligned(wq, 16) || !aligned(scales, 2) || !aligned(yd, 4))
         return MTPV_ERR_INVALID_ARG;
-    if (!ws || !aligned(ws, 4) || ws_bytes < mtpv::kHeadsPairWorkBytes) return MTPV_ERR_WORKSPACE;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < heads_layout(Mt, Md, Kd).total) return MTPV_ERR_WORKSPACE;
     return cuda_status(launch_heads(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, ws, (cudaStream_t)stream));
 }
 
@@ -320,7 +338,7 @@ mtpv_status mtpv_draft_loop(const void *w_draft, const void *s_draft, const void
                                       sizeof(float), B, cudaMemcpyDeviceToDevice, s);
             if (e != cudaSuccess) return cuda_status(e);
         }
-        e = mtpv::launch_lm_head(x, B, h, V, w_draft, s_draft, MTPV_W_INT4_G64, y, s);
+        e = mtpv::launch_lm_head(x, B, h, V, w_draft, s_draft, MTPV_W_INT4_G64, y, at(ws, l.head), s);
         if (e != cudaSuccess) return cuda_status(e);
         mtpv::SamplerParams p = {};
         p.tl = y;
@@ -350,7 +368,7 @@ mtpv_status mtpv_draft_loop(const void *w_draft, const void *s_draft, const void
 
 size_t mtpv_verify_step_workspace_bytes(int B, int K, int V, int h) {
     if (!verify_shape_ok(B, K, V) || B * (K + 1) > 64 || h < 64 || h % 64) return 0;
-    return step_layout(B, K, V).total;
+    return step_layout(B, K, V, h).total;
 }
 
 mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const void *s_draft,
@@ -371,7 +389,7 @@ mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const vo
         return MTPV_ERR_INVALID_ARG;
     if ((target_logits && !aligned(target_logits, 4)) || (draft_logits && !aligned(draft_logits, 4)))
         return MTPV_ERR_INVALID_ARG;
-    const StepWs l = step_layout(B, K, V);
+    const StepWs l = step_layout(B, K, V, h);
     if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MTPV_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     float *tl = target_logits ? target_logits : reinterpret_cast<float *>(at(ws, l.tl));

@@ -26,6 +26,7 @@
 
 #include "common.cuh"
 #include "lm_head.cuh"
+#include "lm_head_tc.cuh"
 
 namespace mtpv {
 
@@ -918,9 +919,22 @@ size_t lm_head_max_smem_rows(int Kd) {
     return (size_t)(227 * 1024) / ((size_t)Kd * sizeof(float));
 }
 
+size_t lm_head_scratch_bytes(int M, int Kd, int fmt) {
+    if (fmt == MTPV_W_BF16 && M > 8 && lm_head_tc_ok(M, Kd, nullptr, nullptr)) return 256;
+    return 0;
+}
+
 cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, const void *scales,
-                           int fmt, float *y, cudaStream_t s) {
+                           int fmt, float *y, void *scratch, cudaStream_t s) {
     const uint16_t *xb = static_cast<const uint16_t *>(x);
+    if (fmt == MTPV_W_BF16 && M > 8 && lm_head_tc_ok(M, Kd, x, w)) {
+        // every weight read once, all rows per tile, on the tensor-memory kernel
+        unsigned int *err = static_cast<unsigned int *>(scratch);
+        if (!err) return cudaErrorInvalidValue;
+        cudaError_t e = cudaMemsetAsync(err, 0, sizeof(unsigned int), s);
+        if (e != cudaSuccess) return e;
+        return launch_lm_head_bf16_tc(x, M, Kd, N, w, y, err, s);
+    }
     if (fmt == MTPV_W_BF16) {
         // the tensor-core kernel: 16 rows per pass when more than 8 rows come
         // and 16 staged rows fit, else passes of up to 8 rows

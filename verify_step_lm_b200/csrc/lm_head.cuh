@@ -10,10 +10,16 @@ namespace mtpv {
 // supported Kd (<= 58112); the int4 path takes passes of min(8, this) rows.
 size_t lm_head_max_smem_rows(int Kd);
 
+// Device scratch of launch_lm_head for this shape (256-byte aligned; 0 when
+// the shape needs none): rows past 8 of the bf16 head run on the tensor-
+// memory kernel, whose first word is its error word (nonzero after the call:
+// a bounded device wait gave up and y is not valid).
+size_t lm_head_scratch_bytes(int M, int Kd, int fmt);
+
 // y[M, N] = x[M, Kd] . Wd[N, Kd]^T; fmt is an mtpv_wfmt.  Arguments are
-// validated by the caller.
+// validated by the caller; scratch holds lm_head_scratch_bytes(M, Kd, fmt).
 cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, const void *scales,
-                           int fmt, float *y, cudaStream_t s);
+                           int fmt, float *y, void *scratch, cudaStream_t s);
 
 // Both heads of a verify step in one launch: yt[Mt, N] = xt . W^T (bf16 head)
 // and yd[Md, N] = xd . deq(Wq, S)^T (int4 group-64 head), same Kd and N.
