@@ -79,3 +79,63 @@ def test_workspace_is_required():
     p = lambda t: ctypes.c_void_p(t.data_ptr())
     st = lib.mtpv_lm_head_smallm(p(x), M, Kd, N, p(W), None, mtpv.W_BF16, p(y), None, 0, None)
     assert st == 3  # MTPV_ERR_WORKSPACE
+
+
+# ---------------------------------------------------------------------------
+# int4 group-64 head (dequantised into tensor memory, fp16 MMA)
+# ---------------------------------------------------------------------------
+def run_int4(x, Wq, S):
+    M, Kd = x.shape
+    N = Wq.shape[0]
+    need = mtpv.lm_head_workspace_bytes(M, Kd, N, mtpv.W_INT4_G64)
+    assert need >= 4
+    ws = torch.full((need,), 0x5A, dtype=torch.uint8, device="cuda")
+    y = torch.full((M, N), float("nan"), dtype=torch.float32, device="cuda")
+    mtpv.lm_head_smallm(x.cuda(), Wq.cuda(), S.cuda(), mtpv.W_INT4_G64, y, ws=ws)
+    torch.cuda.synchronize()
+    assert int(ws[:4].view(torch.int32).item()) == 0, "a bounded wait of the kernel gave up"
+    return y
+
+
+@pytest.mark.parametrize("M,Kd,N", [(9, 512, 4097), (24, 5120, 3001), (32, 1024, 129), (64, 512, 300),
+                                    (17, 2048, 1), (48, 8192, 200)])
+def test_int4_against_oracle(M, Kd, N):
+    W = synth.make_head(N, Kd, 0.02, seed=7 * N + Kd)
+    Wq, S = synth.quantize_int4_g64(W)
+    x = synth.gaussian((M, Kd), 1.0, seed=3 * M + Kd)
+    y = run_int4(x, Wq, S).cpu().numpy()
+    assert np.isfinite(y).all()
+    ref = oracle.lm_head_int4g64(synth.bf16_bits(x), Wq.numpy(), synth.bf16_bits(S), threads=8)
+    assert_logits_close(y, ref)
+
+
+@pytest.mark.parametrize("M,N", [(24, 1500), (9, 300), (64, 129)])
+def test_int4_bit_exact_on_small_integers(M, N):
+    # power-of-two scales, small-integer activations: the products and every
+    # partial sum are exact in fp32 (within 20 bits of each other)
+    rng = np.random.default_rng(100 + M)
+    Kd = 1024
+    Wq = torch.tensor(rng.integers(0, 256, size=(N, Kd // 2)), dtype=torch.uint8)
+    S = torch.tensor(2.0 ** rng.integers(-2, 3, size=(N, Kd // 64)), dtype=torch.float32).to(torch.bfloat16)
+    x = torch.tensor(rng.integers(-3, 4, size=(M, Kd)), dtype=torch.float32).to(torch.bfloat16)
+    y = run_int4(x, Wq, S).cpu().numpy()
+    ref = oracle.lm_head_int4g64(synth.bf16_bits(x), Wq.numpy(), synth.bf16_bits(S))
+    assert np.array_equal(y.astype(np.float64), ref)
+
+
+def test_int4_repeatable_and_wide_scale_range():
+    # rows whose group scales span 2^12 (and one all-zero row): the per-row
+    # power of two keeps every dequantised weight exact in fp16
+    N, Kd, M = 3000, 5120, 24
+    W = synth.make_head(N, Kd, 0.02, seed=21)
+    W[5] *= 4096.0
+    W[6] *= 1.0 / 4096.0
+    W[7] = 0.0
+    W[8, :64] *= 2048.0
+    Wq, S = synth.quantize_int4_g64(W.to(torch.bfloat16))
+    x = synth.gaussian((M, Kd), 1.0, seed=22)
+    a = run_int4(x, Wq, S)
+    b = run_int4(x, Wq, S)
+    assert torch.equal(a, b)
+    ref = oracle.lm_head_int4g64(synth.bf16_bits(x), Wq.numpy(), synth.bf16_bits(S), threads=8)
+    assert_logits_close(a.cpu().numpy(), ref)

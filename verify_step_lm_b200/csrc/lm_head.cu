@@ -921,6 +921,8 @@ size_t lm_head_max_smem_rows(int Kd) {
 
 size_t lm_head_scratch_bytes(int M, int Kd, int fmt) {
     if (fmt == MTPV_W_BF16 && M > 8 && lm_head_tc_ok(M, Kd, nullptr, nullptr)) return 256;
+    if (fmt == MTPV_W_INT4_G64 && M > 8 && lm_head_tc_int4_ok(M, Kd, nullptr, nullptr, nullptr))
+        return lm_head_int4_tc_scratch_bytes(M, Kd);
     return 0;
 }
 
@@ -951,6 +953,8 @@ cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, c
         }
         return cudaSuccess;
     }
+    if (M > 8 && lm_head_tc_int4_ok(M, Kd, x, w, scales))  // one pass, on the tensor-memory kernel
+        return launch_lm_head_int4_tc(x, M, Kd, N, w, scales, y, scratch, s);
     // int4 group-64: passes of up to 8 rows, each on the ring kernel when it
     // takes the shape, else on the direct-load kernel (same bits)
     const int step = (int)std::min<size_t>(8, lm_head_max_smem_rows(Kd));

@@ -15,4 +15,18 @@ bool lm_head_tc_ok(int M, int Kd, const void *x, const void *w);
 cudaError_t launch_lm_head_bf16_tc(const void *x, int M, int Kd, int N, const void *w, float *y,
                                    unsigned int *err, cudaStream_t s);
 
+// The int4 group-64 head on the same path: M in 9..64, Kd a multiple of 512
+// (at most 16384), x, wq and scales 16-byte aligned.
+bool lm_head_tc_int4_ok(int M, int Kd, const void *x, const void *wq, const void *scales);
+
+// Scratch of launch_lm_head_int4_tc: the error word, the activations'
+// power-of-two factors and their fp16 copy.
+size_t lm_head_int4_tc_scratch_bytes(int M, int Kd);
+
+// y[M, N] = x . deq(wq, scales)^T in one pass over the nibbles (a staging
+// launch, then the tensor-memory kernel); scratch's first word is the error
+// word, as for the bf16 kernel.
+cudaError_t launch_lm_head_int4_tc(const void *x, int M, int Kd, int N, const void *wq, const void *scales,
+                                   float *y, void *scratch, cudaStream_t s);
+
 }  // namespace mtpv
