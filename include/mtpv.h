@@ -108,20 +108,25 @@ MTPV_API void mtpv_set_wait_polls(int polls);
  *   y[m][n] = sum_k x[m][k] * Wd[n][k],  0 <= m < M, 0 <= n < N   (fp32 out)
  *
  *   x       device, bf16 [M, Kd] row-major (activations / hidden states).
- *   M       rows, 1 <= M <= 64.  MTPV_W_BF16 runs on the tensor cores
- *           (mma.sync bf16, fp32 accumulation) in passes of up to 8 rows, or
- *           16 when M > 8 and Kd <= 7232; a pass stages its rows as bf16 in
- *           shared memory, so at most floor(232448 / (2 (Kd + 32))) rows go
- *           in one pass.  MTPV_W_INT4_G64 goes in passes of
- *           min(8, floor(232448 / (4 Kd))) rows.  The weights are re-read
- *           once per pass.
+ *   M       rows, 1 <= M <= 64.
+ *           M <= 8: mma.sync on the tensor cores (fp32 accumulation), rows
+ *           staged in shared memory.  MTPV_W_INT4_G64 dequantises exactly to
+ *           fp16 (activations scaled per row by a power of two) with one
+ *           fresh accumulator per 64-weight group: through per-warp
+ *           shared-memory rings when Kd is a multiple of 512, the scales
+ *           are 16-byte aligned and (M + 1)(2 Kd + 16) + Kd/2 <= 75776
+ *           bytes, else with direct register loads (the same bits).
+ *           9 <= M <= 64: one pass over the weights on tcgen05 (fifth-
+ *           generation tensor cores, fp32 accumulators in tensor memory,
+ *           weights streamed by TMA; rows padded to a multiple of 16).
+ *           MTPV_W_BF16 takes it for any Kd; MTPV_W_INT4_G64 when Kd is a
+ *           multiple of 512 and at most 8192 and x, w and scales are 16-byte
+ *           aligned (the nibbles are dequantised to exact fp16 (n - 8) s f,
+ *           f a per-row power of two, and the activations staged once as
+ *           fp16 times a per-row power of two); other int4 shapes go in
+ *           passes of min(8, floor(232448 / (4 Kd))) rows, re-reading the
+ *           weights once per pass.
  *   Kd      reduction length, a positive multiple of 64, at most 58112.
- *           MTPV_W_INT4_G64 runs on the tensor cores (fp16 MMA of exactly
- *           dequantised nibbles, fp32 accumulation per 64-weight group):
- *           through per-warp shared-memory rings when Kd is a multiple of
- *           512, the scales are 16-byte aligned and
- *           (M + 1)(2 Kd + 16) + Kd/2 <= 75776 bytes (M <= 6 at Kd = 5120),
- *           else with direct register loads; both forms give the same bits.
  *   N       output columns (vocabulary rows of the head), N >= 1.
  *   w       device weights, layout per fmt:
  *             MTPV_W_BF16:     bf16 [N, Kd] (nn.Linear out x in layout);
@@ -134,7 +139,13 @@ MTPV_API void mtpv_set_wait_polls(int polls);
  *   scales  device bf16 [N, Kd/64] for MTPV_W_INT4_G64 (2-byte aligned);
  *           ignored for MTPV_W_BF16.
  *   y       device fp32 [M, N] row-major, fully overwritten (4-byte aligned).
- *   ws, ws_bytes  workspace (may be NULL when the query returns 0).
+ *   ws, ws_bytes  workspace of mtpv_lm_head_workspace_bytes() bytes, 256-byte
+ *           aligned (may be NULL when the query returns 0, as it does for
+ *           M <= 8).  On the tcgen05 path its first 32-bit word is an error
+ *           word, cleared by the call: nonzero once the call has run means
+ *           a bounded device-side wait gave up and y is not valid (the
+ *           kernel never hangs).  The int4 path also stages the activations
+ *           there.
  * Accumulation is fp32.  Errors: MTPV_ERR_INVALID_ARG for NULL pointers,
  * M/Kd/N out of range or misaligned x/w; MTPV_ERR_WORKSPACE when ws_bytes is
  * below mtpv_lm_head_workspace_bytes().
@@ -166,9 +177,11 @@ MTPV_API mtpv_status mtpv_lm_head_smallm(const void *x, int M, int Kd, int N, co
  * launches.
  * Either way the values are those mtpv_lm_head_smallm gives (same
  * arithmetic, bit for bit).
- * ws, ws_bytes: at least mtpv_lm_head_pair_workspace_bytes() bytes (256),
- * 4-byte aligned; need not be initialised (the call clears its counter on
- * `stream`).  Errors: as mtpv_lm_head_smallm, and MTPV_ERR_WORKSPACE.
+ * ws, ws_bytes: at least mtpv_lm_head_pair_workspace_bytes() bytes (256,
+ * plus each head's mtpv_lm_head_workspace_bytes() when the heads run as two
+ * launches), 256-byte aligned; need not be initialised (the call clears its
+ * counter on `stream`).  Errors: as mtpv_lm_head_smallm, and
+ * MTPV_ERR_WORKSPACE.
  * ---------------------------------------------------------------------- */
 MTPV_API size_t mtpv_lm_head_pair_workspace_bytes(int Mt, int Md, int Kd, int N);
 MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt,
@@ -193,18 +206,20 @@ MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, fl
  *   x       device bf16 [M, Kd] (16-byte aligned), 1 <= M <= 64.
  *   wq      device uint8 [N, Kd/2] (N = 2F for gate_up), MTPV_W_INT4_G64
  *           nibble order; scales device bf16 [N, Kd/64].
- *   Kd      a positive multiple of 64, at most 2^20.  Passes of up to 8
- *           rows (one MMA n-tile); the weights are read once per pass.  The
- *           activations of a pass are staged once, as fp16 in the MMA
- *           operand order, into the workspace.
+ *   Kd      a positive multiple of 64, at most 2^20.  One launch per pass of
+ *           up to 8 rows (one MMA n-tile); the weights are read once per
+ *           pass.
  *   y, h    device fp32 [M, N] / [M, F], fully overwritten.
- * The reduction over Kd is split into slices when N alone gives too few
- * 16-row tiles to fill the GPU; the slices' partial sums (workspace) are
- * added in a fixed order, so results are deterministic.  Arithmetic: fp16
- * MMA of exactly dequantised weights, fp32 accumulation per group, as
- * mtpv_lm_head_smallm's int4 path.
+ * Arithmetic: bf16 mma.sync of exactly dequantised weights (the nibble n
+ * becomes the bf16 value n - 8) against the bf16 activations as given, a
+ * fresh fp32 accumulator per 64-weight group multiplied by its scale.  The
+ * reduction over Kd is split into slices when N alone gives too few 32-row
+ * work items to fill the GPU; each slice's partial sums go to the workspace
+ * and the last slice of an output tile to finish (a ticket counter) adds them
+ * in a fixed order and writes the tile, so results are deterministic.
  * ws, ws_bytes: at least the matching *_workspace_bytes() bytes, 256-byte
- * aligned.  Errors: MTPV_ERR_INVALID_ARG, MTPV_ERR_WORKSPACE, MTPV_ERR_CUDA.
+ * aligned; need not be initialised.  Errors: MTPV_ERR_INVALID_ARG,
+ * MTPV_ERR_WORKSPACE, MTPV_ERR_CUDA.
  * ---------------------------------------------------------------------- */
 MTPV_API size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N);
 MTPV_API mtpv_status mtpv_int4_proj(const void *x, int M, int Kd, int N, const void *wq,
@@ -257,7 +272,9 @@ MTPV_API mtpv_status mtpv_int4_gate_up(const void *x, int M, int Kd, int F, cons
  *   ws, ws_bytes   workspace of at least mtpv_verify_workspace_bytes(B, K, V)
  *                  bytes, 256-byte aligned.  It need not be initialised: the
  *                  call's first kernel clears what it needs.
- * Arithmetic: exp, sums, ratios and CDFs in fp64 on fp32 logits.
+ * Arithmetic: exp, sums, ratios and CDFs in fp64 on fp32 logits, every sum
+ * in a fixed order (no floating-point atomics), so a call's outputs are the
+ * same bits in every run.
  * Launch: two kernels, each launched as a programmatic dependent of the work
  * before it on `stream` (it may be scheduled while that work drains and
  * waits for its completion before reading its results).

@@ -191,3 +191,40 @@ def test_depth_sweep_cell(heads, k, t, sigma):
     rate = float((acc * np.arange(k + 1)).sum()) / (trials * k)
     print(f"\nK={k} T={t} sigma={sigma}: {trials} steps, {flagged} flagged, acceptance {rate:.3f}")
     assert flagged <= 1
+
+
+def test_large_vocab_batched_step():
+    """Eight sequences at vocabulary 248320 (hidden 5120, K = 3): 32 target
+    rows through the bf16 head and 24 draft rows through the int4 head, both
+    on the tensor-memory kernels (one pass over the weights), then the
+    sampler.  Logits on a strided sample of vocabulary rows against the
+    oracle's fp64 projection; tokens and accept counts against the oracle
+    run on the step's own logits."""
+    B, k, V8 = 8, 3, 248320
+    W = synth.make_head(V8, H, WSTD, seed=4242, device="cuda")
+    Wq, S = synth.quantize_int4_g64(W)
+    Ht, Hd = synth.make_hidden(B, k, H, SIGMA, seed=77, device="cuda")
+    u = synth.step_uniforms(77, 0, B, k)
+    dl0 = torch.empty((B * k, V8), dtype=torch.float32, device="cuda")
+    mtpv.lm_head_smallm(Hd, Wq, S, mtpv.W_INT4_G64, dl0)
+    d = torch.empty((B * k,), dtype=torch.int32, device="cuda")
+    mtpv.sample(dl0, T, TOP_P, torch.as_tensor(u["u_draft"].reshape(-1)).cuda(), d)
+    tl = torch.empty((B, k + 1, V8), dtype=torch.float32, device="cuda")
+    dl = torch.empty((B, k, V8), dtype=torch.float32, device="cuda")
+    ot = torch.full((B, k + 1), -9, dtype=torch.int32, device="cuda")
+    oa = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    rs = torch.full((B,), -9, dtype=torch.int32, device="cuda")
+    mtpv.verify_step(W, Wq, S, Ht, Hd, d.view(B, k), torch.as_tensor(u["u_accept"]).cuda(),
+                     torch.as_tensor(u["u_sample"]).cuda(), B, k, T, TOP_P, ot, oa, rs, tl, dl)
+    torch.cuda.synchronize()
+    assert torch.equal(dl.view(B * k, V8), dl0)  # the step's draft logits are the draft phase's
+    rows = np.unique(np.concatenate([np.arange(0, V8, 89), np.arange(V8 - 200, V8)]))
+    ridx = torch.as_tensor(rows).cuda()
+    ref_t = oracle.lm_head_bf16(synth.bf16_bits(Ht.cpu()), synth.bf16_bits(W[ridx].cpu()), threads=8)
+    ref_d = oracle.lm_head_int4g64(synth.bf16_bits(Hd.cpu()), Wq[ridx].cpu().numpy(),
+                                   synth.bf16_bits(S[ridx].cpu()), threads=8)
+    assert_logits_close(tl.view(B * (k + 1), V8)[:, ridx].cpu().numpy(), ref_t)
+    assert_logits_close(dl.view(B * k, V8)[:, ridx].cpu().numpy(), ref_d)
+    n, f, h = oracle_check(tl.cpu().numpy(), dl.cpu().numpy(), d.view(B, k).cpu().numpy(), u,
+                           ot.cpu().numpy(), oa.cpu().numpy(), rs.cpu().numpy())
+    assert n == B and f <= 1
