@@ -205,7 +205,8 @@ MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, fl
  *
  *   x       device bf16 [M, Kd] (16-byte aligned), 1 <= M <= 64.
  *   wq      device uint8 [N, Kd/2] (N = 2F for gate_up), MTPV_W_INT4_G64
- *           nibble order; scales device bf16 [N, Kd/64].
+ *           nibble order; scales device bf16 [N, Kd/64]; both 16-byte
+ *           aligned.
  *   Kd      a positive multiple of 64, at most 2^20.  One launch per pass of
  *           up to 8 rows (one MMA n-tile); the weights are read once per
  *           pass.
@@ -213,13 +214,21 @@ MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, fl
  * Arithmetic: bf16 mma.sync of exactly dequantised weights (the nibble n
  * becomes the bf16 value n - 8) against the bf16 activations as given, a
  * fresh fp32 accumulator per 64-weight group multiplied by its scale.  The
- * reduction over Kd is split into slices when N alone gives too few 32-row
- * work items to fill the GPU; each slice's partial sums go to the workspace
- * and the last slice of an output tile to finish (a ticket counter) adds them
- * in a fixed order and writes the tile, so results are deterministic.
+ * weights stream through shared memory (TMA) in stages of 128 rows x 8
+ * groups, and the list of stages is cut into one equal run per SM, so a
+ * 128-row output tile may be split between neighbouring SMs; each of them
+ * stores its partial sums in the workspace and the last to finish (a ticket
+ * counter) adds them in SM order and writes the tile.  The summation order
+ * depends only on the shapes and the GPU's SM count: results are
+ * deterministic on a given GPU.
  * ws, ws_bytes: at least the matching *_workspace_bytes() bytes, 256-byte
- * aligned; need not be initialised.  Errors: MTPV_ERR_INVALID_ARG,
- * MTPV_ERR_WORKSPACE, MTPV_ERR_CUDA.
+ * aligned, zero-filled before the first call that uses it; every call
+ * returns its ticket counters to zero, so one zeroing serves all later calls
+ * on the same stream (calls that share a workspace must not run
+ * concurrently).  The first 4 bytes are an error word: a bounded wait that
+ * gave up ORs a nonzero code into it and that launch's outputs are not
+ * valid; it stays set until the caller clears it.  Errors:
+ * MTPV_ERR_INVALID_ARG, MTPV_ERR_WORKSPACE, MTPV_ERR_CUDA.
  * ---------------------------------------------------------------------- */
 MTPV_API size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N);
 MTPV_API mtpv_status mtpv_int4_proj(const void *x, int M, int Kd, int N, const void *wq,

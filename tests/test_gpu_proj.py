@@ -89,3 +89,57 @@ def test_many_rows_take_several_passes():
     ref = oracle.lm_head_int4g64(synth.bf16_bits(x.cpu()), Wq[cols].cpu().numpy(),
                                  synth.bf16_bits(S[cols].cpu()), threads=8)
     assert_logits_close(y[:, cols].cpu().numpy(), ref)
+
+
+# Ragged shapes: a single group, a stage with one valid group (Kd = 576),
+# scale rows that straddle 16-byte chunks (Kd / 64 not a multiple of 8),
+# N not a multiple of the 128-row tile, fewer stages than SMs.
+RAGGED = [(1, 64, 1), (3, 576, 200), (8, 11008, 1000), (5, 192, 129), (2, 1088, 7168), (7, 5120, 130)]
+
+
+@pytest.mark.parametrize("M,Kd,N", RAGGED)
+def test_ragged_projection_against_oracle(M, Kd, N):
+    Wq, S = head(N, Kd, 31)
+    x = hidden(M, Kd, 400 + M)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    ws = mtpv.workspace(mtpv.load().mtpv_int4_proj_workspace_bytes(M, Kd, N))
+    mtpv.int4_proj(x, Wq, S, y, ws=ws)
+    torch.cuda.synchronize()
+    ref = oracle.lm_head_int4g64(synth.bf16_bits(x.cpu()), Wq.cpu().numpy(), synth.bf16_bits(S.cpu()), threads=8)
+    assert_logits_close(y.cpu().numpy(), ref)
+    # the error word is clear and every ticket counter is back at zero
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    tiles = (N + 127) // 128
+    assert not ws[256:256 + 4 * tiles].any()
+
+
+@pytest.mark.parametrize("M,Kd,F", [(1, 64, 1), (4, 576, 1001), (8, 192, 37), (3, 11008, 300)])
+def test_ragged_gate_up_against_oracle(M, Kd, F):
+    Wq, S = head(2 * F, Kd, 32)
+    x = hidden(M, Kd, 500 + M)
+    h = torch.full((M, F), float("nan"), device="cuda")
+    ws = mtpv.workspace(mtpv.load().mtpv_int4_gate_up_workspace_bytes(M, Kd, F))
+    mtpv.int4_gate_up(x, Wq, S, h, ws=ws)
+    torch.cuda.synchronize()
+    ref = oracle.gate_up_int4g64(synth.bf16_bits(x.cpu()), Wq.cpu().numpy(), synth.bf16_bits(S.cpu()), F,
+                                 threads=8)
+    assert_logits_close(h.cpu().numpy(), ref)
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    assert not ws[256:256 + 4 * ((F + 63) // 64)].any()
+
+
+def test_one_workspace_serves_successive_shapes():
+    # the counters a call leaves at zero are what the next call needs
+    shapes = [(3, 5120, 7168), (1, 17408, 5120), (8, 576, 200), (3, 5120, 7168)]
+    need = max(mtpv.load().mtpv_int4_proj_workspace_bytes(M, Kd, N) for M, Kd, N in shapes)
+    shared = mtpv.workspace(need)
+    for M, Kd, N in shapes:
+        Wq, S = head(N, Kd, 33)
+        x = hidden(M, Kd, 600 + M)
+        a = torch.empty((M, N), device="cuda")
+        b = torch.empty((M, N), device="cuda")
+        mtpv.int4_proj(x, Wq, S, a, ws=shared)
+        mtpv.int4_proj(x, Wq, S, b)
+        torch.cuda.synchronize()
+        assert torch.equal(a, b)
+    assert int(shared[:4].view(torch.int32).item()) == 0

@@ -132,8 +132,9 @@ def verify_step_host_workspace_bytes(B: int, K: int, V: int, h: int) -> int:
 
 
 def workspace(nbytes: int, device=None) -> torch.Tensor:
-    """A device byte buffer of at least ``nbytes`` (256-byte aligned)."""
-    return torch.empty(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
+    """A zero-filled device byte buffer of at least ``nbytes`` (256-byte
+    aligned); the projections' workspaces must start zeroed."""
+    return torch.zeros(max(int(nbytes), 1), dtype=torch.uint8, device=device or "cuda")
 
 
 # ---------------------------------------------------------------------------

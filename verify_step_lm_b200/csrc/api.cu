@@ -211,18 +211,21 @@ mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, float *yt, 
     return cuda_status(launch_heads(xt, Mt, w, yt, xd, Md, wq, scales, yd, Kd, N, ws, (cudaStream_t)stream));
 }
 
-size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N) {
+static size_t int4_proj_ws(int M, int Kd, int N, bool gate_up) {
     if (M < 1 || M > 64 || Kd < 64 || Kd % 64 || Kd > (1 << 20) || N < 1 || N > (1 << 28)) return 0;
-    return mtpv::int4_proj_workspace_bytes(M, Kd, N);
+    if (gate_up && N % 2) return 0;
+    return mtpv::int4_proj_workspace_bytes(M, Kd, N, gate_up);
 }
+
+size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N) { return int4_proj_ws(M, Kd, N, false); }
 
 static mtpv_status int4_proj_common(const void *x, int M, int Kd, int N, const void *wq,
                                     const void *scales, float *y, int ldy, bool silu_mul, void *ws,
                                     size_t ws_bytes, mtpv_stream stream) {
     if (!x || !wq || !scales || !y) return MTPV_ERR_INVALID_ARG;
-    const size_t need = mtpv_int4_proj_workspace_bytes(M, Kd, N);
+    const size_t need = int4_proj_ws(M, Kd, N, silu_mul);
     if (need == 0) return MTPV_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(scales, 2) || !aligned(y, 4))
+    if (!aligned(x, 16) || !aligned(wq, 16) || !aligned(scales, 16) || !aligned(y, 4))
         return MTPV_ERR_INVALID_ARG;
     if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return MTPV_ERR_WORKSPACE;
     return cuda_status(
@@ -235,14 +238,14 @@ mtpv_status mtpv_int4_proj(const void *x, int M, int Kd, int N, const void *wq, 
 }
 
 size_t mtpv_int4_gate_up_workspace_bytes(int M, int Kd, int F) {
-    if (F < 1 || F > (1 << 28)) return 0;
-    return mtpv_int4_proj_workspace_bytes(M, Kd, 2 * F);
+    if (F < 1 || F > (1 << 27)) return 0;
+    return int4_proj_ws(M, Kd, 2 * F, true);
 }
 
 mtpv_status mtpv_int4_gate_up(const void *x, int M, int Kd, int F, const void *wq,
                               const void *scales, float *h, void *ws, size_t ws_bytes,
                               mtpv_stream stream) {
-    if (F < 1 || F > (1 << 28)) return MTPV_ERR_INVALID_ARG;
+    if (F < 1 || F > (1 << 27)) return MTPV_ERR_INVALID_ARG;
     return int4_proj_common(x, M, Kd, 2 * F, wq, scales, h, F, true, ws, ws_bytes, stream);
 }
 

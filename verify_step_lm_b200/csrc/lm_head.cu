@@ -330,36 +330,6 @@ __device__ __forceinline__ void int4_f16_stage_x(uint16_t *xb, float *xs, unsign
     __syncthreads();
 }
 
-// The same staging for the split-K projection, once per call into global
-// memory: one CTA per activation row (row blockIdx.x); xs entries of rows
-// past M are zeroed by CTA 0.
-__global__ void __launch_bounds__(kGemvThreads) int4_f16_stage_rows_kernel(
-    const uint16_t *__restrict__ x, int M, int Kd, uint16_t *__restrict__ xb, float *__restrict__ xs,
-    float *__restrict__ row_unscale) {
-    __shared__ unsigned int s_amax;
-    const int m = blockIdx.x;
-    const int Gt = Kd >> 6;
-    const int rowc = Gt * 8 + 1;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-    if (threadIdx.x == 0) s_amax = 0u;
-    __syncthreads();
-    const uint32_t a = int4_row_absmax_warp(x + (size_t)m * Kd, Kd);
-    if (lane == 0 && a) atomicMax(&s_amax, a);
-    __syncthreads();
-    const int sh = int4_row_shift(s_amax);
-    if (threadIdx.x == 0) row_unscale[m] = __uint_as_float((uint32_t)(127 + sh) << 23);
-    uint16_t *dst = xb + (size_t)m * rowc * 8;
-    int4_row_convert(x + (size_t)m * Kd, Kd, sh, dst);
-    __syncthreads();
-    for (int G = warp; G < Gt; G += nw) {
-        const float v = int4_group_offset(dst, G);
-        if (lane == 0) xs[G * 8 + m] = v;
-    }
-    if (m == 0)
-        for (int i = threadIdx.x; i < Gt * 8; i += blockDim.x)
-            if ((i & 7) >= M) xs[i] = 0.0f;
-}
-
 // The 16-row tiles of warp gw of nw warps (grid-wide numbering), streamed
 // through the warp's own ring at `ring`.
 template <int GPS, int NST>
@@ -514,12 +484,10 @@ __global__ void __launch_bounds__(NT) lm_head_int4_f16_kernel(
 // Direct-load form of the fp16 int4 kernel: each lane loads its nibbles
 // straight into registers (8 bytes per row and group) and computes exactly as
 // the ring kernel does (same MMA operands, order and epilogue), so both forms
-// give the same bits.  Used where the ring does not fit and, over slices of
-// the reduction, by the split-K projection kernel.
+// give the same bits.  Used where the ring does not fit.
 // ---------------------------------------------------------------------------
 // Groups [gbeg, gend) of the RB tiles of task `task`, scaled back by the
-// rows' power-of-two factors and stored to y (partial sums when the range
-// is a slice of the reduction).
+// rows' power-of-two factors and stored to y.
 template <int RB, int UI>
 __device__ __forceinline__ void int4_f16_direct_task(const uint4 *xstage, const float *xs,
                                                      const float *row_unscale, int M, int Kd, int N,
@@ -639,56 +607,6 @@ __global__ void __launch_bounds__(kGemvThreads) lm_head_int4_f16_direct_kernel(
     const int tasks = ((N + 15) / 16 + RB - 1) / RB;
     for (int task = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); task < tasks; task += gridDim.x * kGemvWarps)
         int4_f16_direct_task<RB, UI>(smem_dir, xs, row_unscale, M, Kd, N, Wq, S, y, ldy, task, 0, Kd >> 6);
-}
-
-// ---------------------------------------------------------------------------
-// Split-K int4 projection for decoder layers (few output rows per tile, long
-// reductions: N of a few thousand gives too few 16-row tiles to fill 148
-// SMs).  The activations are staged once per call into global memory (one
-// CTA per row), where every work item reads its fragments through the
-// caches; a work item is one task (RB tiles) over one slice of the 64-weight
-// groups; its partial sums go to part[slice][M][N], and a third kernel adds
-// the slices in a fixed order (deterministic), optionally applying the SiLU
-// gate of a gate||up projection.
-// ---------------------------------------------------------------------------
-template <int RB, int UI>
-__global__ void __launch_bounds__(kGemvThreads) lm_head_int4_splitk_kernel(
-    const uint4 *__restrict__ xstage, const float *__restrict__ xs, const float *__restrict__ unscale,
-    int M, int Kd, int N, const uint8_t *__restrict__ Wq, const uint16_t *__restrict__ S,
-    float *__restrict__ part, int slices, int gps) {
-    const int Gt = Kd >> 6;
-    const int tasks = ((N + 15) / 16 + RB - 1) / RB;
-    const int items = tasks * slices;
-    for (int item = blockIdx.x * kGemvWarps + (threadIdx.x >> 5); item < items;
-         item += gridDim.x * kGemvWarps) {
-        const int task = item / slices, sl = item - task * slices;
-        const int gbeg = sl * gps, gend = min(Gt, gbeg + gps);
-        int4_f16_direct_task<RB, UI>(xstage, xs, unscale, M, Kd, N, Wq, S, part + (size_t)sl * M * N, N,
-                                     task, gbeg, gend);
-    }
-}
-
-// y[m][j] = sum over slices of part[s][m][j] (s in order); with silu_mul the
-// N columns are a gate half and an up half and y[m][j] = silu(g) * u for
-// j < N/2, g = column j, u = column j + N/2, silu(g) = g / (1 + e^-g).
-__global__ void __launch_bounds__(kGemvThreads) splitk_reduce_kernel(const float *__restrict__ part,
-                                                                     int slices, int M, int N,
-                                                                     float *__restrict__ y, int ldy,
-                                                                     int silu_mul) {
-    const int cols = silu_mul ? N / 2 : N;
-    const size_t plane = (size_t)M * N;
-    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < M * cols; i += gridDim.x * blockDim.x) {
-        const int m = i / cols, j = i - m * cols;
-        const float *p = part + (size_t)m * N + j;
-        float a = 0.0f;
-        for (int sl = 0; sl < slices; ++sl) a += p[sl * plane];
-        if (silu_mul) {
-            float b = 0.0f;
-            for (int sl = 0; sl < slices; ++sl) b += p[sl * plane + cols];
-            a = a / (1.0f + expf(-a)) * b;
-        }
-        y[(size_t)m * ldy + j] = a;
-    }
 }
 
 constexpr int kMixWarps = 16;      // per CTA, one CTA per SM
@@ -836,81 +754,6 @@ cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *y
         static_cast<const uint16_t *>(xd), Md, static_cast<const uint8_t *>(wq),
         static_cast<const uint16_t *>(scales), yd, Kd, N, wk);
     return cudaGetLastError();
-}
-
-// ---- split-K projection ----------------------------------------------------
-constexpr int kSplitRB = 2, kSplitUI = 4, kSplitRows = 8;  // rows per pass: one MMA n-tile
-
-// Slices of the reduction for a pass over N outputs: enough items to give
-// every warp of the GPU about two, at least kSplitUI groups per slice (the
-// current device's SM count; 148 if it cannot be read).
-static void splitk_plan(int Kd, int N, int *slices, int *gps) {
-    const int Gt = Kd / 64;
-    const int tasks = ((N + 15) / 16 + kSplitRB - 1) / kSplitRB;
-    const int nsm = current_device_sms() > 0 ? current_device_sms() : 148;
-    int sl = (2 * nsm * kGemvWarps + tasks - 1) / tasks;
-    sl = std::max(1, std::min({sl, 16, std::max(1, Gt / kSplitUI)}));
-    const int g = (Gt + sl - 1) / sl;
-    *gps = g;
-    *slices = (Gt + g - 1) / g;
-}
-
-// Workspace: [staged activations: kSplitRows x rowc x 16 B][offset sums: Gt x
-// 8 fp32][row scales: 8 fp32][partial sums: slices x rows x N fp32]
-struct SplitWs {
-    size_t xb, xs, us, part, total;
-};
-static SplitWs splitk_layout(int M, int Kd, int N) {
-    const size_t Gt = (size_t)Kd / 64, rowc = Gt * 8 + 1;
-    int slices, gps;
-    splitk_plan(Kd, N, &slices, &gps);
-    auto up = [](size_t n) { return (n + 255) / 256 * 256; };
-    SplitWs l;
-    l.xb = 0;
-    l.xs = l.xb + up((size_t)kSplitRows * rowc * 16);
-    l.us = l.xs + up(Gt * 8 * sizeof(float));
-    l.part = l.us + up(8 * sizeof(float));
-    l.total = l.part + up((size_t)slices * std::min(M, kSplitRows) * N * sizeof(float));
-    return l;
-}
-
-size_t int4_proj_workspace_bytes(int M, int Kd, int N) { return splitk_layout(M, Kd, N).total; }
-
-cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq, const void *scales,
-                             float *y, int ldy, bool silu_mul, void *ws, cudaStream_t s) {
-    int slices, gps;
-    splitk_plan(Kd, N, &slices, &gps);
-    const SplitWs l = splitk_layout(M, Kd, N);
-    char *w = static_cast<char *>(ws);
-    uint16_t *xb = reinterpret_cast<uint16_t *>(w + l.xb);
-    float *xs = reinterpret_cast<float *>(w + l.xs);
-    float *us = reinterpret_cast<float *>(w + l.us);
-    float *part = reinterpret_cast<float *>(w + l.part);
-    auto k = lm_head_int4_splitk_kernel<kSplitRB, kSplitUI>;
-    const uint16_t *x16 = static_cast<const uint16_t *>(x);
-    for (int m0 = 0; m0 < M; m0 += kSplitRows) {
-        const int mm = std::min(kSplitRows, M - m0);
-        int4_f16_stage_rows_kernel<<<mm, kGemvThreads, 0, s>>>(x16 + (size_t)m0 * Kd, mm, Kd, xb, xs, us);
-        cudaError_t e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-        int occ = 0, sms = 0;
-        e = kernel_setup((const void *)k, kGemvThreads, 0, &occ, &sms);
-        if (e != cudaSuccess) return e;
-        const int tasks = ((N + 15) / 16 + kSplitRB - 1) / kSplitRB;
-        const int need = (tasks * slices + kGemvWarps - 1) / kGemvWarps;
-        k<<<std::min(need, sms * occ), kGemvThreads, 0, s>>>(
-            reinterpret_cast<const uint4 *>(xb), xs, us, mm, Kd, N, static_cast<const uint8_t *>(wq),
-            static_cast<const uint16_t *>(scales), part, slices, gps);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-        const int cols = silu_mul ? N / 2 : N;
-        const int blocks = std::min(sms * 4, (mm * cols + kGemvThreads - 1) / kGemvThreads);
-        splitk_reduce_kernel<<<blocks, kGemvThreads, 0, s>>>(part, slices, mm, N, y + (size_t)m0 * ldy,
-                                                            ldy, silu_mul ? 1 : 0);
-        e = cudaGetLastError();
-        if (e != cudaSuccess) return e;
-    }
-    return cudaSuccess;
 }
 
 size_t lm_head_max_smem_rows(int Kd) {

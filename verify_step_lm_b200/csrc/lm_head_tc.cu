@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "lm_head_tc.cuh"
+#include "tma.cuh"
 
 namespace mtpv {
 
@@ -44,7 +45,6 @@ constexpr int kTcK = 64;                     // reduction elements per stage: on
 constexpr int kTcABytes = kTcRows * kTcK * 2;  // 16 KB per stage
 constexpr int kTcMaxN = 64;                  // activation rows (the MMA's N), padded to 16
 constexpr int kTcBBytesMax = kTcMaxN * kTcK * 2;
-constexpr int kTcWaitLimit = 1 << 20;        // polls of one mbarrier wait before it gives up
 // Partial accumulators per tile: a stage's consecutive 16-element MMAs write
 // different ones, so they need not wait for each other (at these small N a
 // chain of MMAs into one accumulator runs at ~110 ns per MMA on B200); the
@@ -54,37 +54,6 @@ constexpr int kTcParts = 4;
 // ---------------------------------------------------------------------------
 // PTX wrappers
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint32_t su32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void bar_init(uint64_t *b, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count) : "memory");
-}
-__device__ __forceinline__ void bar_arrive_expect(uint64_t *b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void bar_arrive(uint64_t *b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
-}
-// Waits until the barrier's phase with the given parity has completed; false
-// if it gave up after kTcWaitLimit polls.
-__device__ __forceinline__ bool bar_wait(uint64_t *b, uint32_t parity) {
-    for (int i = 0; i < kTcWaitLimit; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-            : "=r"(done)
-            : "r"(su32(b)), "r"(parity)
-            : "memory");
-        if (done) return true;
-    }
-    return false;
-}
-__device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, int x, int y, uint64_t *b) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        ::"r"(su32(dst)), "l"(map), "r"(x), "r"(y), "r"(su32(b))
-        : "memory");
-}
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 // Shared-memory matrix descriptor of a K-major tile with 128-byte rows and the
@@ -668,8 +637,10 @@ cudaError_t encode_fn(PFN_cuTensorMapEncodeTiled_v12000 *fn) {
     return g_encode ? cudaSuccess : cudaErrorNotSupported;
 }
 
-// 2-D tensor map of a row-major [rows, cols] matrix (elem_bytes per element),
-// box of box_cols x box_rows, zero fill out of bounds.
+size_t tc_smem_bytes() { return 1024 + (size_t)kTcStages * (kTcABytes + kTcBBytesMax) + sizeof(TcCtl); }
+
+}  // namespace
+
 cudaError_t map_2d(CUtensorMap *m, const void *ptr, CUtensorMapDataType type, int elem_bytes, int cols,
                    int rows, int box_cols, int box_rows, CUtensorMapSwizzle swizzle) {
     PFN_cuTensorMapEncodeTiled_v12000 enc;
@@ -684,10 +655,6 @@ cudaError_t map_2d(CUtensorMap *m, const void *ptr, CUtensorMapDataType type, in
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
-
-size_t tc_smem_bytes() { return 1024 + (size_t)kTcStages * (kTcABytes + kTcBBytesMax) + sizeof(TcCtl); }
-
-}  // namespace
 
 size_t t4_smem_bytes(int Kd) {
     const size_t sbytes = (size_t)kTcRows * (Kd / 64) * 2;
