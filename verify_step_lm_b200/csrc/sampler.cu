@@ -69,7 +69,7 @@ constexpr int kCandCap = 4096;
 constexpr int kCacheFloats = 9728;  // logits slice kept in shared memory (38 KB), and its exps
 constexpr int kBatch = 8;           // loads in flight per thread in streaming loops
 constexpr int kExpTab = 64;         // entries of the exp table (2^(j/64))
-constexpr int kMaxCluster = 16;     // CTAs per cluster (16, or 8 where 16 cannot be resident)
+constexpr int kMaxCluster = 16;     // CTAs per cluster at most (a power of two; see cluster_size_for)
 
 // Dynamic shared memory of the statistics kernel: a region reused phase by
 // phase, then the small bookkeeping struct.
@@ -86,8 +86,8 @@ constexpr int kDrawBufDoubles = 19456;  // the draw kernel's weight buffer (152 
 constexpr size_t kDrawBufBytes = kDrawBufDoubles * sizeof(double);
 
 struct SamplerSmem {
-    double own_mass[kBins / 8];  // bins owned by this CTA (C >= 8), or radix digits
-    int own_cnt[kBins / 8];
+    double own_mass[256];  // radix select: mass per digit
+    int own_cnt[256];
     double rad_mass[256];
     int rad_cnt[256];
     double red_d[kWarps];
@@ -114,6 +114,7 @@ struct SamplerSmem {
     float cut_l;
     int res_acc;  // draw kernel, CTA 0: the position's acceptance
     unsigned long long bar;  // mbarrier of the bulk copies
+    int wait_ok;             // thread 0's verdict on a bulk copy, for the block
     double exp_tab[kExpTab];  // 2^(j/64), for exp_neg
 };
 
@@ -267,6 +268,20 @@ __device__ __forceinline__ bool mbar_wait(unsigned long long *bar, unsigned phas
         if (done) return true;
     }
     return false;
+}
+// The block's wait for a bulk copy: thread 0 polls (bounded by limit; when
+// that gives up, a second bound of kWaitLimit for the copy in flight) and the
+// block learns the outcome at the barrier, which also orders every thread's
+// reads of the copied data after thread 0 saw the copy complete.  One poller
+// instead of 512 keeps the polling off the barrier the copy completes on.
+__device__ __forceinline__ bool mbar_wait_block(unsigned long long *bar, unsigned phase, int limit, int *flag) {
+    if (threadIdx.x == 0) {
+        const bool ok = mbar_wait(bar, phase, limit);
+        if (!ok) mbar_wait(bar, phase, kWaitLimit);
+        *flag = ok ? 1 : 0;
+    }
+    __syncthreads();
+    return *(volatile int *)flag != 0;
 }
 __device__ __forceinline__ bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 // Shared -> global: the writing threads fence their generic stores into the
@@ -511,9 +526,7 @@ __device__ int cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double *
             bulk_load(wbuf, src.Et + v0, bytes, &s.bar);
             if (src.kind == 1) bulk_load(wbuf + n, src.Ed + v0, bytes, &s.bar);
         }
-        __syncthreads();  // the barrier is initialised before anyone polls it
-        landed = mbar_wait(&s.bar, 0, wait_polls);
-        if (!landed) mbar_wait(&s.bar, 0, kWaitLimit);  // give the copies in flight a second bound
+        landed = mbar_wait_block(&s.bar, 0, wait_polls, &s.wait_ok);
     }
     // Otherwise weights are computed once, coalesced, into shared memory;
     // thread t's sub-chunk lives at wbuf[t * P ..] with an odd stride P (no
@@ -671,11 +684,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 mbar_expect(&s.bar, (unsigned)n * 4u);
                 bulk_load(cache, L + v0, (unsigned)n * 4u, &s.bar);
             }
-            __syncthreads();  // the barrier is initialised before anyone polls it
-            if (!mbar_wait(&s.bar, 0, p.wait_polls)) {
-                bad = 2;                             // the row is reported as timed out
-                mbar_wait(&s.bar, 0, kWaitLimit);    // a second bound for the copy in flight
-            }
+            if (!mbar_wait_block(&s.bar, 0, p.wait_polls, &s.wait_ok)) bad = 2;  // reported as timed out
         }
         for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
             float lv[kBatch];
@@ -814,6 +823,10 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
             // ---------------- P3: crossing bin, exact cut ----------------
             const double thr = __dmul_rn((double)p.top_p, st.Z);
             const int base = rank * per;
+            // masses of the bins this CTA owns (kBins / C of them), in the
+            // histogram's region: its counts went to their owners before the
+            // cluster barrier above, so the region is free
+            double *own = rg.hist_mass;
             // the cluster's histogram on the bins this CTA owns: the C copies'
             // integer sums, turned into an approximate mass
             // e_lo (count + excess eps / qmax), e_lo = exp(-(b + 1) xw)
@@ -828,14 +841,14 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                         ex += v.y;
                     }
                     const double elo = exp_neg(-(double)(base + b + 1) * (double)xw, s.exp_tab);
-                    s.own_mass[b] = elo * ((double)cn + (double)ex * kex);
+                    own[b] = elo * ((double)cn + (double)ex * kex);
                 }
             }
             __syncthreads();
             if (wid == 0) {
                 int f;
                 double bef;
-                const double t = warp_prefix_search(s.own_mass, per, 0.0, 0.0, false, &f, &bef);
+                const double t = warp_prefix_search(own, per, 0.0, 0.0, false, &f, &bef);
                 publish(cluster, s.all_rt, rank, C, t);
             }
             cluster.sync();
@@ -853,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 if (cstar == rank) {
                     int f;
                     double bef;
-                    warp_prefix_search(s.own_mass, per, Pstar, thr, true, &f, &bef);
+                    warp_prefix_search(own, per, Pstar, thr, true, &f, &bef);
                     if (f < 0) f = per - 1;  // not reachable: the range total reached thr
                     bstar = base + f;
                 } else if (cstar < 0 && rank == 0) {
@@ -1272,44 +1285,55 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
 // ---------------------------------------------------------------------------
 namespace {
 
-// Cluster size of each sampler kernel per device (16 when a 16-CTA cluster
-// can be resident, else 8), found once; 0 = not yet known.
-int g_cluster_size[2][64];
+// Cluster size of a sampler launch: the largest power of two up to 16 that
+// can be resident on the device (the occupancy calculator is asked once per
+// kernel and device).  The kernels work with any power of two from 1 to 16,
+// but smaller clusters only pay at many rows if a CTA's slice still fits its
+// shared-memory cache: past it every pass re-reads the row from L2, which on
+// B200 cost more than the waves of 16-CTA clusters it saves (measured: 8
+// sequences x 3 drafts at vocabulary 248320, 459 us with 16-CTA clusters in
+// waves, 581 us with 2-CTA clusters in one wave).
+int g_max_active[2][64][5];  // [kernel][device][log2 C]: clusters resident at once; -1 = cannot launch
+bool g_known[2][64];
 std::mutex g_cluster_mu;
 
 template <typename Kern>
-int cluster_size_for(int which, Kern kernel, size_t smem) {
+int cluster_size_for(int which, Kern kernel, size_t smem, int units) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
         cudaGetLastError();
         return 8;
     }
     std::lock_guard<std::mutex> lock(g_cluster_mu);
-    if (g_cluster_size[which][dev]) return g_cluster_size[which][dev];
-    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-    int best = 8;
-    for (int c : {16, 8}) {
-        cudaLaunchConfig_t cfg = {};
-        cfg.gridDim = dim3(c, 1, 1);
-        cfg.blockDim = dim3(kThreads, 1, 1);
-        cfg.dynamicSmemBytes = smem;
-        cudaLaunchAttribute at[1];
-        at[0].id = cudaLaunchAttributeClusterDimension;
-        at[0].val.clusterDim.x = c;
-        at[0].val.clusterDim.y = 1;
-        at[0].val.clusterDim.z = 1;
-        cfg.attrs = at;
-        cfg.numAttrs = 1;
-        int nclusters = 0;
-        if (cudaOccupancyMaxActiveClusters(&nclusters, kernel, &cfg) == cudaSuccess && nclusters > 0) {
-            best = c;
-            break;
+    if (!g_known[which][dev]) {
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        for (int lg = 0; lg < 5; ++lg) {
+            const int c = 1 << lg;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(c, 1, 1);
+            cfg.blockDim = dim3(kThreads, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeClusterDimension;
+            at[0].val.clusterDim.x = c;
+            at[0].val.clusterDim.y = 1;
+            at[0].val.clusterDim.z = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess || n <= 0) {
+                cudaGetLastError();
+                n = -1;
+            }
+            g_max_active[which][dev][lg] = n;
         }
-        cudaGetLastError();
+        g_known[which][dev] = true;
     }
-    g_cluster_size[which][dev] = best;
-    return best;
+    (void)units;
+    for (int lg = 4; lg >= 0; --lg)
+        if (g_max_active[which][dev][lg] > 0) return 1 << lg;
+    return 8;
 }
 
 // Both sampler kernels are launched as programmatic dependents of the work
@@ -1346,11 +1370,11 @@ cudaError_t launch_sampler(const SamplerParams &params, int rows, cudaStream_t s
     SamplerParams p = params;
     const int polls = g_wait_polls.load();
     p.wait_polls = polls < 0 ? kWaitLimit : polls;
-    const int C1 = cluster_size_for(0, sampler_stats_kernel, kStatsSmemBytes);
+    const int C1 = cluster_size_for(0, sampler_stats_kernel, kStatsSmemBytes, rows);
     cudaError_t e = launch_clusters(sampler_stats_kernel, C1, rows, kStatsSmemBytes, p, stream);
     if (e != cudaSuccess) return e;
-    const int C2 = cluster_size_for(1, sampler_draw_kernel, kDrawSmemBytes);
     const int clusters = p.verify ? p.B * (p.K + 1) : rows;
+    const int C2 = cluster_size_for(1, sampler_draw_kernel, kDrawSmemBytes, clusters);
     return launch_clusters(sampler_draw_kernel, C2, clusters, kDrawSmemBytes, p, stream);
 }
 
