@@ -211,9 +211,12 @@ struct Int4Ring {
 // (64 + n) x, and each group's offset term 72 x (1152 x / 16 per weight) is
 // removed with a precomputed sum: the offset is 72 weight steps, which keeps
 // the fp32 cancellation small (putting the nibble at bit 0 instead would make
-// it 1032 steps).  The activations are fp16, exact after a per-row
-// power-of-two scale that puts the row's largest |x| in [2^9, 2^10) before
-// the division by 16 (undone on the output).  Layouts as in the bf16 kernels.
+// it 1032 steps).  The activations are fp16 after a per-row power-of-two
+// scale that puts the row's largest |x| in [2^9, 2^10) before the division
+// by 16 (undone on the output): a bf16 value carries 8 significant bits, so
+// the fp16 copy is exact for every element down to 2^-23 of the row's largest
+// |x|; smaller ones fall among the fp16 subnormals, off by at most 2^-30 of
+// the row maximum (or flushed to zero).  Layouts as in the bf16 kernels.
 __device__ __forceinline__ void mma_f16_16816(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
     asm volatile(
         "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
