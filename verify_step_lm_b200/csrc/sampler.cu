@@ -284,17 +284,6 @@ __device__ __forceinline__ bool mbar_wait_block(unsigned long long *bar, unsigne
     return *(volatile int *)flag != 0;
 }
 __device__ __forceinline__ bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
-// Shared -> global: the writing threads fence their generic stores into the
-// async proxy and meet at a barrier first; one thread issues and waits.
-__device__ __forceinline__ void fence_to_async_proxy() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void bulk_store_wait(void *dst, const void *src, unsigned bytes) {
-    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_u32(src)),
-                 "r"(bytes)
-                 : "memory");
-    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-}
-
 // Warp-wide (max with its lowest index, min, or) of per-lane partials; every
 // lane ends with the result.
 __device__ __forceinline__ void warp_max_min_arg(float &mx, int &arg, float &mn, int &bad) {
@@ -939,8 +928,21 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                     const int n = (int)total;
                     const unsigned long long key = tid < n ? rg.cand[tid] : 0ull;
                     int r = 0;
-                    if (tid < n)
-                        for (int j = 0; j < n; ++j) r += rg.cand[j] > key ? 1 : 0;
+                    if (tid < n) {
+                        // 16-byte loads, four independent counts: the loop is
+                        // bound by shared-memory latency, not by the compares
+                        const ulonglong2 *c2 = reinterpret_cast<const ulonglong2 *>(rg.cand);
+                        int r0 = 0, r1 = 0, r2 = 0, r3 = 0, j = 0;
+                        for (; j + 4 <= n; j += 4) {
+                            const ulonglong2 a = c2[j >> 1], b = c2[(j >> 1) + 1];
+                            r0 += a.x > key ? 1 : 0;
+                            r1 += a.y > key ? 1 : 0;
+                            r2 += b.x > key ? 1 : 0;
+                            r3 += b.y > key ? 1 : 0;
+                        }
+                        for (; j < n; ++j) r0 += rg.cand[j] > key ? 1 : 0;
+                        r = (r0 + r1) + (r2 + r3);
+                    }
                     const double e = tid < n ? e_of(key_logit(key), md, invT, s.exp_tab) : 0.0;
                     __syncthreads();
                     if (tid < n) {
@@ -1111,15 +1113,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     if (rank == 0 && tid == 0) p.slots[row].st = st;
     if (erow && !bad && T > 0.0) {
         const double md = (double)m;
-        const int n = v1 - v0;
-        if (cached && n > 0 && (n & 1) == 0 && aligned16(erow + v0)) {
-            // masked in place, then one bulk copy of the slice
-            for (int j = v0 + tid; j < v1; j += kThreads)
-                if (!is_kept(st, rg.cache[j - v0], j)) rg.ecache[j - v0] = 0.0;
-            fence_to_async_proxy();
-            __syncthreads();
-            if (tid == 0) bulk_store_wait(erow + v0, rg.ecache, (unsigned)n * 8u);
-        } else if (cached) {
+        if (cached) {  // coalesced 8-byte stores; they drain after the CTA has moved on
             for (int j = v0 + tid; j < v1; j += kThreads)
                 erow[j] = is_kept(st, rg.cache[j - v0], j) ? rg.ecache[j - v0] : 0.0;
         } else {
@@ -1371,6 +1365,15 @@ cudaError_t launch_sampler(const SamplerParams &params, int rows, cudaStream_t s
     const int polls = g_wait_polls.load();
     p.wait_polls = polls < 0 ? kWaitLimit : polls;
     const int C1 = cluster_size_for(0, sampler_stats_kernel, kStatsSmemBytes, rows);
+    // The fp64 weight cache pays only while a CTA's slice (and its exps) stays
+    // in shared memory: then the statistics kernel writes the masked exps it
+    // already holds and the draw kernel bulk-loads them.  Past the slice
+    // cache the statistics kernel would recompute every kept token's exp to
+    // write it, and the draw kernel recomputing them from the logits was
+    // measured faster (8 sequences x 3 drafts at vocabulary 248320: 404 vs
+    // 453 us; at vocabulary 151936 and one sequence the cache wins, 39 vs
+    // 46 us).
+    if (p.ecache && (p.V + C1 - 1) / C1 > kCacheFloats) p.ecache = nullptr;
     cudaError_t e = launch_clusters(sampler_stats_kernel, C1, rows, kStatsSmemBytes, p, stream);
     if (e != cudaSuccess) return e;
     const int clusters = p.verify ? p.B * (p.K + 1) : rows;
