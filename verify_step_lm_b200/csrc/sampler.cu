@@ -654,7 +654,14 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     wait_for_producer();         // the logits
     if (p.verify && row == 0 && rank == 0)  // ticket counters of the draw kernel
         for (int k = tid; k < p.B; k += kThreads) p.counters[k] = 0u;
-    auto lval = [&](int j) -> float { return cached ? cache[j - v0] : L[j]; };
+    // A token's logit: from the slice cache when the slice fits it, else from
+    // global memory.  The source is chosen once: written as a per-element
+    // "cached ? cache[.] : L[.]", the compiler may issue both loads and
+    // select, paying an L2 round trip per batch even when every token is in
+    // shared memory.
+    const float *lsrc = cached ? cache : L;
+    const int loff = cached ? v0 : 0;
+    auto lval = [&](int j) -> float { return lsrc[j - loff]; };
 
     // ---------------- P1: read the slice; max, min, argmax, finiteness ----------------
     float g_m, g_min;
@@ -675,19 +682,38 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
             }
             if (!mbar_wait_block(&s.bar, 0, p.wait_polls, &s.wait_ok)) bad = 2;  // reported as timed out
         }
-        for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
+        if (bulk) {
+            // 16-byte shared loads of contiguous runs, each thread's tokens in
+            // ascending order (the first of equal maxima is kept; the warp
+            // reduction takes the lowest index)
+            const unsigned cbase = smem_u32(cache);
+            for (int i = tid; i < (n >> 2); i += kThreads) {
+                float e[4];
+                asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                             : "=f"(e[0]), "=f"(e[1]), "=f"(e[2]), "=f"(e[3])
+                             : "r"(cbase + 16u * (unsigned)i));
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const float l = e[k];
+                    if (!isfinite(l)) bad |= 1;
+                    if (l > mx) { mx = l; arg = v0 + 4 * i + k; }
+                    mn = fminf(mn, l);
+                }
+            }
+        }
+        for (int j0 = v0 + tid; !bulk && j0 < v1; j0 += kBatch * kThreads) {
             float lv[kBatch];
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
                 const int j = j0 + q * kThreads;
-                lv[q] = j < v1 ? (bulk ? cache[j - v0] : __ldg(L + j)) : 0.0f;
+                lv[q] = j < v1 ? __ldg(L + j) : 0.0f;
             }
 #pragma unroll
             for (int q = 0; q < kBatch; ++q) {
                 const int j = j0 + q * kThreads;
                 if (j < v1) {
                     const float l = lv[q];
-                    if (cached && !bulk) cache[j - v0] = l;
+                    if (cached) cache[j - v0] = l;
                     if (!isfinite(l)) bad |= 1;
                     if (l > mx) { mx = l; arg = j; }
                     mn = fminf(mn, l);
@@ -879,17 +905,36 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 if (tid == 0) s.local_n = 0u;
                 __syncthreads();
                 double a_loc = 0.0, m_loc = 0.0;
-                for (int j = v0 + tid; j < v1; j += kThreads) {
-                    const float l = lval(j);
-                    const int b = bin_of(l, m, inv_w);
-                    if (b <= bstar) {
-                        const double e = cached ? rg.ecache[j - v0] : e_of(l, md, invT, s.exp_tab);
-                        if (b < bstar) {
-                            a_loc = __dadd_rn(a_loc, e);
-                        } else {
-                            m_loc = __dadd_rn(m_loc, e);
-                            const unsigned slot = atomicAdd(&s.local_n, 1u);
-                            if (slot < (unsigned)kCandCap) stage[slot] = rank_key(l, j);
+                // each thread's tokens in ascending order (the sums' order);
+                // kBatch logits loaded before any is used, and the weight
+                // source chosen outside the loop (not per token)
+                auto take = [&](float l, int j, double e) {
+                    if (bin_of(l, m, inv_w) < bstar) {
+                        a_loc = __dadd_rn(a_loc, e);
+                    } else {
+                        m_loc = __dadd_rn(m_loc, e);
+                        const unsigned slot = atomicAdd(&s.local_n, 1u);
+                        if (slot < (unsigned)kCandCap) stage[slot] = rank_key(l, j);
+                    }
+                };
+                for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
+                    float lv[kBatch];
+#pragma unroll
+                    for (int q = 0; q < kBatch; ++q) {
+                        const int j = j0 + q * kThreads;
+                        lv[q] = j < v1 ? lval(j) : 0.0f;
+                    }
+                    if (cached) {
+#pragma unroll
+                        for (int q = 0; q < kBatch; ++q) {
+                            const int j = j0 + q * kThreads;
+                            if (j < v1 && bin_of(lv[q], m, inv_w) <= bstar) take(lv[q], j, rg.ecache[j - v0]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int q = 0; q < kBatch; ++q) {
+                            const int j = j0 + q * kThreads;
+                            if (j < v1 && bin_of(lv[q], m, inv_w) <= bstar) take(lv[q], j, e_of(lv[q], md, invT, s.exp_tab));
                         }
                     }
                 }
