@@ -82,6 +82,9 @@ constexpr size_t kOffCand = kOffHistMass + kBins * sizeof(double);
 constexpr size_t kOffCandE = kOffCand + kCandCap * sizeof(unsigned long long);
 constexpr size_t kRegionBytes = kOffCandE + kCandCap * sizeof(double);
 static_assert(kOffExp % 16 == 0 && kOffHistMass % 16 == 0, "region alignment");
+// A slice too long for its exps as well still keeps its logits in shared
+// memory, using the exps' room too (114 KB: 29184 floats).
+constexpr int kCacheFloatsLogits = (int)(kOffHistMass / sizeof(float));
 constexpr int kDrawBufDoubles = 19456;  // the draw kernel's weight buffer (152 KB: two rows' slices)
 constexpr size_t kDrawBufBytes = kDrawBufDoubles * sizeof(double);
 
@@ -643,7 +646,8 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     const int V = p.V;
     const int slice = (V + C - 1) / C;
     const int v0 = min(V, rank * slice), v1 = min(V, v0 + slice);
-    const bool cached = (v1 - v0) <= kCacheFloats;
+    const bool cached_e = (v1 - v0) <= kCacheFloats;        // logits and their exps in shared memory
+    const bool cached = (v1 - v0) <= kCacheFloatsLogits;    // logits in shared memory
     const float *L = row_ptr(p, row);
     const double T = (double)p.T;
     const double invT = T > 0.0 ? 1.0 / T : 0.0;
@@ -801,7 +805,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                 const int j = j0 + q * kThreads;
                 if (j < v1) {
                     zt += ev[q];
-                    if (cached) rg.ecache[j - v0] = ev[q];
+                    if (cached_e) rg.ecache[j - v0] = ev[q];
                     if (!topp_all) {
                         const int b = bin_of(lv[q], m, inv_w);
                         // excess exp(x) - 1 over the lower edge, x in [0, xw] (xw is
@@ -924,7 +928,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                         const int j = j0 + q * kThreads;
                         lv[q] = j < v1 ? lval(j) : 0.0f;
                     }
-                    if (cached) {
+                    if (cached_e) {
 #pragma unroll
                         for (int q = 0; q < kBatch; ++q) {
                             const int j = j0 + q * kThreads;
@@ -1105,7 +1109,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                             const unsigned long long key = rank_key(l, j);
                             if ((key & mask) != prefix) continue;
                             const int d = (int)((key >> shift) & 255ull);
-                            const double e = cached ? rg.ecache[j - v0] : e_of(l, md, invT, s.exp_tab);
+                            const double e = cached_e ? rg.ecache[j - v0] : e_of(l, md, invT, s.exp_tab);
                             if (d != cur) {
                                 if (cur >= 0) { atomicAdd(&s.rad_mass[cur], cacc); atomicAdd(&s.rad_cnt[cur], ccnt); }
                                 cur = d; cacc = 0.0; ccnt = 0;
@@ -1158,7 +1162,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
     if (rank == 0 && tid == 0) p.slots[row].st = st;
     if (erow && !bad && T > 0.0) {
         const double md = (double)m;
-        if (cached) {  // coalesced 8-byte stores; they drain after the CTA has moved on
+        if (cached_e) {  // coalesced 8-byte stores; they drain after the CTA has moved on
             for (int j = v0 + tid; j < v1; j += kThreads)
                 erow[j] = is_kept(st, rg.cache[j - v0], j) ? rg.ecache[j - v0] : 0.0;
         } else {
