@@ -78,7 +78,7 @@ def test_projection_exact_on_small_integers_and_deterministic():
 
 
 def test_many_rows_take_several_passes():
-    # 20 rows at Kd = 17408: passes of 6 rows; every row checked on sampled columns
+    # 20 rows at Kd = 17408: one pass of the wide kernel; every row checked on sampled columns
     M, Kd, N = 20, 17408, 5120
     Wq, S = head(N, Kd, 21)
     x = hidden(M, Kd, 300)
@@ -143,3 +143,51 @@ def test_one_workspace_serves_successive_shapes():
         torch.cuda.synchronize()
         assert torch.equal(a, b)
     assert int(shared[:4].view(torch.int32).item()) == 0
+
+
+# Passes of 9..32 rows run on the wide kernel (2..4 n-tiles of 8 rows);
+# 33 and 40 rows take a wide pass and a narrow one.
+@pytest.mark.parametrize("M,Kd,N", [(9, 5120, 7168), (12, 576, 200), (16, 192, 129), (24, 5120, 1000),
+                                    (32, 11008, 1000), (33, 1088, 300), (40, 5120, 130)])
+def test_wide_passes_against_oracle(M, Kd, N):
+    Wq, S = head(N, Kd, 41)
+    x = hidden(M, Kd, 700 + M)
+    y = torch.full((M, N), float("nan"), device="cuda")
+    ws = mtpv.workspace(mtpv.load().mtpv_int4_proj_workspace_bytes(M, Kd, N))
+    mtpv.int4_proj(x, Wq, S, y, ws=ws)
+    torch.cuda.synchronize()
+    cols = np.arange(0, N, 5) if N > 2000 else np.arange(N)
+    ref = oracle.lm_head_int4g64(synth.bf16_bits(x.cpu()), Wq[cols].cpu().numpy(), synth.bf16_bits(S[cols].cpu()),
+                                 threads=8)
+    assert_logits_close(y[:, cols].cpu().numpy(), ref)
+    assert not torch.isnan(y).any()
+    assert int(ws[:4].view(torch.int32).item()) == 0
+    assert not ws[256:512].any()  # ticket counters (one per SM) back at zero
+
+
+@pytest.mark.parametrize("M,Kd,F", [(12, 5120, 1001), (20, 576, 37)])
+def test_wide_gate_up_against_oracle(M, Kd, F):
+    Wq, S = head(2 * F, Kd, 42)
+    x = hidden(M, Kd, 800 + M)
+    h = torch.full((M, F), float("nan"), device="cuda")
+    mtpv.int4_gate_up(x, Wq, S, h)
+    torch.cuda.synchronize()
+    ref = oracle.gate_up_int4g64(synth.bf16_bits(x.cpu()), Wq.cpu().numpy(), synth.bf16_bits(S.cpu()), F,
+                                 threads=8)
+    assert_logits_close(h.cpu().numpy(), ref)
+
+
+def test_wide_pass_exact_on_small_integers_and_deterministic():
+    M, Kd, N = 24, 4096, 700
+    g = torch.Generator().manual_seed(19)
+    Wq = torch.randint(0, 256, (N, Kd // 2), generator=g, dtype=torch.int32).to(torch.uint8)
+    S = torch.pow(2.0, torch.randint(-2, 3, (N, Kd // 64), generator=g).float()).to(torch.bfloat16)
+    x = torch.randint(-3, 4, (M, Kd), generator=g).float().to(torch.bfloat16)
+    y1 = torch.empty((M, N), device="cuda")
+    y2 = torch.empty((M, N), device="cuda")
+    mtpv.int4_proj(x.cuda(), Wq.cuda(), S.cuda(), y1)
+    mtpv.int4_proj(x.cuda(), Wq.cuda(), S.cuda(), y2)
+    torch.cuda.synchronize()
+    ref = oracle.lm_head_int4g64(synth.bf16_bits(x), Wq.numpy(), synth.bf16_bits(S), threads=8)
+    assert (y1.cpu().double().numpy() == ref).all()
+    assert torch.equal(y1, y2)

@@ -229,7 +229,7 @@ static mtpv_status int4_proj_common(const void *x, int M, int Kd, int N, const v
         return MTPV_ERR_INVALID_ARG;
     if (!ws || !aligned(ws, kAlign) || ws_bytes < need) return MTPV_ERR_WORKSPACE;
     return cuda_status(
-        mtpv::launch_int4_proj(x, M, Kd, N, wq, scales, y, ldy, silu_mul, ws, (cudaStream_t)stream));
+        mtpv::launch_int4_proj(x, M, Kd, N, wq, scales, y, ldy, silu_mul, ws, false, (cudaStream_t)stream));
 }
 
 mtpv_status mtpv_int4_proj(const void *x, int M, int Kd, int N, const void *wq, const void *scales,

@@ -765,8 +765,17 @@ size_t lm_head_max_smem_rows(int Kd) {
     return (size_t)(227 * 1024) / ((size_t)Kd * sizeof(float));
 }
 
+// Which kernel takes an int4 head of M > 8 rows: the streamed mma.sync kernel
+// (proj_wide.cu) for up to 32 rows, one pass over the weights; the
+// tensor-memory kernel for 33..64 rows, where the streamed kernel would need
+// two passes.  Measured on B200 at vocabulary 248320, hidden 5120: streamed
+// 307 / 313 / 394 / 449 us at 9 / 16 / 24 / 32 rows, tensor memory ~487 us
+// at each (its single MMA-issuing thread bounds it, not the row count).
+static bool int4_head_streamed(int M, int Kd) { return M > 8 && M <= 32 && Kd % 64 == 0; }
+
 size_t lm_head_scratch_bytes(int M, int Kd, int fmt) {
     if (fmt == MTPV_W_BF16 && M > 8 && lm_head_tc_ok(M, Kd, nullptr, nullptr)) return 256;
+    if (fmt == MTPV_W_INT4_G64 && int4_head_streamed(M, Kd)) return int4_proj_workspace_bytes(M, Kd, 0, false);
     if (fmt == MTPV_W_INT4_G64 && M > 8 && lm_head_tc_int4_ok(M, Kd, nullptr, nullptr, nullptr))
         return lm_head_int4_tc_scratch_bytes(M, Kd);
     return 0;
@@ -799,8 +808,15 @@ cudaError_t launch_lm_head(const void *x, int M, int Kd, int N, const void *w, c
         }
         return cudaSuccess;
     }
-    if (M > 8 && lm_head_tc_int4_ok(M, Kd, x, w, scales))  // one pass, on the tensor-memory kernel
+    if (int4_head_streamed(M, Kd)) {
+        // one pass, streamed mma.sync; unaligned operands take the passes
+        // below instead, which need no scratch (the workspace was sized for
+        // this kernel, never for the tensor-memory one)
+        if (!((uintptr_t)x & 15) && !((uintptr_t)w & 15) && !((uintptr_t)scales & 15))
+            return launch_int4_proj(x, M, Kd, N, w, scales, y, N, false, scratch, true, s);
+    } else if (M > 8 && lm_head_tc_int4_ok(M, Kd, x, w, scales)) {  // one pass, on the tensor-memory kernel
         return launch_lm_head_int4_tc(x, M, Kd, N, w, scales, y, scratch, s);
+    }
     // int4 group-64: passes of up to 8 rows, each on the ring kernel when it
     // takes the shape, else on the direct-load kernel (same bits)
     const int step = (int)std::min<size_t>(8, lm_head_max_smem_rows(Kd));

@@ -34,14 +34,16 @@ cudaError_t launch_lm_heads_pair(const void *xt, int Mt, const void *w, float *y
                                  int N, void *work, cudaStream_t s);
 
 // Int4 group-64 projection y[M, N] = x . deq(wq, scales)^T for decoder
-// layers (any N; M up to 64 in passes of 8 rows, one launch per pass).  With
-// silu_mul, N is a gate half and an up half and y[M, N/2] = silu(gate) * up.
-// ws holds int4_proj_workspace_bytes(M, Kd, N, silu_mul) bytes, zeroed before
-// its first use: the error word, the tiles' ticket counters (each call returns
-// them to zero) and the partial sums of tiles split between SMs.  x, wq and
+// layers and the batched int4 head (any N; M rows in passes of up to 32, one
+// launch per pass, the weights read once per pass).  With silu_mul, N is a
+// gate half and an up half and y[M, N/2] = silu(gate) * up.  ws holds
+// int4_proj_workspace_bytes(M, Kd, N, silu_mul) bytes: the error word, one
+// ticket counter per SM (each call returns them to zero: zero the workspace
+// once before its first use, or pass reset_tickets to clear them on the
+// stream first) and the partial sums of tiles split between SMs.  x, wq and
 // scales 16-byte aligned.
 size_t int4_proj_workspace_bytes(int M, int Kd, int N, bool gate_up);
 cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq, const void *scales,
-                             float *y, int ldy, bool silu_mul, void *ws, cudaStream_t s);
+                             float *y, int ldy, bool silu_mul, void *ws, bool reset_tickets, cudaStream_t s);
 
 }  // namespace mtpv

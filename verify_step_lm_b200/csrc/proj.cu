@@ -1,13 +1,15 @@
-// Decoder-layer projections with int4 group-64 weights for 1..8 activation
-// rows (more in passes of 8), one launch per pass:
+// Int4 group-64 projections for a handful of activation rows:
 //   y[M, N] = x[M, Kd] . deq(Wq, S)^T,   deq = s_g (n - 8)
 //   gate_up: h[M, F] = silu(x . G^T) * (x . U^T), G and U the two halves
 // (hazakura.dev MTPLX notes, Layer 0: the verify pass's matmuls run with a
 // handful of rows; gist.science BaseRT explainer, methodology: per-format
-// GEMV with dequantisation in the inner loop, fused op chains).
+// GEMV with dequantisation in the inner loop, fused op chains).  This file
+// holds the kernel for passes of up to 8 rows and the launch that splits M
+// into passes: up to 8 rows here, 9..32 rows per pass on the wide kernel
+// (proj_wide.cu), which keeps more n-tiles in registers.
 //
-// The nibbles (14-95 MB per matrix) are the whole cost, so the kernel streams
-// them through shared memory at HBM rate:
+// The nibbles (14-95 MB per decoder matrix) are the whole cost, so the
+// kernel streams them through shared memory at HBM rate:
 //   * the work is a list of stages, one stage = a tile of 128 weight rows
 //     (128 output columns; gate_up: 64 gate rows and the matching 64 up rows)
 //     times 8 groups of 64 weights; the tile-major list is cut into one equal
@@ -25,10 +27,11 @@
 //     whose A is -136 everywhere) leaves sum_k (n_k - 8) x_k; the group's
 //     scale multiplies it into the warp's running sum;
 //   * at the end of a tile (or of its run) the CTA adds its warps' sums in a
-//     fixed order; a CTA that covered the whole tile writes y, otherwise it
-//     stores its partial sums and takes a ticket on the tile, and the CTA
-//     that draws the last ticket adds the partials in CTA order (fixed for a
-//     given SM count, so results are deterministic) and writes y.
+//     fixed order; a CTA that covered the whole tile writes y (gate_up:
+//     silu(g) u), otherwise it stores its partial tile and takes a ticket,
+//     and the CTA that draws the last ticket adds the partials in CTA order
+//     (fixed for a given SM count, so results are deterministic), writes y
+//     and resets the ticket.
 // Every mbarrier wait is bounded; a wait that gives up ORs a code into the
 // workspace's error word, the CTA stops computing (it still takes its
 // tickets, so the counters stay consistent) and the producer waits, bounded,
@@ -39,141 +42,30 @@
 
 #include "common.cuh"
 #include "lm_head.cuh"
-#include "tma.cuh"
+#include "proj.cuh"
 
 namespace mtpv {
 
 namespace {
 
-constexpr int kPjCW = 16;                        // consumer warps
-constexpr int kPjThreads = 32 * (kPjCW + 1);     // + the producer warp (the last one)
-constexpr int kPjTileRows = 128;                 // weight rows per tile
-constexpr int kPjG = 8;                          // 64-weight groups per stage
-constexpr int kPjRows = 8;                       // activation rows per pass (one MMA n-tile)
-constexpr int kPjWBytes = kPjTileRows * kPjG * 32;  // nibbles of a stage: 2 boxes of 128-byte rows
-constexpr int kPjXBox = 1024;                    // one group of up to 8 activation rows
-constexpr int kPjXBytes = kPjG * kPjXBox;
-constexpr int kPjSBytes = kPjTileRows * 32;      // scales: two 16-byte chunks per row
-constexpr int kPjStage = kPjWBytes + kPjXBytes + kPjSBytes;
-constexpr int kPjMaxStages = 8;
-constexpr int kPjRed = kPjCW * 16 * 32;          // floats: each warp's 16 sums per lane
-constexpr int kPjPart = 1024;                    // floats of one partial tile
-constexpr int kPjSmemCap = 227 * 1024;
-
-struct PjCtl {
-    uint64_t full[kPjMaxStages];   // a stage's nibbles, activations and scales landed
-    uint64_t empty[kPjMaxStages];  // the consumer warps are done with a stage
-    int abort;                     // a wait gave up: no more copies, no more compute
-    int last;                      // this CTA drew the tile's last ticket
-};
-
-struct PjArgs {
-    const uint16_t *s;       // scales [N, Kd/64] bf16
-    float *y;                // [M, ldy]
-    float *part;             // [grid][2][kPjPart] partial tiles
-    unsigned int *tickets;   // [tiles], zero between calls
-    unsigned int *err;
-    long long T;             // stages in all (tiles x stages per tile)
-    int M, Kd, N, F, ldy;    // F: output columns (N, or N/2 for gate_up)
-    int spt;                 // stages per tile
-    int stages;              // ring depth
-};
-
-// shared-memory loads at 32-bit shared addresses
-__device__ __forceinline__ uint32_t lds32(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ uint4 lds128(uint32_t a) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
-    return v;
-}
-__device__ __forceinline__ float lds_bf16(uint32_t a) {
-    uint32_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=r"(v) : "r"(a));
-    return __uint_as_float(v << 16);
-}
-
-// 16 bytes at base + off into shared memory, zero-filled past total bytes
-// (nothing is read there).
-__device__ __forceinline__ void cp_async16(void *dst, const void *base, size_t off, size_t total) {
-    const uint32_t n = off >= total ? 0u : (uint32_t)min((size_t)16, total - off);
-    const char *src = static_cast<const char *>(base) + (n ? off : 0);
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(su32(dst)), "l"(src), "r"(n) : "memory");
-}
-// Arrive on the mbarrier once this thread's cp.async copies so far have landed.
-__device__ __forceinline__ void cp_async_arrive(uint64_t *b) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(su32(b)) : "memory");
-}
-// Waits for the barrier phase like bar_wait, but gives up early once the
-// CTA's abort word (a 32-bit shared address) is set; the word is read only
-// while the phase is still pending, so the wait that succeeds at once costs
-// one try_wait.
-__device__ __forceinline__ bool bar_wait_or_abort(uint64_t *b, uint32_t parity, uint32_t abort_addr) {
-    for (int i = 0; i < kBarWaitLimit; ++i) {
-        uint32_t done;
-        asm volatile(
-            "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n selp.u32 %0, 1, 0, p;\n}"
-            : "=r"(done)
-            : "r"(su32(b)), "r"(parity)
-            : "memory");
-        if (done) return true;
-        uint32_t ab;
-        asm volatile("ld.volatile.shared.u32 %0, [%1];" : "=r"(ab) : "r"(abort_addr) : "memory");
-        if (ab) return false;
-    }
-    return false;
-}
-__device__ __forceinline__ void consumers_sync() {
-    asm volatile("bar.sync 1, %0;" ::"n"(kPjCW * 32) : "memory");
-}
-
-__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-    asm("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
-        "{%0,%1,%2,%3};"
-        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-// bf16 pairs (128 + n_i, 128 + n_{i+4}) of the eight nibbles of a word,
-// i = 0..3: the nibble lands in the low mantissa bits of 128.0 (explicit
-// shr + lop3; on sm_100 this is ~1.4x faster than the compiler's code for
-// the same C expression).  The offset 136 is taken off through the
-// accumulator (see offset_mma), not per element.
-__device__ __forceinline__ uint32_t nib_or_128(uint32_t v) {
-    uint32_t r;
-    asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(v));  // (v & m) | c
-    return r;
-}
-__device__ __forceinline__ void nib_pairs_bf16(uint32_t w, uint32_t (&p)[4]) {
-    uint32_t s4, s8, s12;
-    asm("shr.b32 %0, %1, 4;" : "=r"(s4) : "r"(w));
-    asm("shr.b32 %0, %1, 8;" : "=r"(s8) : "r"(w));
-    asm("shr.b32 %0, %1, 12;" : "=r"(s12) : "r"(w));
-    p[0] = nib_or_128(w);
-    p[1] = nib_or_128(s4);
-    p[2] = nib_or_128(s8);
-    p[3] = nib_or_128(s12);
-}
-
-__device__ __forceinline__ float silu(float v) { return v / (1.0f + __expf(-v)); }
-
-// The CTA whose run holds stage a (runs: [c T / grid, (c + 1) T / grid)).
-__device__ __forceinline__ long long run_owner(long long a, long long T, long long grid) {
-    return ((a + 1) * grid + T - 1) / T - 1;
-}
+constexpr int kNarrowCW = 16;                      // consumer warps
+constexpr int kNarrowThreads = 32 * (kNarrowCW + 1);  // + the producer warp (the last one)
+constexpr int kNarrowXBox = 1024;                  // one group of up to 8 activation rows
+constexpr int kNarrowXBytes = pj::kG * kNarrowXBox;
+constexpr int kNarrowStage = pj::kWBytes + kNarrowXBytes + pj::kSBytes;
+constexpr int kNarrowRed = kNarrowCW * 16 * 32;    // floats: each warp's 16 sums per lane
+constexpr int kNarrowRows = 8;                     // activation rows per pass
+constexpr int kWideRows = 8 * pj::kMaxNT;          // rows per pass of the wide kernel
 
 }  // namespace
 
 template <bool GU>
-__global__ void __launch_bounds__(kPjThreads, 1)
-    int4_proj_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, PjArgs a) {
+__global__ void __launch_bounds__(kNarrowThreads, 1)
+    int4_proj_narrow_kernel(const __grid_constant__ CUtensorMap tmW, const __grid_constant__ CUtensorMap tmX, pj::Args a) {
     extern __shared__ __align__(1024) unsigned char pj_smem[];
     unsigned char *ring = reinterpret_cast<unsigned char *>(((uintptr_t)pj_smem + 1023) & ~(uintptr_t)1023);
-    float *red = reinterpret_cast<float *>(ring + (size_t)a.stages * kPjStage);
-    PjCtl &c = *reinterpret_cast<PjCtl *>(red + kPjRed);
+    float *red = reinterpret_cast<float *>(ring + (size_t)a.stages * kNarrowStage);
+    pj::Ctl &c = *reinterpret_cast<pj::Ctl *>(red + kNarrowRed);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int Gt = a.Kd >> 6;
     const long long grid = gridDim.x;
@@ -183,7 +75,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) {
             bar_init(&c.full[i], 33);  // the producer's expect_tx + its 32 lanes' cp.async arrivals
-            bar_init(&c.empty[i], kPjCW);
+            bar_init(&c.empty[i], kNarrowCW);
         }
         c.abort = 0;
         c.last = 0;
@@ -191,18 +83,18 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     }
     __syncthreads();
 
-    if (warp == kPjCW) {
+    if (warp == kNarrowCW) {
         // ---------------- producer ----------------
         const size_t sbytes = (size_t)a.N * Gt * 2;
         const bool two_chunks = ((2 * Gt) & 15) != 0;  // a row's 8 scales straddle 16-byte chunks
-        const uint32_t tx = kPjWBytes + kPjG * a.M * 128;
+        const uint32_t tx = pj::kWBytes + pj::kG * a.M * 128;
         const uint32_t abort32 = su32(&c.abort);
         int slot = 0;
         uint32_t phase = 0;
         long long issued = 0;
         int X = (int)(s0 / a.spt), ch = (int)(s0 - (long long)X * a.spt);
         for (long long s = s0; s < s1; ++s) {
-            const bool ok = __all_sync(0xffffffffu, bar_wait_or_abort(&c.empty[slot], phase ^ 1, abort32));
+            const bool ok = __all_sync(0xffffffffu, pj::bar_wait_or_abort(&c.empty[slot], phase ^ 1, abort32));
             if (!ok) {
                 if (lane == 0) {
                     atomicOr(a.err, 1u);
@@ -210,36 +102,36 @@ __global__ void __launch_bounds__(kPjThreads, 1)
                 }
                 break;
             }
-            unsigned char *st = ring + (size_t)slot * kPjStage;
+            unsigned char *st = ring + (size_t)slot * kNarrowStage;
             if (lane == 0) {
                 bar_arrive_expect(&c.full[slot], tx);
 #pragma unroll
                 for (int p = 0; p < 2; ++p) {  // groups 4p .. 4p+3 of the stage: 128-byte rows
-                    const int xc = (ch * kPjG + 4 * p) * 32;
+                    const int xc = (ch * pj::kG + 4 * p) * 32;
                     if (GU) {
                         tma_load_2d(st + p * 16384, &tmW, xc, X * 64, &c.full[slot]);
                         tma_load_2d(st + p * 16384 + 8192, &tmW, xc, a.F + X * 64, &c.full[slot]);
                     } else {
-                        tma_load_2d(st + p * 16384, &tmW, xc, X * kPjTileRows, &c.full[slot]);
+                        tma_load_2d(st + p * 16384, &tmW, xc, X * pj::kTileRows, &c.full[slot]);
                     }
                 }
 #pragma unroll
-                for (int jj = 0; jj < kPjG; ++jj)
-                    tma_load_2d(st + kPjWBytes + jj * kPjXBox, &tmX, (ch * kPjG + jj) * 64, 0, &c.full[slot]);
+                for (int jj = 0; jj < pj::kG; ++jj)
+                    tma_load_2d(st + pj::kWBytes + jj * kNarrowXBox, &tmX, (ch * pj::kG + jj) * 64, 0, &c.full[slot]);
             }
             // scales of tile rows lane + 32 i: the aligned 16-byte chunk(s) holding groups 8 ch .. 8 ch + 7
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = lane + 32 * i;
                 const long long row = GU ? (r < 64 ? (long long)X * 64 + r : (long long)a.F + X * 64 + (r - 64))
-                                         : (long long)X * kPjTileRows + r;
-                const size_t off = ((size_t)row * Gt + (size_t)ch * kPjG) * 2;
+                                         : (long long)X * pj::kTileRows + r;
+                const size_t off = ((size_t)row * Gt + (size_t)ch * pj::kG) * 2;
                 const size_t al = off & ~(size_t)15;
-                unsigned char *dst = st + kPjWBytes + kPjXBytes + r * 32;
-                cp_async16(dst, a.s, al, sbytes);
-                if (two_chunks) cp_async16(dst + 16, a.s, al + 16, sbytes);
+                unsigned char *dst = st + pj::kWBytes + kNarrowXBytes + r * 32;
+                pj::cp_async16(dst, a.s, al, sbytes);
+                if (two_chunks) pj::cp_async16(dst + 16, a.s, al + 16, sbytes);
             }
-            cp_async_arrive(&c.full[slot]);
+            pj::cp_async_arrive(&c.full[slot]);
             ++issued;
             if (++slot == a.stages) {
                 slot = 0;
@@ -272,9 +164,9 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     const uint32_t ring32 = su32(ring);
     const uint32_t wofs0 = (uint32_t)((j >> 2) * 16384 + (16 * 4 * hb + g) * 128 + ((c0 ^ g) << 4) + 4 * t);
     const uint32_t wofs1 = (uint32_t)((j >> 2) * 16384 + (16 * 4 * hb + g) * 128 + (((c0 + 1) ^ g) << 4) + 4 * t);
-    const uint32_t xofs0 = (uint32_t)(kPjWBytes + j * kPjXBox + g * 128 + ((t ^ g) << 4));
-    const uint32_t xofs1 = (uint32_t)(kPjWBytes + j * kPjXBox + g * 128 + (((4 + t) ^ g) << 4));
-    const uint32_t sofs = (uint32_t)(kPjWBytes + kPjXBytes + soff + 2 * j + (16 * 4 * hb + g) * 32);
+    const uint32_t xofs0 = (uint32_t)(pj::kWBytes + j * kNarrowXBox + g * 128 + ((t ^ g) << 4));
+    const uint32_t xofs1 = (uint32_t)(pj::kWBytes + j * kNarrowXBox + g * 128 + (((4 + t) ^ g) << 4));
+    const uint32_t sofs = (uint32_t)(pj::kWBytes + kNarrowXBytes + soff + 2 * j + (16 * 4 * hb + g) * 32);
     float acc[4][4];
 #pragma unroll
     for (int tt = 0; tt < 4; ++tt)
@@ -287,7 +179,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
     int X = (int)(s0 / a.spt), ch = (int)(s0 - (long long)X * a.spt);
     for (long long s = s0; s < s1; ++s) {
         if (!bad) {
-            const bool ok = __all_sync(0xffffffffu, bar_wait_or_abort(&c.full[slot], phase, abort32));
+            const bool ok = __all_sync(0xffffffffu, pj::bar_wait_or_abort(&c.full[slot], phase, abort32));
             if (!ok) {
                 bad = true;
                 if (lane == 0) {
@@ -296,13 +188,13 @@ __global__ void __launch_bounds__(kPjThreads, 1)
                 }
             }
         }
-        if (!bad && ch * kPjG + j < Gt) {
-            const uint32_t st = ring32 + (uint32_t)slot * kPjStage;
+        if (!bad && ch * pj::kG + j < Gt) {
+            const uint32_t st = ring32 + (uint32_t)slot * kNarrowStage;
             // activations of row g: elements 8t .. 8t+7 and 32+8t .. 32+8t+7 of the group
             uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
             if (has_row) {
-                x0 = lds128(st + xofs0);
-                x1 = lds128(st + xofs1);
+                x0 = pj::lds128(st + xofs0);
+                x1 = pj::lds128(st + xofs1);
             }
             // MMA i takes, for lane (g, t), the physical k pairs (8t+i, 8t+i+4)
             // and (32+8t+i, 32+8t+i+4) as its logical (2t, 2t+1) and (2t+8, 2t+9)
@@ -320,22 +212,22 @@ __global__ void __launch_bounds__(kPjThreads, 1)
             {
                 const uint32_t am[4] = {0xC308C308u, 0xC308C308u, 0xC308C308u, 0xC308C308u};
 #pragma unroll
-                for (int i = 0; i < 4; ++i) mma_bf16(off, am, b0[i], b1[i]);
+                for (int i = 0; i < 4; ++i) pj::mma_bf16(off, am, b0[i], b1[i]);
             }
 #pragma unroll
             for (int tt = 0; tt < 4; ++tt) {  // rows ra = 16 (4 hb + tt) + g and rb = ra + 8
                 uint32_t pa0[4], pa1[4], pb0[4], pb1[4];
-                nib_pairs_bf16(lds32(st + wofs0 + tt * 2048), pa0);
-                nib_pairs_bf16(lds32(st + wofs1 + tt * 2048), pa1);
-                nib_pairs_bf16(lds32(st + wofs0 + tt * 2048 + 1024), pb0);
-                nib_pairs_bf16(lds32(st + wofs1 + tt * 2048 + 1024), pb1);
-                const float sa = lds_bf16(st + sofs + tt * 512), sc = lds_bf16(st + sofs + tt * 512 + 256);
+                pj::nib_pairs<false>(pj::lds32(st + wofs0 + tt * 2048), pa0);
+                pj::nib_pairs<false>(pj::lds32(st + wofs1 + tt * 2048), pa1);
+                pj::nib_pairs<false>(pj::lds32(st + wofs0 + tt * 2048 + 1024), pb0);
+                pj::nib_pairs<false>(pj::lds32(st + wofs1 + tt * 2048 + 1024), pb1);
+                const float sa = pj::lds_bf16(st + sofs + tt * 512), sc = pj::lds_bf16(st + sofs + tt * 512 + 256);
                 // sum_k (128 + n_k) x_k, then + (-136 sum_k x_k) = sum_k (n_k - 8) x_k
                 float cc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const uint32_t af[4] = {pa0[i], pb0[i], pa1[i], pb1[i]};
-                    mma_bf16(cc, af, b0[i], b1[i]);
+                    pj::mma_bf16(cc, af, b0[i], b1[i]);
                 }
                 acc[tt][0] = fmaf(sa, cc[0] + off[0], acc[tt][0]);
                 acc[tt][1] = fmaf(sa, cc[1] + off[1], acc[tt][1]);
@@ -363,7 +255,7 @@ __global__ void __launch_bounds__(kPjThreads, 1)
             red[(warp * 16 + v) * 32 + lane] = acc[v >> 2][v & 3];
             acc[v >> 2][v & 3] = 0.0f;
         }
-        consumers_sync();
+        pj::named_sync<kNarrowCW * 32>();
         // thread q: entry (v, lane') of both row halves b = 0, 1 (warps 8b .. 8b+7)
         const int q = threadIdx.x, v = q >> 5, lq = q & 31;
         const int m = 2 * (lq & 3) + (v & 1);
@@ -376,58 +268,58 @@ __global__ void __launch_bounds__(kPjThreads, 1)
             for (int jj = 0; jj < 8; ++jj) sum += red[((b * 8 + jj) * 16 + v) * 32 + lq];
             val[b] = sum;
         }
-        const long long cf = run_owner((long long)Xs * a.spt, a.T, grid);
-        const long long cl = run_owner((long long)Xs * a.spt + a.spt - 1, a.T, grid);
+        const long long cf = pj::run_owner((long long)Xs * a.spt, a.T, grid);
+        const long long cl = pj::run_owner((long long)Xs * a.spt + a.spt - 1, a.T, grid);
         if (cf == cl) {  // the whole tile is this CTA's
             if (m < a.M) {
                 if (GU) {
                     const int col = Xs * 64 + rloc;
-                    if (col < a.F) a.y[(size_t)m * a.ldy + col] = silu(val[0]) * val[1];
+                    if (col < a.F) a.y[(size_t)m * a.ldy + col] = pj::silu(val[0]) * val[1];
                 } else {
 #pragma unroll
                     for (int b = 0; b < 2; ++b) {
-                        const int col = Xs * kPjTileRows + 64 * b + rloc;
+                        const int col = Xs * pj::kTileRows + 64 * b + rloc;
                         if (col < a.N) a.y[(size_t)m * a.ldy + col] = val[b];
                     }
                 }
             }
-            consumers_sync();  // red is read before the next tile's sums go there
+            pj::named_sync<kNarrowCW * 32>();  // red is read before the next tile's sums go there
             continue;
         }
         const int pslot = (s0 / a.spt == Xs) ? 0 : 1;  // the run's first tile, or its last
-        float *pp = a.part + ((size_t)blockIdx.x * 2 + pslot) * kPjPart;
+        float *pp = a.part + ((size_t)blockIdx.x * 2 + pslot) * pj::kPart;
         if (m < a.M) {
             pp[q] = val[0];
             pp[512 + q] = val[1];
         }
-        consumers_sync();
+        pj::named_sync<kNarrowCW * 32>();
         if (q == 0) {  // the barrier made the CTA's stores this thread's; the fence publishes them
             __threadfence();
-            const unsigned int old = atomicAdd(&a.tickets[Xs], 1u);
+            const unsigned int old = atomicAdd(&a.tickets[cf], 1u);
             const int last = (old == (unsigned int)(cl - cf)) ? 1 : 0;
             if (last) __threadfence();
             *(volatile int *)&c.last = last;
         }
-        consumers_sync();
+        pj::named_sync<kNarrowCW * 32>();
         if (*(volatile int *)&c.last) {
             if (m < a.M) {
                 float v0 = 0.0f, v1 = 0.0f;
                 for (long long cc = cf; cc <= cl; ++cc) {  // contributors in CTA order
                     const int sl = ((cc * a.T / grid) / a.spt == Xs) ? 0 : 1;
-                    const float *qp = a.part + ((size_t)cc * 2 + sl) * kPjPart;
+                    const float *qp = a.part + ((size_t)cc * 2 + sl) * pj::kPart;
                     v0 += __ldcg(qp + q);
                     v1 += __ldcg(qp + 512 + q);
                 }
                 if (GU) {
                     const int col = Xs * 64 + rloc;
-                    if (col < a.F) a.y[(size_t)m * a.ldy + col] = silu(v0) * v1;
+                    if (col < a.F) a.y[(size_t)m * a.ldy + col] = pj::silu(v0) * v1;
                 } else {
-                    const int col0 = Xs * kPjTileRows + rloc;
+                    const int col0 = Xs * pj::kTileRows + rloc;
                     if (col0 < a.N) a.y[(size_t)m * a.ldy + col0] = v0;
                     if (col0 + 64 < a.N) a.y[(size_t)m * a.ldy + col0 + 64] = v1;
                 }
             }
-            if (q == 0) a.tickets[Xs] = 0u;  // ready for the next call
+            if (q == 0) a.tickets[cf] = 0u;  // ready for the next call
         }
     }
 }
@@ -437,26 +329,14 @@ __global__ void __launch_bounds__(kPjThreads, 1)
 // ---------------------------------------------------------------------------
 namespace {
 
-constexpr size_t kPjCtlBytes = (sizeof(PjCtl) + 15) / 16 * 16;
-
-int pj_stages() {
-    const int n = (kPjSmemCap - 1024 - kPjRed * 4 - (int)kPjCtlBytes) / kPjStage;
-    return std::min(n, kPjMaxStages);
+int narrow_stages() {
+    const int n = (pj::kSmemCap - 1024 - kNarrowRed * 4 - (int)pj::kCtlBytes) / kNarrowStage;
+    return std::min(n, pj::kMaxStages);
 }
-size_t pj_smem(int stages) { return 1024 + (size_t)stages * kPjStage + kPjRed * 4 + kPjCtlBytes; }
+size_t narrow_smem(int stages) { return 1024 + (size_t)stages * kNarrowStage + kNarrowRed * 4 + pj::kCtlBytes; }
 
-int pj_tiles(int N, bool gate_up) { return gate_up ? (N / 2 + 63) / 64 : (N + kPjTileRows - 1) / kPjTileRows; }
-
-struct PjWs {
-    size_t tickets, part, total;
-};
-PjWs proj_layout(int N, bool gate_up, int sms) {
-    PjWs l;
-    l.tickets = 256;  // after the error word
-    l.part = l.tickets + ((size_t)pj_tiles(N, gate_up) * sizeof(unsigned int) + 255) / 256 * 256;
-    l.total = l.part + (size_t)sms * 2 * kPjPart * sizeof(float);
-    return l;
-}
+// n-tiles the widest pass of M rows needs (the narrow kernel's partials are one n-tile)
+int passes_nt(int M) { return M <= kNarrowRows ? 1 : std::min(pj::kMaxNT, (std::min(M, kWideRows) + 7) / 8); }
 
 int plan_sms() {
     const int n = current_device_sms();
@@ -466,56 +346,68 @@ int plan_sms() {
 }  // namespace
 
 size_t int4_proj_workspace_bytes(int M, int Kd, int N, bool gate_up) {
-    (void)M;
     (void)Kd;
-    return proj_layout(N, gate_up, plan_sms()).total;
+    (void)N;
+    (void)gate_up;
+    return pj::layout(passes_nt(M), plan_sms()).total;
 }
 
 cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq, const void *scales,
-                             float *y, int ldy, bool silu_mul, void *ws, cudaStream_t s) {
+                             float *y, int ldy, bool silu_mul, void *ws, bool reset_tickets, cudaStream_t s) {
     if (((uintptr_t)x & 15) || ((uintptr_t)wq & 15) || ((uintptr_t)scales & 15) || Kd % 64 || M < 1)
         return cudaErrorInvalidValue;
-    const void *kernel = silu_mul ? (const void *)int4_proj_kernel<true> : (const void *)int4_proj_kernel<false>;
-    const int stages = pj_stages();
-    const size_t smem = pj_smem(stages);
-    int occ = 0, sms = 0;
-    cudaError_t e = kernel_setup(kernel, kPjThreads, smem, &occ, &sms);
-    if (e != cudaSuccess) return e;
-    const int psms = plan_sms();  // the workspace holds partial tiles for this many CTAs
-    const int tiles = pj_tiles(N, silu_mul);
-    const int spt = (Kd / 64 + kPjG - 1) / kPjG;
-    const PjWs l = proj_layout(N, silu_mul, psms);
+    const int psms = plan_sms();  // the workspace holds tickets and partial tiles for this many CTAs
+    const int spt = (Kd / 64 + pj::kG - 1) / pj::kG;
+    const pj::Ws l = pj::layout(passes_nt(M), psms);
     char *w = static_cast<char *>(ws);
-    PjArgs a;
+    pj::Args a;
     a.s = static_cast<const uint16_t *>(scales);
     a.part = reinterpret_cast<float *>(w + l.part);
     a.tickets = reinterpret_cast<unsigned int *>(w + l.tickets);
     a.err = reinterpret_cast<unsigned int *>(w);
-    a.T = (long long)tiles * spt;
+    a.T = (long long)pj::tiles(N, silu_mul) * spt;
     a.Kd = Kd;
     a.N = N;
     a.F = silu_mul ? N / 2 : N;
     a.ldy = ldy;
     a.spt = spt;
-    a.stages = stages;
-    const int grid = (int)std::max(1LL, std::min<long long>(a.T, std::min(sms, psms)));
+    a.stages = 0;
+    cudaError_t e;
+    if (reset_tickets) {
+        e = cudaMemsetAsync(w, 0, l.part, s);  // error word and tickets
+        if (e != cudaSuccess) return e;
+    }
     CUtensorMap tmW;
-    e = map_2d(&tmW, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Kd / 2, N, 128, silu_mul ? 64 : kPjTileRows,
+    e = map_2d(&tmW, wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Kd / 2, N, 128, silu_mul ? 64 : pj::kTileRows,
                CU_TENSOR_MAP_SWIZZLE_128B);
     if (e != cudaSuccess) return e;
-    for (int m0 = 0; m0 < M; m0 += kPjRows) {
-        const int mp = std::min(kPjRows, M - m0);
+    const int rows = M <= kNarrowRows ? kNarrowRows : kWideRows;
+    for (int m0 = 0; m0 < M; m0 += rows) {
+        const int mp = std::min(rows, M - m0);
         CUtensorMap tmX;
         e = map_2d(&tmX, static_cast<const uint16_t *>(x) + (size_t)m0 * Kd, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
                    Kd, mp, 64, mp, CU_TENSOR_MAP_SWIZZLE_128B);
         if (e != cudaSuccess) return e;
         a.M = mp;
         a.y = y + (size_t)m0 * ldy;
-        if (silu_mul)
-            int4_proj_kernel<true><<<grid, kPjThreads, smem, s>>>(tmW, tmX, a);
-        else
-            int4_proj_kernel<false><<<grid, kPjThreads, smem, s>>>(tmW, tmX, a);
-        e = cudaGetLastError();
+        if (mp > kNarrowRows) {
+            e = pj::launch_wide_pass(tmW, tmX, a, (mp + 7) / 8, silu_mul, psms, s);
+        } else {
+            const int stages = narrow_stages();
+            const size_t smem = narrow_smem(stages);
+            const void *kernel = silu_mul ? (const void *)int4_proj_narrow_kernel<true>
+                                          : (const void *)int4_proj_narrow_kernel<false>;
+            int occ = 0, sms = 0;
+            e = kernel_setup(kernel, kNarrowThreads, smem, &occ, &sms);
+            if (e != cudaSuccess) return e;
+            a.stages = stages;
+            const int grid = (int)std::max(1LL, std::min<long long>(a.T, std::min(sms, psms)));
+            if (silu_mul)
+                int4_proj_narrow_kernel<true><<<grid, kNarrowThreads, smem, s>>>(tmW, tmX, a);
+            else
+                int4_proj_narrow_kernel<false><<<grid, kNarrowThreads, smem, s>>>(tmW, tmX, a);
+            e = cudaGetLastError();
+        }
         if (e != cudaSuccess) return e;
     }
     return cudaSuccess;
