@@ -116,14 +116,20 @@ MTPV_API void mtpv_set_wait_polls(int polls);
  *           shared-memory rings when Kd is a multiple of 512, the scales
  *           are 16-byte aligned and (M + 1)(2 Kd + 16) + Kd/2 <= 75776
  *           bytes, else with direct register loads (the same bits).
- *           9 <= M <= 64: one pass over the weights on tcgen05 (fifth-
- *           generation tensor cores, fp32 accumulators in tensor memory,
- *           weights streamed by TMA; rows padded to a multiple of 16).
- *           MTPV_W_BF16 takes it for any Kd; MTPV_W_INT4_G64 when Kd is a
+ *           9 <= M <= 64, MTPV_W_BF16: one pass over the weights on
+ *           tcgen05 (fifth-generation tensor cores, fp32 accumulators in
+ *           tensor memory, weights streamed by TMA; rows padded to a
+ *           multiple of 16), for any Kd.
+ *           9 <= M <= 32, MTPV_W_INT4_G64, x, w and scales 16-byte aligned:
+ *           one pass over the weights streamed by TMA through shared
+ *           memory into mma.sync (the nibble n becomes the bf16 value n - 8
+ *           exactly; the computation of mtpv_int4_proj, two to four n-tiles
+ *           of 8 rows per pass).
+ *           33 <= M <= 64, MTPV_W_INT4_G64: one pass on tcgen05 when Kd is a
  *           multiple of 512 and at most 8192 and x, w and scales are 16-byte
  *           aligned (the nibbles are dequantised to exact fp16 (n - 8) s f,
  *           f a per-row power of two, and the activations staged once as
- *           fp16 times a per-row power of two); other int4 shapes go in
+ *           fp16 times a per-row power of two).  Other int4 shapes go in
  *           passes of min(8, floor(232448 / (4 Kd))) rows, re-reading the
  *           weights once per pass.
  *   Kd      reduction length, a positive multiple of 64, at most 58112.
@@ -141,11 +147,12 @@ MTPV_API void mtpv_set_wait_polls(int polls);
  *   y       device fp32 [M, N] row-major, fully overwritten (4-byte aligned).
  *   ws, ws_bytes  workspace of mtpv_lm_head_workspace_bytes() bytes, 256-byte
  *           aligned (may be NULL when the query returns 0, as it does for
- *           M <= 8).  On the tcgen05 path its first 32-bit word is an error
- *           word, cleared by the call: nonzero once the call has run means
- *           a bounded device-side wait gave up and y is not valid (the
- *           kernel never hangs).  The int4 path also stages the activations
- *           there.
+ *           M <= 8).  For M > 8 its first 32-bit word is an error word,
+ *           cleared by the call: nonzero once the call has run means a
+ *           bounded device-side wait gave up and y is not valid (the kernel
+ *           never hangs).  The rest holds, per path, the streamed kernel's
+ *           ticket counters (cleared by the call) and partial sums, or the
+ *           tcgen05 int4 kernel's staged activations.
  * Accumulation is fp32.  Errors: MTPV_ERR_INVALID_ARG for NULL pointers,
  * M/Kd/N out of range or misaligned x/w; MTPV_ERR_WORKSPACE when ws_bytes is
  * below mtpv_lm_head_workspace_bytes().
@@ -207,9 +214,10 @@ MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, fl
  *   wq      device uint8 [N, Kd/2] (N = 2F for gate_up), MTPV_W_INT4_G64
  *           nibble order; scales device bf16 [N, Kd/64]; both 16-byte
  *           aligned.
- *   Kd      a positive multiple of 64, at most 2^20.  One launch per pass of
- *           up to 8 rows (one MMA n-tile); the weights are read once per
- *           pass.
+ *   Kd      a positive multiple of 64, at most 2^20.  One launch per pass:
+ *           M <= 8 in one pass of one MMA n-tile; more rows in passes of up
+ *           to 32 (two to four n-tiles of 8 rows, a second kernel with the
+ *           same arithmetic); the weights are read once per pass.
  *   y, h    device fp32 [M, N] / [M, F], fully overwritten.
  * Arithmetic: bf16 mma.sync of exactly dequantised weights (the nibble n
  * becomes the bf16 value n - 8) against the bf16 activations as given, a
