@@ -153,7 +153,8 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
     // ---------------- consumers ----------------
     const int g = lane >> 2, t = lane & 3;
     const int j = warp & 7, hb = warp >> 3;  // group of the stage; MMA tiles 4 hb .. 4 hb + 3
-    const bool has_row = g < a.M;
+    const int xr = pj::act_row(g);  // the activation row behind this lane's MMA column
+    const bool has_row = xr < a.M;
     // byte offset of group 0 of the stage inside a row's scale chunk: rows of
     // this lane are = g (mod 8) in the tile, and (F + g) for gate_up's up rows
     const int srow = (GU && hb) ? ((a.F + g) & 7) : g;
@@ -164,8 +165,8 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
     const uint32_t ring32 = su32(ring);
     const uint32_t wofs0 = (uint32_t)((j >> 2) * 16384 + (16 * 4 * hb + g) * 128 + ((c0 ^ g) << 4) + 4 * t);
     const uint32_t wofs1 = (uint32_t)((j >> 2) * 16384 + (16 * 4 * hb + g) * 128 + (((c0 + 1) ^ g) << 4) + 4 * t);
-    const uint32_t xofs0 = (uint32_t)(pj::kWBytes + j * kNarrowXBox + g * 128 + ((t ^ g) << 4));
-    const uint32_t xofs1 = (uint32_t)(pj::kWBytes + j * kNarrowXBox + g * 128 + (((4 + t) ^ g) << 4));
+    const uint32_t xofs0 = (uint32_t)(pj::kWBytes + j * kNarrowXBox + xr * 128 + ((t ^ xr) << 4));
+    const uint32_t xofs1 = (uint32_t)(pj::kWBytes + j * kNarrowXBox + xr * 128 + (((4 + t) ^ xr) << 4));
     const uint32_t sofs = (uint32_t)(pj::kWBytes + kNarrowXBytes + soff + 2 * j + (16 * 4 * hb + g) * 32);
     float acc[4][4];
 #pragma unroll
@@ -190,7 +191,7 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
         }
         if (!bad && ch * pj::kG + j < Gt) {
             const uint32_t st = ring32 + (uint32_t)slot * kNarrowStage;
-            // activations of row g: elements 8t .. 8t+7 and 32+8t .. 32+8t+7 of the group
+            // activations of row act_row(g): elements 8t .. 8t+7 and 32+8t .. 32+8t+7 of the group
             uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
             if (has_row) {
                 x0 = pj::lds128(st + xofs0);
@@ -258,7 +259,7 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
         pj::named_sync<kNarrowCW * 32>();
         // thread q: entry (v, lane') of both row halves b = 0, 1 (warps 8b .. 8b+7)
         const int q = threadIdx.x, v = q >> 5, lq = q & 31;
-        const int m = 2 * (lq & 3) + (v & 1);
+        const int m = pj::act_row(2 * (lq & 3) + (v & 1));
         const int rloc = 16 * (v >> 2) + (lq >> 2) + 8 * ((v >> 1) & 1);  // row within a 64-row half
         float val[2];
 #pragma unroll

@@ -126,6 +126,13 @@ __device__ __forceinline__ void nib_pairs(uint32_t w, uint32_t (&p)[4]) {
 
 __device__ __forceinline__ float silu(float v) { return v / (1.0f + __expf(-v)); }
 
+// The activation row behind MMA column c of an n-tile: (c >> 1) | ((c & 1) << 2),
+// i.e. columns 0..7 take rows 0, 4, 1, 5, 2, 6, 3, 7.  Lanes g and g + 1 of a
+// quarter-warp then read rows whose 128-byte-swizzle keys differ in bit 2, so
+// their 16-byte activation chunks fall in disjoint bank groups (with row = c
+// both rows' chunks collided, a 2-way conflict on every fragment load).
+__host__ __device__ __forceinline__ int act_row(int c) { return (c >> 1) | ((c & 1) << 2); }
+
 // The CTA whose run holds stage a (runs: [c T / grid, (c + 1) T / grid)).
 __device__ __forceinline__ long long run_owner(long long a, long long T, long long grid) {
     return ((a + 1) * grid + T - 1) / T - 1;

@@ -132,6 +132,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
     const int soff = (((2 * Gt) & 15) * srow) & 15;
     const uint32_t ring32 = su32(ring);
     // per-lane offsets inside a stage, for each of the warp's two groups
+    const int xr = pj::act_row(g);  // the activation row (within an n-tile) behind this lane's MMA column
     uint32_t wofs0[2], wofs1[2], xofs0[2], xofs1[2], sofs[2];
 #pragma unroll
     for (int jj = 0; jj < 2; ++jj) {
@@ -139,8 +140,8 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         const int rowb = (j >> 2) * 16384 + (32 * tp + g) * 128;
         wofs0[jj] = (uint32_t)(rowb + ((c0 ^ g) << 4) + 4 * t);
         wofs1[jj] = (uint32_t)(rowb + (((c0 + 1) ^ g) << 4) + 4 * t);
-        xofs0[jj] = (uint32_t)(pj::kWBytes + j * NT * 1024 + g * 128 + ((t ^ g) << 4));
-        xofs1[jj] = (uint32_t)(pj::kWBytes + j * NT * 1024 + g * 128 + (((4 + t) ^ g) << 4));
+        xofs0[jj] = (uint32_t)(pj::kWBytes + j * NT * 1024 + xr * 128 + ((t ^ xr) << 4));
+        xofs1[jj] = (uint32_t)(pj::kWBytes + j * NT * 1024 + xr * 128 + (((4 + t) ^ xr) << 4));
         sofs[jj] = (uint32_t)(pj::kWBytes + kXBytes + soff + 2 * j + (32 * tp + g) * 32);
     }
     float acc[2][NT][4];
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
             for (int jj = 0; jj < 2; ++jj) {
                 if (ch * pj::kG + 2 * gp + jj >= Gt) continue;  // past the row's last group (warp-uniform)
-                // activations: row 8 nt + g, elements 8t .. 8t+7 and 32+8t .. 32+8t+7 of
+                // activations: row 8 nt + act_row(g), elements 8t .. 8t+7 and 32+8t .. 32+8t+7 of
                 // the group; MMA i takes, for lane (g, t), the physical k pairs
                 // (8t+i, 8t+i+4) and (32+8t+i, 32+8t+i+4) as its logical (2t, 2t+1)
                 // and (2t+8, 2t+9)
@@ -178,7 +179,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
 #pragma unroll
                 for (int nt = 0; nt < NT; ++nt) {
                     uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
-                    if (8 * nt + g < a.M) {
+                    if (8 * nt + xr < a.M) {
                         x0 = pj::lds128(st + xofs0[jj] + nt * 1024);
                         x1 = pj::lds128(st + xofs1[jj] + nt * 1024);
                     }
@@ -263,7 +264,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
                 val0 += red[((4 * gq + tq) * 8 + v) * 32 + lq];
                 val1 += red[((4 * gq + tq + 2) * 8 + v) * 32 + lq];
             }
-            const int m = 8 * nt + 2 * (lq & 3) + (v & 1);
+            const int m = 8 * nt + pj::act_row(2 * (lq & 3) + (v & 1));
             if (sole) {
                 if (m < a.M) {
                     if (GU) {
@@ -299,7 +300,7 @@ __global__ void __launch_bounds__(kWideThreads, 1)
         if (*(volatile int *)&c.last) {
 #pragma unroll
             for (int nt = 0; nt < NT; ++nt) {
-                const int m = 8 * nt + 2 * (lq & 3) + (v & 1);
+                const int m = 8 * nt + pj::act_row(2 * (lq & 3) + (v & 1));
                 if (m >= a.M) continue;
                 float v0 = 0.0f, v1 = 0.0f;
                 for (long long cc = cf; cc <= cl; ++cc) {  // contributors in CTA order
