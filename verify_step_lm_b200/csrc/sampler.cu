@@ -74,17 +74,20 @@ constexpr int kMaxCluster = 16;     // CTAs per cluster at most (a power of two;
 // Dynamic shared memory of the statistics kernel: a region reused phase by
 // phase, then the small bookkeeping struct.
 //   region: [logits slice: kCacheFloats fp32][their exps: kCacheFloats fp64]
+//           (or, for a longer slice, its logits alone: kCacheFloatsLogits fp32)
 //           [hist_mass: kBins fp64][cand: kCandCap u64]
 //           [cand_e: kCandCap fp64]
+// kCacheFloatsLogits holds a slice of vocabulary 248320 over 8 CTAs.
+constexpr int kCacheFloatsLogits = 31232;
 constexpr size_t kOffExp = kCacheFloats * sizeof(float);
-constexpr size_t kOffHistMass = kOffExp + kCacheFloats * sizeof(double);
+constexpr size_t kOffHistMass = (kOffExp + kCacheFloats * sizeof(double)) > kCacheFloatsLogits * sizeof(float)
+                                    ? (kOffExp + kCacheFloats * sizeof(double))
+                                    : kCacheFloatsLogits * sizeof(float);
 constexpr size_t kOffCand = kOffHistMass + kBins * sizeof(double);
 constexpr size_t kOffCandE = kOffCand + kCandCap * sizeof(unsigned long long);
 constexpr size_t kRegionBytes = kOffCandE + kCandCap * sizeof(double);
 static_assert(kOffExp % 16 == 0 && kOffHistMass % 16 == 0, "region alignment");
-// A slice too long for its exps as well still keeps its logits in shared
-// memory, using the exps' room too (114 KB: 29184 floats).
-constexpr int kCacheFloatsLogits = (int)(kOffHistMass / sizeof(float));
+static_assert(kOffHistMass % 16 == 0, "region alignment");
 constexpr int kDrawBufDoubles = 19456;  // the draw kernel's weight buffer (152 KB: two rows' slices)
 constexpr size_t kDrawBufBytes = kDrawBufDoubles * sizeof(double);
 
@@ -1330,12 +1333,12 @@ namespace {
 
 // Cluster size of a sampler launch: the largest power of two up to 16 that
 // can be resident on the device (the occupancy calculator is asked once per
-// kernel and device).  The kernels work with any power of two from 1 to 16,
-// but smaller clusters only pay at many rows if a CTA's slice still fits its
-// shared-memory cache: past it every pass re-reads the row from L2, which on
-// B200 cost more than the waves of 16-CTA clusters it saves (measured: 8
-// sequences x 3 drafts at vocabulary 248320, 459 us with 16-CTA clusters in
-// waves, 581 us with 2-CTA clusters in one wave).
+// kernel and device); launch_sampler may halve it for many rows.  The kernels
+// work with any power of two from 1 to 16, but smaller clusters only pay if a
+// CTA's slice still fits its shared-memory cache: past it every pass re-reads
+// the row from L2, which on B200 cost more than the waves it saves (8
+// sequences x 3 drafts at vocabulary 248320, before the logits-only cache:
+// 459 us with 16-CTA clusters in waves, 581 us with 2-CTA clusters in one).
 int g_max_active[2][64][5];  // [kernel][device][log2 C]: clusters resident at once; -1 = cannot launch
 bool g_known[2][64];
 std::mutex g_cluster_mu;
@@ -1379,6 +1382,20 @@ int cluster_size_for(int which, Kern kernel, size_t smem, int units) {
     return 8;
 }
 
+// Clusters of size c (a power of two) of a kernel whose table is filled (by
+// cluster_size_for) that the device holds at once; 0 if unknown.
+int max_active_clusters(int which, int c) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 0;
+    }
+    int lg = 0;
+    while ((1 << lg) < c && lg < 4) ++lg;
+    std::lock_guard<std::mutex> lock(g_cluster_mu);
+    return g_known[which][dev] ? std::max(0, g_max_active[which][dev][lg]) : 0;
+}
+
 // Both sampler kernels are launched as programmatic dependents of the work
 // before them on the stream: their CTAs may be scheduled while that work
 // drains, and each waits (griddepcontrol.wait) for it to complete before
@@ -1413,7 +1430,18 @@ cudaError_t launch_sampler(const SamplerParams &params, int rows, cudaStream_t s
     SamplerParams p = params;
     const int polls = g_wait_polls.load();
     p.wait_polls = polls < 0 ? kWaitLimit : polls;
-    const int C1 = cluster_size_for(0, sampler_stats_kernel, kStatsSmemBytes, rows);
+    int C1 = cluster_size_for(0, sampler_stats_kernel, kStatsSmemBytes, rows);
+    // When the rows need several waves of these clusters, halve the cluster
+    // while the halved slices still keep their logits in shared memory and
+    // more clusters fit at once: more rows per wave, each CTA twice the
+    // tokens (and, past the exps' room, the draw kernel recomputing the kept
+    // weights).  Measured per verify at vocabulary 151936: 2 / 4 / 8 / 16
+    // sequences 63 -> 61, 117 -> 109, 237 -> 205, 467 -> 399 us; at vocabulary
+    // 248320 and 8 sequences 347 -> 286 us; one sequence (7 rows, one wave)
+    // keeps 16-CTA clusters.
+    while (C1 > 1 && rows > max_active_clusters(0, C1) && (p.V + C1 / 2 - 1) / (C1 / 2) <= kCacheFloatsLogits &&
+           max_active_clusters(0, C1 / 2) > max_active_clusters(0, C1))
+        C1 /= 2;
     // The fp64 weight cache pays only while a CTA's slice (and its exps) stays
     // in shared memory: then the statistics kernel writes the masked exps it
     // already holds and the draw kernel bulk-loads them.  Past the slice
