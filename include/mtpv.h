@@ -424,11 +424,19 @@ MTPV_API mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft,
 
 /* ------------------------------------------------------------------------
  * mtpv_verify_step_host -- mtpv_verify_step with the per-step inputs and
- * outputs in HOST memory: h_target, h_draft, draft_tokens, u_accept, u_sample
- * are copied host->device, out_tokens / out_accepted / row_status (row_status
- * may be NULL) device->host, all on `stream`, and the call returns after the
- * stream has drained.  Weights and ws stay on the device.  Page-locked host
- * buffers give asynchronous copies; pageable ones work but are slower.
+ * outputs in HOST memory; the call returns after the stream has drained.
+ * Weights and ws stay on the device.
+ *   h_target, h_draft  copied host->device on `stream` (page-locked buffers
+ *                   give asynchronous copies; pageable ones work, slower).
+ *   draft_tokens, u_accept, u_sample  read by the host during the call and
+ *                   passed to the sampler by value in its launch parameters
+ *                   (no copy of their own; B*(K+1) <= 64 always holds here).
+ *   out_tokens, out_accepted, row_status (row_status may be NULL)  written
+ *                   by the sampler kernel itself when every one of them is
+ *                   page-locked host memory mapped into the device's address
+ *                   space (cudaPointerGetAttributes reports a device
+ *                   pointer for it); otherwise written to ws and copied
+ *                   device->host on `stream`.
  * ws of at least mtpv_verify_step_host_workspace_bytes(B, K, V, h) bytes.
  * ---------------------------------------------------------------------- */
 MTPV_API size_t mtpv_verify_step_host_workspace_bytes(int B, int K, int V, int h);

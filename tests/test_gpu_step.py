@@ -77,18 +77,31 @@ def test_tiny_step_against_oracle_and_components(B):
     assert agree >= 0.8 * total
 
 
-def test_host_io_step_equals_device_step():
-    B, K, V, h = 2, 3, 4096, 512
+# Outputs of mtpv_verify_step_host: all page-locked (the sampler writes them
+# in host memory itself), all pageable (written to the workspace and copied
+# back), one of each kind (copied back), no row_status.  B (K + 1) = 64 fills
+# the by-value block of per-position inputs.
+@pytest.mark.parametrize("B,K,outputs", [(2, 3, "pinned"), (2, 3, "pageable"), (2, 3, "mixed"),
+                                         (2, 3, "no_status"), (16, 3, "pinned"), (8, 7, "pageable")])
+def test_host_io_step_equals_device_step(B, K, outputs):
+    V, h = 4096, 512
     W, Wq, S, Ht, Hd, u = make_inputs(B, K, V, h, 5, 0.05)
     d, _ = draft_tokens_from_oracle(Hd, Wq, S, B, K, u)
     _, _, ot, oa, rs = run_step(W, Wq, S, Ht, Hd, d, u, B, K)
     pin = lambda t: torch.as_tensor(t).contiguous().pin_memory()
-    ot_h = torch.full((B, K + 1), -9, dtype=torch.int32).pin_memory()
-    oa_h = torch.full((B,), -9, dtype=torch.int32).pin_memory()
-    rs_h = torch.full((B,), -9, dtype=torch.int32).pin_memory()
-    mtpv.verify_step_host(cuda(W), cuda(Wq), cuda(S), pin(Ht), pin(Hd), pin(np.asarray(d, np.int32)),
-                          pin(u["u_accept"]), pin(u["u_sample"]), B, K, T, TOP_P, ot_h, oa_h, rs_h)
-    assert torch.equal(ot_h, ot.cpu()) and torch.equal(oa_h, oa.cpu()) and torch.equal(rs_h, rs.cpu())
+    mk = lambda shape, pinned: (torch.full(shape, -9, dtype=torch.int32).pin_memory() if pinned
+                                else torch.full(shape, -9, dtype=torch.int32))
+    ot_h = mk((B, K + 1), outputs in ("pinned", "mixed", "no_status"))
+    oa_h = mk((B,), outputs in ("pinned", "no_status"))
+    rs_h = None if outputs == "no_status" else mk((B,), outputs == "pinned")
+    # drafts and uniforms may sit in pageable memory: the host reads them
+    d_h = torch.from_numpy(np.ascontiguousarray(d, np.int32))
+    ua_h = torch.as_tensor(u["u_accept"]).contiguous()
+    mtpv.verify_step_host(cuda(W), cuda(Wq), cuda(S), pin(Ht), pin(Hd), d_h, ua_h, pin(u["u_sample"]), B, K,
+                          T, TOP_P, ot_h, oa_h, rs_h)
+    assert torch.equal(ot_h, ot.cpu()) and torch.equal(oa_h, oa.cpu())
+    if rs_h is not None:
+        assert torch.equal(rs_h, rs.cpu())
 
 
 def test_qwen_class_step_full_size():

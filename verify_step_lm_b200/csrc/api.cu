@@ -1,5 +1,6 @@
 // extern "C" entry points of libmtpv: argument checks, workspace layout and
 // kernel launches.  Semantics and citations are in include/mtpv.h.
+#include <cstring>
 #include <math.h>
 #include <stdint.h>
 
@@ -130,10 +131,11 @@ cudaError_t launch_heads(const void *xt, int Mt, const void *w, float *yt, const
     return mtpv::launch_lm_head(xd, Md, Kd, N, wq, scales, MTPV_W_INT4_G64, yd, at(ws, l.d), s);
 }
 
+// inl (optional): the per-position inputs by value, in place of drafts / ua / us.
 mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *drafts, const float *ua,
                           const float *us, int B, int K, int V, float T, float top_p,
                           int32_t *out_tokens, int32_t *out_acc, int32_t *row_status, void *ws,
-                          cudaStream_t s) {
+                          cudaStream_t s, const mtpv::SamplerInline *inl = nullptr) {
     const VerifyWs l = verify_layout(B, K, V);
     unsigned int *counters = reinterpret_cast<unsigned int *>(at(ws, l.counters));
     mtpv::SamplerParams p;
@@ -154,6 +156,10 @@ mtpv_status launch_verify(const float *tl, const float *dl, const int32_t *draft
     p.slots = reinterpret_cast<mtpv::RowSlot *>(at(ws, l.stats));
     p.counters = counters;
     p.ecache = reinterpret_cast<double *>(at(ws, l.ecache));
+    if (inl) {
+        p.inline_inputs = 1;
+        p.inl = *inl;
+    }
     return cuda_status(mtpv::launch_sampler(p, B * (2 * K + 1), s));
 }
 
@@ -374,16 +380,16 @@ size_t mtpv_verify_step_workspace_bytes(int B, int K, int V, int h) {
     return step_layout(B, K, V, h).total;
 }
 
-mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const void *s_draft,
-                             const void *h_target, const void *h_draft,
-                             const int32_t *draft_tokens, const float *u_accept,
-                             const float *u_sample, int B, int K, int V, int h, float temperature,
-                             float top_p, int32_t *out_tokens, int32_t *out_accepted,
-                             int32_t *row_status, float *target_logits, float *draft_logits,
-                             void *ws, size_t ws_bytes, mtpv_stream stream) {
-    if (!w_target || !w_draft || !s_draft || !h_target || !h_draft || !draft_tokens || !u_accept ||
-        !u_sample || !out_tokens || !out_accepted)
-        return MTPV_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// Arguments of a verify step other than the per-position inputs and outputs.
+mtpv_status step_check(const void *w_target, const void *w_draft, const void *s_draft,
+                       const void *h_target, const void *h_draft, int B, int K, int V, int h,
+                       float temperature, float top_p, const float *target_logits,
+                       const float *draft_logits, const void *ws, size_t ws_bytes) {
+    if (!w_target || !w_draft || !s_draft || !h_target || !h_draft) return MTPV_ERR_INVALID_ARG;
     if (!verify_shape_ok(B, K, V) || B * (K + 1) > 64 || !lm_head_shape_ok(B * (K + 1), h, V) ||
         !sampling_params_ok(temperature, top_p))
         return MTPV_ERR_INVALID_ARG;
@@ -392,16 +398,56 @@ mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const vo
         return MTPV_ERR_INVALID_ARG;
     if ((target_logits && !aligned(target_logits, 4)) || (draft_logits && !aligned(draft_logits, 4)))
         return MTPV_ERR_INVALID_ARG;
+    if (!ws || !aligned(ws, kAlign) || ws_bytes < step_layout(B, K, V, h).total) return MTPV_ERR_WORKSPACE;
+    return MTPV_OK;
+}
+
+// Both heads, then the sampler (arguments checked by step_check).
+mtpv_status step_launch(const void *w_target, const void *w_draft, const void *s_draft,
+                        const void *h_target, const void *h_draft, const int32_t *draft_tokens,
+                        const float *u_accept, const float *u_sample, const mtpv::SamplerInline *inl,
+                        int B, int K, int V, int h, float temperature, float top_p,
+                        int32_t *out_tokens, int32_t *out_accepted, int32_t *row_status,
+                        float *target_logits, float *draft_logits, void *ws, cudaStream_t s) {
     const StepWs l = step_layout(B, K, V, h);
-    if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MTPV_ERR_WORKSPACE;
-    cudaStream_t s = (cudaStream_t)stream;
     float *tl = target_logits ? target_logits : reinterpret_cast<float *>(at(ws, l.tl));
     float *dl = draft_logits ? draft_logits : reinterpret_cast<float *>(at(ws, l.dl));
     const cudaError_t e = launch_heads(h_target, B * (K + 1), w_target, tl, h_draft, B * K, w_draft,
                                        s_draft, dl, h, V, at(ws, l.heads), s);
     if (e != cudaSuccess) return cuda_status(e);
     return launch_verify(tl, dl, draft_tokens, u_accept, u_sample, B, K, V, temperature, top_p,
-                         out_tokens, out_accepted, row_status, at(ws, l.verify), s);
+                         out_tokens, out_accepted, row_status, at(ws, l.verify), s, inl);
+}
+
+// The device address of a page-locked host buffer mapped into this device's
+// address space, else null (pageable memory, or no mapping).
+void *mapped_device_alias(void *host) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, host) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return nullptr;
+    }
+    return a.type == cudaMemoryTypeHost ? a.devicePointer : nullptr;
+}
+
+}  // namespace
+
+extern "C" {
+
+mtpv_status mtpv_verify_step(const void *w_target, const void *w_draft, const void *s_draft,
+                             const void *h_target, const void *h_draft,
+                             const int32_t *draft_tokens, const float *u_accept,
+                             const float *u_sample, int B, int K, int V, int h, float temperature,
+                             float top_p, int32_t *out_tokens, int32_t *out_accepted,
+                             int32_t *row_status, float *target_logits, float *draft_logits,
+                             void *ws, size_t ws_bytes, mtpv_stream stream) {
+    if (!draft_tokens || !u_accept || !u_sample || !out_tokens || !out_accepted) return MTPV_ERR_INVALID_ARG;
+    const mtpv_status st = step_check(w_target, w_draft, s_draft, h_target, h_draft, B, K, V, h, temperature,
+                                      top_p, target_logits, draft_logits, ws, ws_bytes);
+    if (st != MTPV_OK) return st;
+    return step_launch(w_target, w_draft, s_draft, h_target, h_draft, draft_tokens, u_accept, u_sample, nullptr,
+                       B, K, V, h, temperature, top_p, out_tokens, out_accepted, row_status, target_logits,
+                       draft_logits, ws, (cudaStream_t)stream);
 }
 
 size_t mtpv_verify_step_host_workspace_bytes(int B, int K, int V, int h) {
@@ -424,32 +470,41 @@ mtpv_status mtpv_verify_step_host(const void *w_target, const void *w_draft, con
     if (!ws || !aligned(ws, kAlign) || ws_bytes < l.total) return MTPV_ERR_WORKSPACE;
     cudaStream_t s = (cudaStream_t)stream;
     const size_t nt = (size_t)B * (K + 1), nd = (size_t)B * K;
-    struct Copy { void *dst; const void *src; size_t bytes; };
-    const Copy in[] = {
-        {at(ws, l.ht), h_target_host, nt * h * 2},
-        {at(ws, l.hd), h_draft_host, nd * h * 2},
-        {at(ws, l.drafts), draft_tokens_host, nd * sizeof(int32_t)},
-        {at(ws, l.ua), u_accept_host, nd * sizeof(float)},
-        {at(ws, l.us), u_sample_host, nt * sizeof(float)},
-    };
-    for (const Copy &c : in) {
-        cudaError_t e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, s);
-        if (e != cudaSuccess) return cuda_status(e);
+    const mtpv_status chk = step_check(w_target, w_draft, s_draft, at(ws, l.ht), at(ws, l.hd), B, K, V, h,
+                                       temperature, top_p, nullptr, nullptr, at(ws, l.step), l.ht);
+    if (chk != MTPV_OK) return chk;
+    // The hidden states are copied in; drafts and uniforms (a few bytes per
+    // position) travel by value in the sampler's launch parameters instead.
+    cudaError_t e = cudaMemcpyAsync(at(ws, l.ht), h_target_host, nt * h * 2, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess) e = cudaMemcpyAsync(at(ws, l.hd), h_draft_host, nd * h * 2, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return cuda_status(e);
+    mtpv::SamplerInline inl;
+    std::memcpy(inl.drafts, draft_tokens_host, nd * sizeof(int32_t));
+    std::memcpy(inl.u_acc, u_accept_host, nd * sizeof(float));
+    std::memcpy(inl.u_samp, u_sample_host, nt * sizeof(float));
+    // Outputs: written by the kernel straight into the host buffers when all
+    // of them are page-locked and mapped into the device's address space,
+    // else into the workspace and copied back.
+    int32_t *tok = static_cast<int32_t *>(mapped_device_alias(out_tokens_host));
+    int32_t *acc = static_cast<int32_t *>(mapped_device_alias(out_accepted_host));
+    int32_t *rs = row_status_host ? static_cast<int32_t *>(mapped_device_alias(row_status_host)) : nullptr;
+    const bool direct = tok && acc && (!row_status_host || rs);
+    if (!direct) {
+        tok = reinterpret_cast<int32_t *>(at(ws, l.tok));
+        acc = reinterpret_cast<int32_t *>(at(ws, l.acc));
+        rs = reinterpret_cast<int32_t *>(at(ws, l.rs));
     }
-    int32_t *tok = reinterpret_cast<int32_t *>(at(ws, l.tok));
-    int32_t *acc = reinterpret_cast<int32_t *>(at(ws, l.acc));
-    int32_t *rs = reinterpret_cast<int32_t *>(at(ws, l.rs));
-    mtpv_status st = mtpv_verify_step(
-        w_target, w_draft, s_draft, at(ws, l.ht), at(ws, l.hd),
-        reinterpret_cast<const int32_t *>(at(ws, l.drafts)), reinterpret_cast<const float *>(at(ws, l.ua)),
-        reinterpret_cast<const float *>(at(ws, l.us)), B, K, V, h, temperature, top_p, tok, acc, rs,
-        nullptr, nullptr, at(ws, l.step), l.ht, stream);
+    const mtpv_status st = step_launch(w_target, w_draft, s_draft, at(ws, l.ht), at(ws, l.hd), nullptr, nullptr,
+                                       nullptr, &inl, B, K, V, h, temperature, top_p, tok, acc, rs, nullptr,
+                                       nullptr, at(ws, l.step), s);
     if (st != MTPV_OK) return st;
-    cudaError_t e = cudaMemcpyAsync(out_tokens_host, tok, nt * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess)
-        e = cudaMemcpyAsync(out_accepted_host, acc, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
-    if (e == cudaSuccess && row_status_host)
-        e = cudaMemcpyAsync(row_status_host, rs, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    if (!direct) {
+        e = cudaMemcpyAsync(out_tokens_host, tok, nt * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess)
+            e = cudaMemcpyAsync(out_accepted_host, acc, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+        if (e == cudaSuccess && row_status_host)
+            e = cudaMemcpyAsync(row_status_host, rs, (size_t)B * sizeof(int32_t), cudaMemcpyDeviceToHost, s);
+    }
     if (e == cudaSuccess) e = cudaStreamSynchronize(s);
     return cuda_status(e);
 }

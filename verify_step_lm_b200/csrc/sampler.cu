@@ -53,6 +53,7 @@
 #include <math.h>
 
 #include <atomic>
+#include <type_traits>
 #include <mutex>
 
 #include "common.cuh"
@@ -200,10 +201,26 @@ __device__ __forceinline__ double e_of(float l, double m, double invT, const dou
     return exp_neg(__dmul_rn(__dsub_rn((double)l, m), invT), tab);
 }
 
+// Small integers through the fp32 adder instead of the conversion unit (which
+// runs at a fraction of the adder's rate): 2^23 + y rounded to an integer
+// holds that integer in its low mantissa bits, exactly while 0 <= y < 2^22.
+// floor_small(y) == (int)y and rint_small(y) == __float2uint_rn(y) there;
+// small_float(b) == (float)b for 0 <= b < 2^22.
+__device__ __forceinline__ int floor_small(float y) {
+    return (int)(__float_as_uint(__fadd_rd(y, 8388608.0f)) - 0x4b000000u);
+}
+__device__ __forceinline__ unsigned rint_small(float y) {
+    return __float_as_uint(__fadd_rn(y, 8388608.0f)) - 0x4b000000u;
+}
+__device__ __forceinline__ float small_float(int b) {
+    return __fsub_rn(__uint_as_float(0x4b000000u + (unsigned)b), 8388608.0f);
+}
+
 // Level-1 bin of a logit: linear in (m - l) over the row's range; monotone
-// (non-increasing) in l, equal logits share a bin.
+// (non-increasing) in l, equal logits share a bin.  (m - l) inv_w lies in
+// [0, kBins (1 + 2^-22)] for every logit of a finite row.
 __device__ __forceinline__ int bin_of(float l, float m, float inv_w) {
-    return min(kBins - 1, (int)__fmul_rn(__fsub_rn(m, l), inv_w));
+    return min(kBins - 1, max(0, floor_small(__fmul_rn(__fsub_rn(m, l), inv_w))));
 }
 
 __device__ __forceinline__ bool is_kept(const RowStats &st, float l, int j) {
@@ -235,6 +252,33 @@ __device__ double block_sum_d(double v, SamplerSmem &s) {
     double r = s.red_d[0];
     __syncthreads();
     return r;
+}
+
+// block_sum_d of two values at once (each summed exactly as block_sum_d would).
+__device__ void block_sum_d2(double &a, double &b, SamplerSmem &s) {
+    a = warp_sum_d(a);
+    b = warp_sum_d(b);
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    __syncthreads();
+    if (lane == 0) {
+        s.red_d[w] = a;
+        s.warp_tot[w] = b;
+    }
+    __syncthreads();
+    if (w == 0) {
+        double ra = lane < kWarps ? s.red_d[lane] : 0.0;
+        double rb = lane < kWarps ? s.warp_tot[lane] : 0.0;
+        ra = warp_sum_d(ra);
+        rb = warp_sum_d(rb);
+        if (lane == 0) {
+            s.red_d[0] = ra;
+            s.warp_tot[0] = rb;
+        }
+    }
+    __syncthreads();
+    a = s.red_d[0];
+    b = s.warp_tot[0];
+    __syncthreads();
 }
 
 // Programmatic dependent launch: wait until the grids this one depends on
@@ -630,7 +674,7 @@ __device__ int cluster_draw(cg::cluster_group &cluster, SamplerSmem &s, double *
 // ---------------------------------------------------------------------------
 // statistics kernel: one cluster per logits row
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParams p) {
+__global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(const __grid_constant__ SamplerParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SamplerSmem &s = *reinterpret_cast<SamplerSmem *>(smem_raw + kRegionBytes);
     Region rg;
@@ -793,18 +837,22 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
             __syncthreads();
         }
         double zt = 0.0;
-        for (int j0 = v0 + tid; j0 < v1; j0 += kBatch * kThreads) {
-            float lv[kBatch];
-            double ev[kBatch];
+        // NB tokens per thread at a time, loads before exps before the
+        // histogram; full batches first, then the slice's tail in batches of
+        // two, so that no exp is spent past its end
+        auto p2_batch = [&](auto nb, int j0) {
+            constexpr int NB = decltype(nb)::value;
+            float lv[NB];
+            double ev[NB];
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
+            for (int q = 0; q < NB; ++q) {
                 const int j = j0 + q * kThreads;
                 lv[q] = j < v1 ? lval(j) : m;
             }
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) ev[q] = e_of(lv[q], md, invT, s.exp_tab);
+            for (int q = 0; q < NB; ++q) ev[q] = e_of(lv[q], md, invT, s.exp_tab);
 #pragma unroll
-            for (int q = 0; q < kBatch; ++q) {
+            for (int q = 0; q < NB; ++q) {
                 const int j = j0 + q * kThreads;
                 if (j < v1) {
                     zt += ev[q];
@@ -813,15 +861,19 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                         const int b = bin_of(lv[q], m, inv_w);
                         // excess exp(x) - 1 over the lower edge, x in [0, xw] (xw is
                         // small: a third-order series is ample for locating)
-                        const float lo = __fsub_rn(m, __fmul_rn((float)(b + 1), bw));
+                        const float lo = __fsub_rn(m, __fmul_rn(small_float(b + 1), bw));
                         const float x = fminf(xw, fmaxf(0.0f, __fmul_rn(__fsub_rn(lv[q], lo), (float)invT)));
                         const float ex = __fmul_rn(x, __fmaf_rn(x, __fmaf_rn(x, 0.16666667f, 0.5f), 1.0f));
                         atomicAdd(&hcnt[b], 1u);
-                        atomicAdd(&hexc[b], min(qmax, __float2uint_rn(__fmul_rn(ex, qscale))));
+                        atomicAdd(&hexc[b], min(qmax, rint_small(__fmul_rn(ex, qscale))));
                     }
                 }
             }
-        }
+        };
+        int j0 = v0 + tid;
+        for (; j0 + (kBatch - 1) * kThreads < v1; j0 += kBatch * kThreads)
+            p2_batch(std::integral_constant<int, kBatch>{}, j0);
+        for (; j0 < v1; j0 += 2 * kThreads) p2_batch(std::integral_constant<int, 2>{}, j0);
         const double zc = block_sum_d(zt, s);  // its barriers also complete the histogram
         // publish Z, and send every CTA the part of this CTA's histogram that
         // it owns (bins [r per, (r + 1) per) to CTA r, slot rank): warp r
@@ -945,8 +997,8 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                         }
                     }
                 }
-                const double a_cta = block_sum_d(a_loc, s);  // also completes the staging
-                const double m_cta = block_sum_d(m_loc, s);
+                double a_cta = a_loc, m_cta = m_loc;
+                block_sum_d2(a_cta, m_cta, s);  // also completes the staging
                 if (wid == 0) {
                     publish(cluster, s.all_part, rank, C, a_cta);
                     publish(cluster, s.all_M, rank, C, m_cta);
@@ -978,22 +1030,38 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
                     // and its exp in descending order; a block scan of the
                     // sorted exps gives every candidate its preceding mass
                     const int n = (int)total;
-                    const unsigned long long key = tid < n ? rg.cand[tid] : 0ull;
+                    // with few candidates, `parts` threads share one: thread
+                    // part * S + i counts the keys above candidate i in the
+                    // part-th run of the list (runs of even length, so the
+                    // 16-byte loads stay aligned); the counts are added below
+                    const int parts = n <= kThreads / 4 ? 4 : n <= kThreads / 2 ? 2 : 1;
+                    const int S = kThreads / parts, ci = tid % S, part = tid / S;
+                    const int L = (((n + parts - 1) / parts) + 1) & ~1;
+                    const int k0 = min(n, part * L), k1 = min(n, k0 + L);
+                    const unsigned long long key = ci < n ? rg.cand[ci] : 0ull;
                     int r = 0;
-                    if (tid < n) {
-                        // 16-byte loads, four independent counts: the loop is
-                        // bound by shared-memory latency, not by the compares
+                    if (ci < n) {
+                        // 16-byte loads, four in flight, four independent
+                        // counts: the loop is bound by shared-memory latency
                         const ulonglong2 *c2 = reinterpret_cast<const ulonglong2 *>(rg.cand);
-                        int r0 = 0, r1 = 0, r2 = 0, r3 = 0, j = 0;
-                        for (; j + 4 <= n; j += 4) {
+                        int r0 = 0, r1 = 0, r2 = 0, r3 = 0, j = k0;
+                        for (; j + 8 <= k1; j += 8) {
                             const ulonglong2 a = c2[j >> 1], b = c2[(j >> 1) + 1];
-                            r0 += a.x > key ? 1 : 0;
-                            r1 += a.y > key ? 1 : 0;
-                            r2 += b.x > key ? 1 : 0;
-                            r3 += b.y > key ? 1 : 0;
+                            const ulonglong2 c = c2[(j >> 1) + 2], d = c2[(j >> 1) + 3];
+                            r0 += (a.x > key ? 1 : 0) + (c.x > key ? 1 : 0);
+                            r1 += (a.y > key ? 1 : 0) + (c.y > key ? 1 : 0);
+                            r2 += (b.x > key ? 1 : 0) + (d.x > key ? 1 : 0);
+                            r3 += (b.y > key ? 1 : 0) + (d.y > key ? 1 : 0);
                         }
-                        for (; j < n; ++j) r0 += rg.cand[j] > key ? 1 : 0;
+                        for (; j < k1; ++j) r0 += rg.cand[j] > key ? 1 : 0;
                         r = (r0 + r1) + (r2 + r3);
+                    }
+                    if (parts > 1) {
+                        int *rp = reinterpret_cast<int *>(s.thr_excl);
+                        rp[tid] = r;
+                        __syncthreads();
+                        if (part == 0)
+                            for (int q = 1; q < parts; ++q) r += rp[q * S + ci];
                     }
                     const double e = tid < n ? e_of(key_logit(key), md, invT, s.exp_tab) : 0.0;
                     __syncthreads();
@@ -1192,7 +1260,18 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(SamplerParam
 // ---------------------------------------------------------------------------
 // draw kernel: one cluster per draft position (verify) or per row (sample)
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams p) {
+// A verify call's per-position inputs, from the launch parameters or from memory.
+__device__ __forceinline__ int32_t draft_at(const SamplerParams &p, size_t k) {
+    return p.inline_inputs ? p.inl.drafts[k] : p.drafts[k];
+}
+__device__ __forceinline__ float u_acc_at(const SamplerParams &p, size_t k) {
+    return p.inline_inputs ? p.inl.u_acc[k] : p.u_acc[k];
+}
+__device__ __forceinline__ float u_samp_at(const SamplerParams &p, size_t k) {
+    return p.inline_inputs ? p.inl.u_samp[k] : p.u_samp[k];
+}
+
+__global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(const __grid_constant__ SamplerParams p) {
     extern __shared__ __align__(16) unsigned char smem_raw[];
     SamplerSmem &s = *reinterpret_cast<SamplerSmem *>(smem_raw + kDrawBufBytes);
     double *wbuf = reinterpret_cast<double *>(smem_raw);
@@ -1233,7 +1312,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
     int status = p.slots[rt].st.status;
     int d = 0;
     if (residual) {
-        d = p.drafts[(size_t)b * K + i];
+        d = draft_at(p, (size_t)b * K + i);
         const int sd = p.slots[rd].st.status;
         if (d < 0 || d >= V) status = MTPV_ROW_BAD_DRAFT;
         else if (sd != MTPV_ROW_OK && status == MTPV_ROW_OK) status = sd;
@@ -1254,7 +1333,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
             qd = warped_prob(st_d, Ld, d, T, invT, s.exp_tab);
         }
         const double ratio = (qd == 0.0) ? (pt > 0.0 ? INFINITY : 0.0) : pt / qd;
-        s.res_acc = (double)p.u_acc[(size_t)b * K + i] < ratio ? 1 : 0;
+        s.res_acc = (double)u_acc_at(p, (size_t)b * K + i) < ratio ? 1 : 0;
     }
 
     // ---------------- this position's residual / bonus draw ----------------
@@ -1274,7 +1353,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
         src.tab = s.exp_tab;
         src.rho = residual ? st_t.Zk / st_d.Zk : 1.0;
         src.kind = residual ? 1 : 0;
-        const float u = p.verify ? p.u_samp[(size_t)b * (K + 1) + i] : p.u_samp[c];
+        const float u = p.verify ? u_samp_at(p, (size_t)b * (K + 1) + i) : p.u_samp[c];
         drew = cluster_draw(cluster, s, wbuf, src, residual, invT, u, v0, v1, x_dst, p.wait_polls);
     }
     if (drew == kDrawTimeout) status = MTPV_ROW_TIMEOUT;
@@ -1317,7 +1396,7 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_draw_kernel(SamplerParams
         for (int k = 0; k <= K; ++k) ot[k] = -1;
         p.out_acc[b] = -1;
     } else {
-        for (int k = 0; k < n; ++k) ot[k] = p.drafts[(size_t)b * K + k];
+        for (int k = 0; k < n; ++k) ot[k] = draft_at(p, (size_t)b * K + k);
         ot[n] = __ldcg(&p.slots[b * S + n].rec.x);
         for (int k = n + 1; k <= K; ++k) ot[k] = -1;
         p.out_acc[b] = n;

@@ -34,6 +34,16 @@ union RowSlot {
     PosRecord rec;
 };
 
+// A verify call's per-position inputs carried by value in the launch
+// parameters, so that a call whose inputs start in host memory needs no copy
+// for them: at most kInlinePositions positions (B (K + 1)).
+constexpr int kInlinePositions = 64;
+struct SamplerInline {
+    int32_t drafts[kInlinePositions];  // [B, K]
+    float u_acc[kInlinePositions];     // [B, K]
+    float u_samp[kInlinePositions];    // [B, K+1]
+};
+
 struct SamplerParams {
     const float *tl;        // verify: target logits [B, K+1, V]; sample: logits [R, V]
     const float *dl;        // verify: draft logits [B, K, V]
@@ -50,6 +60,8 @@ struct SamplerParams {
     unsigned int *counters;  // verify: [B]; zeroed by the statistics kernel
     double *ecache;       // [rows][V]: exp((l_j - m)/T) of kept tokens, 0 elsewhere (T > 0), or null
     int wait_polls;       // polls of a bounded device-side wait before it gives up (set by launch_sampler)
+    int inline_inputs = 0;  // verify: drafts / u_acc / u_samp are read from inl instead
+    SamplerInline inl;
 };
 
 // Process-wide bound of the sampler's device-side waits, in polls (< 0: the
