@@ -77,17 +77,18 @@ def load() -> ctypes.CDLL:
 
 
 def _ptr(t):
+    # a plain int (or None for NULL): ctypes converts it for a c_void_p argument
     if t is None:
         return None
     if isinstance(t, torch.Tensor):
-        return ctypes.c_void_p(t.data_ptr())
-    return ctypes.c_void_p(int(t))
+        return t.data_ptr()
+    return int(t)
 
 
 def _stream(stream=None):
     if stream is None:
         stream = torch.cuda.current_stream()
-    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+    return stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
 
 
 def _check(fn: str, st: int):
