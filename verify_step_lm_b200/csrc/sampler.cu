@@ -32,7 +32,10 @@
 //       more than kCandCap tokens (massive ties, degenerate ranges) falls back
 //       to an 8-pass weighted radix select on the same key.
 //   out the row's statistics, and (workspace permitting) the row's weights
-//       e_j of kept tokens, 0 elsewhere: p'_j = e_j / Z' with no further test
+//       e_j of kept tokens, 0 elsewhere: p'_j = e_j / Z' with no further test.
+//       When the located bin holds the cut, the other CTAs store the weights
+//       masked by bin while CTA 0 computes the cut; CTA 0 then zeroes its
+//       candidates past the cut.
 // Draw kernel, one cluster per draft position i of a sequence (sampling: per
 // row).  The acceptance test of d_i reads two weights; the cluster then draws
 // position i's residual token (the bonus at i == K) with u_samp[i], as if the
@@ -118,6 +121,7 @@ struct SamplerSmem {
     // derived by every CTA for itself
     double draw_total, cut_Zk;
     int wstar, x_found, first_fail, cut_idx;
+    int cut_pos, cut_n;  // statistics kernel, CTA 0: the cut's place among the sorted candidates, their number
     float cut_l;
     int res_acc;  // draw kernel, CTA 0: the position's acceptance
     unsigned long long bar;  // mbarrier of the bulk copies
@@ -392,6 +396,10 @@ __device__ __forceinline__ double ordered_sum(const double *vals, int C, int wan
     if (excl) *excl = ex;
     return acc;
 }
+
+// The two halves of a cluster barrier (every thread of every CTA arrives once).
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
 
 // Write v into slot `rank` of arr in every CTA of the cluster: lanes 0..C-1
 // of the calling warp each store to one CTA (v uniform over the warp).
@@ -1079,15 +1087,12 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(const __grid
                     if (cut < 0) cut = 0;  // A < thr by construction: the first is kept
                     if (tid == cut) {
                         s.cut_Zk = __dadd_rn(A, incl);
+                        s.cut_pos = cut;
                         s.cut_idx = key_index(rg.cand[cut]);
                         s.cut_l = key_logit(rg.cand[cut]);
                     }
                     __syncthreads();
-                    if (wid == 0 && lane < C) {  // the cut, into every CTA of the cluster
-                        *cluster.map_shared_rank(&s.cut_Zk, lane) = s.cut_Zk;
-                        *cluster.map_shared_rank(&s.cut_idx, lane) = s.cut_idx;
-                        *cluster.map_shared_rank(&s.cut_l, lane) = s.cut_l;
-                    }
+                    if (tid == 0) s.cut_n = n;
                 } else if (rank == 0) {
                     // more candidates than threads: shared-memory bitonic sort
                     const int n = min((int)s.cand_count, kCandCap);
@@ -1150,20 +1155,52 @@ __global__ void __launch_bounds__(kThreads, 1) sampler_stats_kernel(const __grid
                         double ex = s.thr_excl[tid];
                         for (int i = i0; i < cut; ++i) ex = __dadd_rn(ex, rg.cand_e[i]);
                         s.cut_Zk = __dadd_rn(A, __dadd_rn(ex, rg.cand_e[cut]));
+                        s.cut_pos = cut;
                         s.cut_idx = key_index(rg.cand[cut]);
                         s.cut_l = key_logit(rg.cand[cut]);
                     }
                     __syncthreads();
-                    if (wid == 0 && lane < C) {  // the cut, into every CTA of the cluster
-                        *cluster.map_shared_rank(&s.cut_Zk, lane) = s.cut_Zk;
-                        *cluster.map_shared_rank(&s.cut_idx, lane) = s.cut_idx;
-                        *cluster.map_shared_rank(&s.cut_l, lane) = s.cut_l;
+                    if (tid == 0) s.cut_n = n;
+                }
+                // Only CTA 0 needs the cut.  Meanwhile the weights go out
+                // masked by bin (above the located bin kept, below it not, in
+                // it kept for now): every other CTA stores its own slice and a
+                // share of CTA 0's (read from CTA 0's shared memory, which the
+                // cut does not touch), arrives on a cluster barrier and leaves.
+                // CTA 0 waits there (the peers' stores and reads are done),
+                // zeroes its candidates past the cut and writes the statistics.
+                // (with a weight cache every slice fits shared memory with its
+                // exps: the launch drops the cache otherwise, so the test is the
+                // same in every CTA)
+                const bool store = erow && slice <= kCacheFloats;
+                if (store) {
+                    auto store_masked = [&](const float *lc, const double *ec, int jb, int i0, int i1) {
+                        for (int i = i0 + tid; i < i1; i += kThreads)
+                            erow[jb + i] = bin_of(lc[i], m, inv_w) <= bstar ? ec[i] : 0.0;
+                    };
+                    const int n0 = min(V, slice);  // CTA 0's slice: [0, n0)
+                    if (rank != 0) {
+                        store_masked(rg.cache, rg.ecache, v0, 0, v1 - v0);
+                        const int q = (((n0 + C - 2) / (C - 1)) + 31) & ~31;
+                        store_masked(cluster.map_shared_rank(rg.cache, 0), cluster.map_shared_rank(rg.ecache, 0), 0,
+                                     min(n0, (rank - 1) * q), min(n0, rank * q));
+                    } else if (C == 1) {
+                        store_masked(rg.cache, rg.ecache, v0, 0, v1 - v0);
                     }
                 }
-                cluster.sync();
+                cluster_arrive();
+                if (rank != 0) return;
+                cluster_wait();
+                if (store) {
+                    // candidates past the cut are not kept
+                    for (int i = s.cut_pos + 1 + tid; i < s.cut_n; i += kThreads)
+                        erow[key_index(rg.cand[i])] = 0.0;
+                }
                 st.Zk = s.cut_Zk;
                 st.idxstar = s.cut_idx;
                 st.lstar = s.cut_l;
+                if (tid == 0) p.slots[row].st = st;
+                return;
             } else {
                 // weighted radix select on the 64-bit key, 8 bits per pass
                 unsigned long long prefix = 0ull, mask = 0ull;
