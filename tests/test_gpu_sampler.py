@@ -114,6 +114,33 @@ def test_ties_on_a_coarse_logit_grid():
         check_parity(*make_case(64, 3, 4096, seed=710 + seed, T=0.0, grid=0.25), 0.0, TOPP_PAGES)
 
 
+def crossing_bin_size(row, T, top_p):
+    """Tokens in the level-1 bin where the descending mass reaches top_p Z
+    (2048 bins linear in (m - l) over the row's range, fp32 as the kernel
+    bins them; masses exact here)."""
+    L = np.asarray(row, dtype=np.float32)
+    m, mn = L.max(), L.min()
+    inv_w = np.float32(2048) / np.float32(m - mn)
+    b = np.minimum(2047, np.floor((m - L) * inv_w)).astype(np.int64)
+    e = np.exp((L.astype(np.float64) - float(m)) / T)
+    mass = np.bincount(b, weights=e, minlength=2048)
+    c = np.cumsum(mass)
+    return int(np.bincount(b, minlength=2048)[min(2047, int(np.searchsorted(c, top_p * c[-1])))])
+
+
+def test_crossing_bins_sorted_by_the_bitonic_network():
+    # logits on a 0.5 grid over 30000 tokens: the crossing logit value is
+    # shared by hundreds to thousands of tokens, more than one thread each
+    # (512) and within the candidate buffer (4096), so CTA 0 sorts them with
+    # its bitonic network before the exact cut
+    B, K, V = 8, 3, 30000
+    tl, dl, d, u = make_case(B, K, V, seed=930, grid=0.5)
+    rows = list(tl.reshape(-1, V).numpy()) + list(dl.reshape(-1, V).numpy())
+    sizes = [crossing_bin_size(r, T_PAGES, TOPP_PAGES) for r in rows]
+    assert any(512 < n <= 4096 for n in sizes), sizes
+    check_parity(tl, dl, d, u, T_PAGES, TOPP_PAGES)
+
+
 def test_degenerate_rows_take_the_radix_path():
     # all-equal rows and a two-level row: the crossing bin holds far more
     # tokens than the candidate buffer, so the cut comes from the radix select
