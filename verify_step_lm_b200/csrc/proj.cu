@@ -71,6 +71,8 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
     const long long grid = gridDim.x;
     const long long s0 = (long long)blockIdx.x * a.T / grid;
     const long long s1 = (long long)(blockIdx.x + 1) * a.T / grid;
+    // a dependent launch may be scheduled onto SMs as this grid's CTAs leave
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
     if (threadIdx.x == 0) {
         for (int i = 0; i < a.stages; ++i) {
@@ -89,19 +91,11 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
         const bool two_chunks = ((2 * Gt) & 15) != 0;  // a row's 8 scales straddle 16-byte chunks
         const uint32_t tx = pj::kWBytes + pj::kG * a.M * 128;
         const uint32_t abort32 = su32(&c.abort);
-        int slot = 0;
-        uint32_t phase = 0;
-        long long issued = 0;
-        int X = (int)(s0 / a.spt), ch = (int)(s0 - (long long)X * a.spt);
-        for (long long s = s0; s < s1; ++s) {
-            const bool ok = __all_sync(0xffffffffu, pj::bar_wait_or_abort(&c.empty[slot], phase ^ 1, abort32));
-            if (!ok) {
-                if (lane == 0) {
-                    atomicOr(a.err, 1u);
-                    *(volatile int *)&c.abort = 1;
-                }
-                break;
-            }
+        // stage s into ring slot `slot`: its weights (nibbles by TMA, scales by
+        // cp.async into a 32-byte slot per row: the aligned 16-byte chunk(s)
+        // holding groups 8 ch .. 8 ch + 7), and its activations (TMA)
+        auto issue_weights = [&](long long s, int slot) {
+            const int X = (int)(s / a.spt), ch = (int)(s - (long long)X * a.spt);
             unsigned char *st = ring + (size_t)slot * kNarrowStage;
             if (lane == 0) {
                 bar_arrive_expect(&c.full[slot], tx);
@@ -115,11 +109,7 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
                         tma_load_2d(st + p * 16384, &tmW, xc, X * pj::kTileRows, &c.full[slot]);
                     }
                 }
-#pragma unroll
-                for (int jj = 0; jj < pj::kG; ++jj)
-                    tma_load_2d(st + pj::kWBytes + jj * kNarrowXBox, &tmX, (ch * pj::kG + jj) * 64, 0, &c.full[slot]);
             }
-            // scales of tile rows lane + 32 i: the aligned 16-byte chunk(s) holding groups 8 ch .. 8 ch + 7
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 const int r = lane + 32 * i;
@@ -132,14 +122,41 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
                 if (two_chunks) pj::cp_async16(dst + 16, a.s, al + 16, sbytes);
             }
             pj::cp_async_arrive(&c.full[slot]);
+        };
+        auto issue_acts = [&](long long s, int slot) {
+            if (lane == 0) {
+                const int ch = (int)(s % a.spt);
+                unsigned char *st = ring + (size_t)slot * kNarrowStage;
+#pragma unroll
+                for (int jj = 0; jj < pj::kG; ++jj)
+                    tma_load_2d(st + pj::kWBytes + jj * kNarrowXBox, &tmX, (ch * pj::kG + jj) * 64, 0, &c.full[slot]);
+            }
+        };
+        // The ring's first stages: weights and scales before waiting for the
+        // grid before this one on the stream (nothing on the stream writes
+        // them), the activations once that grid has completed.
+        const long long fill = std::min<long long>(a.stages, s1 - s0);
+        for (long long k = 0; k < fill; ++k) issue_weights(s0 + k, (int)k);
+        asm volatile("griddepcontrol.wait;" ::: "memory");
+        for (long long k = 0; k < fill; ++k) issue_acts(s0 + k, (int)k);
+        long long issued = fill;
+        int slot = (int)(fill % a.stages);
+        uint32_t phase = fill == a.stages ? 1u : 0u;
+        for (long long s = s0 + fill; s < s1; ++s) {
+            const bool ok = __all_sync(0xffffffffu, pj::bar_wait_or_abort(&c.empty[slot], phase ^ 1, abort32));
+            if (!ok) {
+                if (lane == 0) {
+                    atomicOr(a.err, 1u);
+                    *(volatile int *)&c.abort = 1;
+                }
+                break;
+            }
+            issue_weights(s, slot);
+            issue_acts(s, slot);
             ++issued;
             if (++slot == a.stages) {
                 slot = 0;
                 phase ^= 1;
-            }
-            if (++ch == a.spt) {
-                ch = 0;
-                ++X;
             }
         }
         // the copies still in flight land before the CTA may exit
@@ -151,6 +168,9 @@ __global__ void __launch_bounds__(kNarrowThreads, 1)
     }
 
     // ---------------- consumers ----------------
+    // (the workspace and y are touched only after the grid before this one
+    // on the stream has completed)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int g = lane >> 2, t = lane & 3;
     const int j = warp & 7, hb = warp >> 3;  // group of the stage; MMA tiles 4 hb .. 4 hb + 3
     const int xr = pj::act_row(g);  // the activation row behind this lane's MMA column
@@ -403,11 +423,20 @@ cudaError_t launch_int4_proj(const void *x, int M, int Kd, int N, const void *wq
             if (e != cudaSuccess) return e;
             a.stages = stages;
             const int grid = (int)std::max(1LL, std::min<long long>(a.T, std::min(sms, psms)));
-            if (silu_mul)
-                int4_proj_narrow_kernel<true><<<grid, kNarrowThreads, smem, s>>>(tmW, tmX, a);
-            else
-                int4_proj_narrow_kernel<false><<<grid, kNarrowThreads, smem, s>>>(tmW, tmX, a);
-            e = cudaGetLastError();
+            // a programmatic dependent of the grid before it on the stream:
+            // its CTAs start streaming weights as that grid's CTAs leave
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(grid, 1, 1);
+            cfg.blockDim = dim3(kNarrowThreads, 1, 1);
+            cfg.dynamicSmemBytes = smem;
+            cfg.stream = s;
+            cudaLaunchAttribute at[1];
+            at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+            at[0].val.programmaticStreamSerializationAllowed = 1;
+            cfg.attrs = at;
+            cfg.numAttrs = 1;
+            e = silu_mul ? cudaLaunchKernelEx(&cfg, int4_proj_narrow_kernel<true>, tmW, tmX, a)
+                         : cudaLaunchKernelEx(&cfg, int4_proj_narrow_kernel<false>, tmW, tmX, a);
         }
         if (e != cudaSuccess) return e;
     }
