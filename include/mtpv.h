@@ -237,6 +237,12 @@ MTPV_API mtpv_status mtpv_lm_head_pair(const void *xt, int Mt, const void *w, fl
  * gave up ORs a nonzero code into it and that launch's outputs are not
  * valid; it stays set until the caller clears it.  Errors:
  * MTPV_ERR_INVALID_ARG, MTPV_ERR_WORKSPACE, MTPV_ERR_CUDA.
+ * Launch: a pass of up to 8 rows is a programmatic dependent launch (it may
+ * start while the kernel before it on the stream finishes, so that
+ * back-to-back projections overlap one's start with the other's tail).  It
+ * reads x, ws and y only after that kernel has completed, but it may read
+ * wq and scales earlier: a preceding kernel that allows its dependents to
+ * launch early (griddepcontrol.launch_dependents) must not write them.
  * ---------------------------------------------------------------------- */
 MTPV_API size_t mtpv_int4_proj_workspace_bytes(int M, int Kd, int N);
 MTPV_API mtpv_status mtpv_int4_proj(const void *x, int M, int Kd, int N, const void *wq,
