@@ -478,6 +478,8 @@ mtpv_status mtpv_verify_step_host(const void *w_target, const void *w_draft, con
     cudaError_t e = cudaMemcpyAsync(at(ws, l.ht), h_target_host, nt * h * 2, cudaMemcpyHostToDevice, s);
     if (e == cudaSuccess) e = cudaMemcpyAsync(at(ws, l.hd), h_draft_host, nd * h * 2, cudaMemcpyHostToDevice, s);
     if (e != cudaSuccess) return cuda_status(e);
+    // (mtpv_verify_step's limit B (K + 1) <= 64, checked by step_check, fits the block)
+    static_assert(mtpv::kInlinePositions >= 64, "per-position inputs of a verify step by value");
     mtpv::SamplerInline inl;
     std::memcpy(inl.drafts, draft_tokens_host, nd * sizeof(int32_t));
     std::memcpy(inl.u_acc, u_accept_host, nd * sizeof(float));
