@@ -125,7 +125,7 @@ struct SamplerSmem {
     float cut_l;
     int res_acc;  // draw kernel, CTA 0: the position's acceptance
     unsigned long long bar;  // mbarrier of the bulk copies
-    int wait_ok;             // thread 0's verdict on a bulk copy, for the block
+    int wait_ok;             // thread 0's outcome of a bulk-copy wait, for the block
     double exp_tab[kExpTab];  // 2^(j/64), for exp_neg
 };
 
